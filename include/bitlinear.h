@@ -1,0 +1,161 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so, the B200 (sm_100a) ternary BitLinear
+ * mixed-precision matmul (BitNet b1.58, I2_S-style "int2 with scale").
+ *
+ * The path, per linear layer with latent weights W[M,K] (row-major, torch
+ * nn.Linear [out_features, in_features]) and activations x[N,K]:
+ *
+ *   offline   alpha = mean|W| (fp32, exact sum, rounded once),
+ *             c = clamp(round_half_even(W/alpha), -1, 1), packed 2 bits/weight
+ *   per step  amax_n = max_k|x[n,k]|, q = clamp(round_half_even(x * (127/amax_n)))
+ *             acc[n,m] = sum_k c[m,k] q[n,k]   (int32)
+ *             y[n,m]   = (float)acc * (alpha * (amax_n / 127))
+ *
+ * Sources: "Bitnet.cpp: Efficient Edge Inference for Ternary LLMs" reading
+ * notes -- section 1.1 (weights in {-1,0,1}), section 2.3 (I2_S: ternary
+ * weights with a scale, int8 activations, 2.0 bits per weight, lossless),
+ * section 4.1 (MAD-based int8 multiply-add; lossless-inference conditions);
+ * FairyFuse article, "fused kernel design" (unpack and accumulate in one pass
+ * over bit-packed codes, no intermediate writes).
+ *
+ * Packed weight layout ("I2_S-style", defined by this library):
+ *   row m occupies K/16 little-endian uint32 words (K/4 bytes), rows contiguous;
+ *   weight k lives in word k/16 at bit 8*(k%4) + 2*((k%16)/4);
+ *   the 2-bit field holds c+1 (0 -> -1, 1 -> 0, 2 -> +1); 3 is never written.
+ *   So (word >> 2j) & 0x03030303 gives, one per byte, the fields of weights
+ *   16*(k/16)+4j .. +3 in k order.
+ *
+ * Conventions for every entry point:
+ *   - Ownership: the caller owns every buffer.  The library allocates no
+ *     device or host memory and keeps no per-call state.
+ *   - Pointers are DEVICE pointers unless stated otherwise, 16-byte aligned.
+ *   - Shapes: K must be a positive multiple of 128 and at most 131072; M >= 1
+ *     (a multiple of 128 for bitlinear_gemm); M*K <= 2^40.  N = 0 is a no-op.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default
+ *     stream).  Argument errors are returned synchronously before anything is
+ *     launched; a failed launch returns BITLINEAR_ERR_CUDA.
+ *   - Activations q are int8 [N,K] row-major; outputs y are fp32 [N,M]
+ *     row-major (token-major); the optional acc is int32 [N,M].
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define BITLINEAR_API __attribute__((visibility("default")))
+#else
+#define BITLINEAR_API
+#endif
+
+/* ABI-identical to cudaStream_t. */
+typedef struct CUstream_st* bitlinear_stream_t;
+
+typedef enum {
+    BITLINEAR_OK = 0,
+    BITLINEAR_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size */
+    BITLINEAR_ERR_UNSUPPORTED_SHAPE = 2, /* K % 128, M % 128 (GEMM), N range, size limits */
+    BITLINEAR_ERR_MISALIGNED = 3,        /* pointer not 16-byte aligned */
+    BITLINEAR_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than required */
+    BITLINEAR_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+    BITLINEAR_ERR_DEVICE_TIMEOUT = 6     /* a kernel gave up a bounded wait */
+} bitlinear_status;
+
+/* Static, human-readable name of a status code.  Never NULL. */
+BITLINEAR_API const char* bitlinear_status_string(int status);
+
+/* Library ABI version (major*100 + minor). */
+BITLINEAR_API int bitlinear_version(void);
+
+/* ---------------------------------------------------------------- weights */
+
+/* Bytes of device workspace bitlinear_pack_weights needs (exponent bins and a
+ * flag word); the contents need not be initialised. */
+BITLINEAR_API size_t bitlinear_pack_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * Absmean-ternarise and pack one weight tensor (reading notes section 1.1 and
+ * 2.3; scale rule as in BitNet b1.58, alpha = mean|W|).
+ *   W        fp32 [M,K] latent weights (device, read only)
+ *   packed   uint32 [M, K/16] output in the layout above (M*K/4 bytes)
+ *   alpha    fp32 [1] output: mean|W| rounded to nearest-even once, from an
+ *            exact, order-independent sum; 0 when W is all zero (every code 0)
+ *   workspace, workspace_bytes: scratch of bitlinear_pack_workspace_bytes()
+ * If W holds inf or NaN, *alpha is written as NaN and every code is 0.
+ * Tie rule: |W/alpha| == 0.5 exactly gives code 0 (round half to even).
+ */
+BITLINEAR_API bitlinear_status bitlinear_pack_weights(const float* W, int64_t M, int64_t K,
+                                        uint32_t* packed, float* alpha,
+                                        void* workspace, size_t workspace_bytes,
+                                        bitlinear_stream_t stream);
+
+/* ------------------------------------------------------------ activations */
+
+/*
+ * Per-token absmax int8 quantisation (reading notes section 2.3: int8
+ * activations; one scale per token row).
+ *   x     fp32 [N,K] (device, read only)
+ *   xq    int8 [N,K] output: clamp(round_half_even(x * (127/amax)), -128, 127)
+ *   amax  fp32 [N] output: max_k |x[n,k]| (exact)
+ *   xsum  int32 [N] output sum_k xq[n,k], or NULL to skip it
+ * A token with amax == 0 gets xq = 0.  If 127/amax overflows to inf, +-inf
+ * products clamp to 127/-128 and 0*inf is taken as 0.
+ */
+BITLINEAR_API bitlinear_status bitlinear_quant_act(const float* x, int64_t N, int64_t K,
+                                     int8_t* xq, float* amax, int32_t* xsum,
+                                     bitlinear_stream_t stream);
+
+/* ----------------------------------------------------------------- matmul */
+
+/*
+ * Decode GEMV, 1 <= N <= 16 tokens, on the CUDA cores: streams the packed
+ * weights once, accumulates the ternary x int8 products in int32 and fuses
+ * the rescale (reading notes section 4.1 "MAD-based"; FairyFuse "fused kernel
+ * design").
+ *   packed, alpha   from bitlinear_pack_weights (alpha is a device pointer)
+ *   xq, amax, xsum  from bitlinear_quant_act (xsum is required here)
+ *   y    fp32 [N,M] output: (float)acc * (alpha * (amax[n]/127))
+ *   acc  int32 [N,M] output of the raw accumulators, or NULL
+ * N > 16 returns BITLINEAR_ERR_UNSUPPORTED_SHAPE.
+ */
+BITLINEAR_API bitlinear_status bitlinear_gemv(const uint32_t* packed, const float* alpha,
+                                int64_t M, int64_t K,
+                                const int8_t* xq, const float* amax, const int32_t* xsum,
+                                int64_t N, float* y, int32_t* acc,
+                                bitlinear_stream_t stream);
+
+/*
+ * Prefill GEMM, any N >= 1, on the int8 tensor cores (tcgen05.mma kind::i8,
+ * accumulators in tensor memory): packed weight tiles are brought in by TMA,
+ * expanded to int8 in shared memory and multiplied with TMA-loaded int8
+ * activation tiles; the rescale is fused into the epilogue.  Same arguments
+ * and results as bitlinear_gemv; M must be a multiple of 128.
+ * The reading notes (section 4.4) name prefill, where the work turns
+ * compute-bound, as the stage their CPU kernels leave unoptimised.
+ */
+BITLINEAR_API bitlinear_status bitlinear_gemm(const uint32_t* packed, const float* alpha,
+                                int64_t M, int64_t K,
+                                const int8_t* xq, const float* amax, const int32_t* xsum,
+                                int64_t N, float* y, int32_t* acc,
+                                bitlinear_stream_t stream);
+
+/* ------------------------------------------------------------ diagnostics */
+
+/*
+ * Read (and, if clear != 0, reset) the device-side error word that kernels set
+ * when a bounded wait gives up.  Synchronises the device.  *status_out is
+ * BITLINEAR_OK or BITLINEAR_ERR_DEVICE_TIMEOUT; the return value reports
+ * whether the read itself worked.
+ */
+BITLINEAR_API bitlinear_status bitlinear_device_error(int* status_out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -1,0 +1,120 @@
+"""ctypes view of libbitlinear.so: one Python function per C entry point.
+
+Argument marshalling only -- every step of the path runs in the CUDA kernels
+behind include/bitlinear.h.  There is no CPU fallback: if the shared library
+is missing or a call fails, an exception is raised.
+"""
+import ctypes
+import os
+import re
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libbitlinear.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "bitlinear.h")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED_SHAPE = 2
+ERR_MISALIGNED = 3
+ERR_WORKSPACE = 4
+ERR_CUDA = 5
+ERR_DEVICE_TIMEOUT = 6
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (where, status_string(status), status))
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the shared library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError("libbitlinear.so not built at %s; run "
+                          "`python -m ternary_weight_bit_bitlinear_b200.build`" % path)
+    L = ctypes.CDLL(path)
+    i64, p, st, sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.bitlinear_status_string.argtypes = [ctypes.c_int]
+    L.bitlinear_status_string.restype = ctypes.c_char_p
+    L.bitlinear_version.argtypes = []
+    L.bitlinear_version.restype = ctypes.c_int
+    L.bitlinear_pack_workspace_bytes.argtypes = [i64, i64]
+    L.bitlinear_pack_workspace_bytes.restype = sz
+    L.bitlinear_pack_weights.argtypes = [p, i64, i64, p, p, p, sz, p]
+    L.bitlinear_pack_weights.restype = st
+    L.bitlinear_quant_act.argtypes = [p, i64, i64, p, p, p, p]
+    L.bitlinear_quant_act.restype = st
+    for name in ("bitlinear_gemv", "bitlinear_gemm"):
+        f = getattr(L, name)
+        f.argtypes = [p, p, i64, i64, p, p, p, i64, p, p, p]
+        f.restype = st
+    L.bitlinear_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+    L.bitlinear_device_error.restype = st
+    _lib = L
+    return L
+
+
+def header_symbols(header: str = HEADER):
+    """Names of the functions include/bitlinear.h declares."""
+    text = open(header).read()
+    return sorted(set(re.findall(r"BITLINEAR_API\s+[\w\s\*]+?\b(bitlinear_\w+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return load().bitlinear_status_string(int(status)).decode()
+
+
+def check(status: int, where: str):
+    if status != OK:
+        raise BitLinearError(status, where)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+# --------------------------------------------------------------- raw entry points
+# Each takes torch tensors (already allocated, on the current CUDA device) and
+# returns the C status code unchanged.
+
+def bitlinear_pack_weights(W, M, K, packed, alpha, workspace, workspace_bytes, stream=None):
+    return load().bitlinear_pack_weights(_p(W), M, K, _p(packed), _p(alpha), _p(workspace),
+                                         workspace_bytes, _stream(stream))
+
+
+def bitlinear_quant_act(x, N, K, xq, amax, xsum, stream=None):
+    return load().bitlinear_quant_act(_p(x), N, K, _p(xq), _p(amax), _p(xsum), _stream(stream))
+
+
+def bitlinear_gemv(packed, alpha, M, K, xq, amax, xsum, N, y, acc=None, stream=None):
+    return load().bitlinear_gemv(_p(packed), _p(alpha), M, K, _p(xq), _p(amax), _p(xsum), N,
+                                 _p(y), _p(acc), _stream(stream))
+
+
+def bitlinear_gemm(packed, alpha, M, K, xq, amax, xsum, N, y, acc=None, stream=None):
+    return load().bitlinear_gemm(_p(packed), _p(alpha), M, K, _p(xq), _p(amax), _p(xsum), N,
+                                 _p(y), _p(acc), _stream(stream))
+
+
+def bitlinear_pack_workspace_bytes(M, K):
+    return load().bitlinear_pack_workspace_bytes(M, K)
+
+
+def bitlinear_device_error(clear=True):
+    out = ctypes.c_int(0)
+    check(load().bitlinear_device_error(ctypes.byref(out), 1 if clear else 0),
+          "bitlinear_device_error")
+    return out.value

@@ -1,0 +1,105 @@
+"""Torch-facing calls of the ternary BitLinear path.
+
+Each function checks dtype, device and contiguity, allocates its outputs with
+torch (device memory is torch's job here), and hands raw pointers to one C
+entry point of libbitlinear.so.  All arithmetic runs in the CUDA kernels;
+nothing here falls back to the CPU.
+"""
+import torch
+
+from . import _lib
+
+# Largest token count the CUDA-core GEMV handles; above it the tensor-core
+# GEMM takes over (the crossover table lives in `matmul`).
+GEMV_MAX_TOKENS = 16
+
+
+def _need(t, dtype, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (no CPU path exists)" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def pack_weights(W, stream=None):
+    """fp32 W[M,K] -> (packed int32 [M, K/16] holding the uint32 words, alpha fp32 [1])."""
+    _need(W, torch.float32, "W")
+    M, K = W.shape
+    packed = torch.empty((M, K // 16), dtype=torch.int32, device=W.device)
+    alpha = torch.empty(1, dtype=torch.float32, device=W.device)
+    nbytes = _lib.bitlinear_pack_workspace_bytes(M, K)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _lib.check(_lib.bitlinear_pack_weights(W, M, K, packed, alpha, ws, nbytes, stream),
+               "bitlinear_pack_weights")
+    return packed, alpha
+
+
+def quant_act(x, stream=None, with_sum=True):
+    """fp32 x[N,K] -> (xq int8 [N,K], amax fp32 [N], xsum int32 [N] or None)."""
+    _need(x, torch.float32, "x")
+    N, K = x.shape
+    xq = torch.empty((N, K), dtype=torch.int8, device=x.device)
+    amax = torch.empty(N, dtype=torch.float32, device=x.device)
+    xsum = torch.empty(N, dtype=torch.int32, device=x.device) if with_sum else None
+    _lib.check(_lib.bitlinear_quant_act(x, N, K, xq, amax, xsum, stream), "bitlinear_quant_act")
+    return xq, amax, xsum
+
+
+def _matmul(fn, name, packed, alpha, xq, amax, xsum, M, with_acc, stream, out=None):
+    _need(packed, torch.int32, "packed")
+    _need(alpha, torch.float32, "alpha")
+    _need(xq, torch.int8, "xq")
+    _need(amax, torch.float32, "amax")
+    _need(xsum, torch.int32, "xsum")
+    N, K = xq.shape
+    if packed.shape != (M, K // 16):
+        raise ValueError("packed must be [M, K/16] = [%d, %d], got %s" % (M, K // 16,
+                                                                         tuple(packed.shape)))
+    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=xq.device)
+    acc = torch.empty((N, M), dtype=torch.int32, device=xq.device) if with_acc else None
+    _lib.check(fn(packed, alpha, M, K, xq, amax, xsum, N, y, acc, stream), name)
+    return (y, acc) if with_acc else y
+
+
+def gemv(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out=None):
+    """Decode GEMV (N <= 16): y[N,M] fp32 (and int32 acc if with_acc)."""
+    M = packed.shape[0] if M is None else M
+    return _matmul(_lib.bitlinear_gemv, "bitlinear_gemv", packed, alpha, xq, amax, xsum, M,
+                   with_acc, stream, out)
+
+
+def gemm(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out=None):
+    """Tensor-core GEMM (any N, M % 128 == 0): y[N,M] fp32 (and int32 acc)."""
+    M = packed.shape[0] if M is None else M
+    return _matmul(_lib.bitlinear_gemm, "bitlinear_gemm", packed, alpha, xq, amax, xsum, M,
+                   with_acc, stream, out)
+
+
+def matmul(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out=None):
+    """GEMV for N <= GEMV_MAX_TOKENS (or when M is not a multiple of 128), else GEMM."""
+    M = packed.shape[0] if M is None else M
+    if xq.shape[0] <= GEMV_MAX_TOKENS or M % 128 != 0:
+        return gemv(packed, alpha, xq, amax, xsum, M, with_acc, stream, out)
+    return gemm(packed, alpha, xq, amax, xsum, M, with_acc, stream, out)
+
+
+class TernaryLinear:
+    """A BitLinear layer: packed 2-bit ternary weights + alpha, applied to fp32
+    activations as quant_act -> GEMV/GEMM with the fused rescale."""
+
+    def __init__(self, packed, alpha, in_features, out_features):
+        self.packed, self.alpha = packed, alpha
+        self.in_features, self.out_features = in_features, out_features
+
+    @classmethod
+    def from_float(cls, W, stream=None):
+        packed, alpha = pack_weights(W, stream)
+        return cls(packed, alpha, W.shape[1], W.shape[0])
+
+    def __call__(self, x, stream=None):
+        xq, amax, xsum = quant_act(x, stream)
+        return matmul(self.packed, self.alpha, xq, amax, xsum, self.out_features, stream=stream)

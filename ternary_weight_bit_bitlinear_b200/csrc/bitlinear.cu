@@ -1,0 +1,266 @@
+// bitlinear.cu -- the C ABI of libbitlinear.so (declared in include/bitlinear.h):
+// argument checks, launch configuration and TMA descriptor set-up around the
+// sm_100a kernels in pack.cuh, quant.cuh, gemv.cuh and gemm.cuh.
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cstdint>
+#include <mutex>
+
+#include "bitlinear.h"
+#include "gemm.cuh"
+#include "gemv.cuh"
+#include "pack.cuh"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int64_t kMaxK = 131072;
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bitlinear_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
+}
+
+bitlinear_status check_mk(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return BITLINEAR_ERR_INVALID_ARG;
+  if (M == 0 || K == 0 || K % 128 != 0 || K > kMaxK) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  if (M > INT_MAX / 2 || M * K > kMaxElems) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  return BITLINEAR_OK;
+}
+
+// Per-device facts, looked up once per device.
+struct DeviceInfo {
+  int sms = 0;
+  bool gemm_attr_set[2] = {false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+bitlinear_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return BITLINEAR_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    d.sms = sms;
+  }
+  *out = &d;
+  return BITLINEAR_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 2-D uint8 tensor [rows][cols] with row pitch `cols` bytes, box {box_cols, box_rows}.
+bool encode_u8_2d(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows,
+                  uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int NT>
+void launch_gemv(const uint32_t* packed, const float* alpha, int M, int K, const int8_t* xq,
+                 const float* amax, const int32_t* xsum, float* y, int32_t* acc,
+                 cudaStream_t s) {
+  const int rows_per_block = (bl::kGemvThreads / 32) * bl::kGemvRows;
+  const int grid = (M + rows_per_block - 1) / rows_per_block;
+  bl::gemv_kernel<NT><<<grid, bl::kGemvThreads, 0, s>>>(
+      reinterpret_cast<const uint4*>(packed), M, K / 64, reinterpret_cast<const uint4*>(xq),
+      alpha, amax, xsum, y, acc);
+}
+
+template <int BN, int STAGES>
+bitlinear_status launch_gemm(const bl::GemmParams& p, DeviceInfo* dev, int slot, cudaStream_t s) {
+  auto kernel = bl::gemm_i8_tcgen05_kernel<BN, STAGES>;
+  const int smem = static_cast<int>(sizeof(bl::GemmSmem<BN, STAGES>)) + 1024;
+  if (!dev->gemm_attr_set[slot]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    dev->gemm_attr_set[slot] = true;
+  }
+  const int grid = p.total_tiles < dev->sms ? p.total_tiles : dev->sms;
+  kernel<<<grid, bl::kGemmThreads, smem, s>>>(p);
+  return launch_status();
+}
+
+bitlinear_status check_matmul_args(const uint32_t* packed, const float* alpha, int64_t M,
+                                   int64_t K, const int8_t* xq, const float* amax,
+                                   const int32_t* xsum, int64_t N, float* y, int32_t* acc) {
+  bitlinear_status st = check_mk(M, K);
+  if (st != BITLINEAR_OK) return st;
+  if (N < 0) return BITLINEAR_ERR_INVALID_ARG;
+  if (N == 0) return BITLINEAR_OK;
+  if (N > INT_MAX / 2) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  if (!packed || !alpha || !xq || !amax || !xsum || !y) return BITLINEAR_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(xq) || !aligned16(y) || (acc && !aligned16(acc)))
+    return BITLINEAR_ERR_MISALIGNED;
+  if (!aligned16(alpha) || !aligned16(amax) || !aligned16(xsum)) return BITLINEAR_ERR_MISALIGNED;
+  return BITLINEAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bitlinear_status_string(int status) {
+  switch (status) {
+    case BITLINEAR_OK: return "ok";
+    case BITLINEAR_ERR_INVALID_ARG: return "invalid argument";
+    case BITLINEAR_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case BITLINEAR_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case BITLINEAR_ERR_WORKSPACE: return "workspace missing or too small";
+    case BITLINEAR_ERR_CUDA: return "CUDA error";
+    case BITLINEAR_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int bitlinear_version(void) { return 100; }
+
+size_t bitlinear_pack_workspace_bytes(int64_t M, int64_t K) {
+  (void)M;
+  (void)K;
+  return bl::kPackWorkspaceBytes;
+}
+
+bitlinear_status bitlinear_pack_weights(const float* W, int64_t M, int64_t K, uint32_t* packed,
+                                        float* alpha, void* workspace, size_t workspace_bytes,
+                                        bitlinear_stream_t stream) {
+  bitlinear_status st = check_mk(M, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!W || !packed || !alpha) return BITLINEAR_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < bl::kPackWorkspaceBytes) return BITLINEAR_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(workspace) || !aligned16(alpha))
+    return BITLINEAR_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != BITLINEAR_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto* bins = static_cast<unsigned long long*>(workspace);
+  auto* flag = reinterpret_cast<unsigned int*>(bins + bl::kBins);
+  if (cudaMemsetAsync(workspace, 0, bl::kPackWorkspaceBytes, s) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  const int64_t n4 = M * K / 4;
+  int grid = dev->sms * 4;
+  bl::abs_bins_kernel<<<grid, bl::kBinsThreads, 0, s>>>(reinterpret_cast<const float4*>(W), n4,
+                                                         bins, flag);
+  bl::alpha_finalize_kernel<<<1, 32, 0, s>>>(bins, flag, static_cast<uint64_t>(M * K), alpha);
+  const int64_t words = M * K / 16;
+  int64_t g = (words + 255) / 256;
+  if (g > dev->sms * 16) g = dev->sms * 16;
+  bl::ternarize_pack_kernel<<<static_cast<int>(g), 256, 0, s>>>(
+      reinterpret_cast<const float4*>(W), words, alpha, packed);
+  return launch_status();
+}
+
+bitlinear_status bitlinear_quant_act(const float* x, int64_t N, int64_t K, int8_t* xq,
+                                     float* amax, int32_t* xsum, bitlinear_stream_t stream) {
+  if (N < 0 || K < 0) return BITLINEAR_ERR_INVALID_ARG;
+  if (K == 0 || K % 128 != 0 || K > kMaxK || N > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0) return BITLINEAR_OK;
+  if (!x || !xq || !amax) return BITLINEAR_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(amax) || (xsum && !aligned16(xsum)))
+    return BITLINEAR_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bl::quant_act_kernel<<<static_cast<int>(N), bl::kQuantThreads, 0, s>>>(x, static_cast<int>(K),
+                                                                          xq, amax, xsum);
+  return launch_status();
+}
+
+bitlinear_status bitlinear_gemv(const uint32_t* packed, const float* alpha, int64_t M, int64_t K,
+                                const int8_t* xq, const float* amax, const int32_t* xsum,
+                                int64_t N, float* y, int32_t* acc, bitlinear_stream_t stream) {
+  bitlinear_status st = check_matmul_args(packed, alpha, M, K, xq, amax, xsum, N, y, acc);
+  if (st != BITLINEAR_OK || N == 0) return st;
+  if (N > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int m = static_cast<int>(M), k = static_cast<int>(K);
+  switch (N) {
+#define BL_GEMV_CASE(n) \
+  case n: launch_gemv<n>(packed, alpha, m, k, xq, amax, xsum, y, acc, s); break;
+    BL_GEMV_CASE(1) BL_GEMV_CASE(2) BL_GEMV_CASE(3) BL_GEMV_CASE(4)
+    BL_GEMV_CASE(5) BL_GEMV_CASE(6) BL_GEMV_CASE(7) BL_GEMV_CASE(8)
+    BL_GEMV_CASE(9) BL_GEMV_CASE(10) BL_GEMV_CASE(11) BL_GEMV_CASE(12)
+    BL_GEMV_CASE(13) BL_GEMV_CASE(14) BL_GEMV_CASE(15) BL_GEMV_CASE(16)
+#undef BL_GEMV_CASE
+    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  }
+  return launch_status();
+}
+
+bitlinear_status bitlinear_gemm(const uint32_t* packed, const float* alpha, int64_t M, int64_t K,
+                                const int8_t* xq, const float* amax, const int32_t* xsum,
+                                int64_t N, float* y, int32_t* acc, bitlinear_stream_t stream) {
+  bitlinear_status st = check_matmul_args(packed, alpha, M, K, xq, amax, xsum, N, y, acc);
+  if (st != BITLINEAR_OK || N == 0) return st;
+  if (M % 128 != 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != BITLINEAR_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool wide = N > 128;
+  const int BN = wide ? 256 : 128;
+  bl::GemmParams p;
+  memset(&p, 0, sizeof p);
+  if (!encode_u8_2d(&p.tmA[0], packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(M),
+                    bl::kGemmPackedRowBytes, bl::kGemmBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_u8_2d(&p.tmB[0], xq, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                    bl::kGemmBK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BITLINEAR_ERR_CUDA;
+  bl::GemmProblem& pr = p.prob[0];
+  pr.alpha = alpha;
+  pr.amax = amax;
+  pr.xsum = xsum;
+  pr.y = y;
+  pr.acc = acc;
+  pr.M = static_cast<int>(M);
+  pr.K = static_cast<int>(K);
+  pr.N = static_cast<int>(N);
+  pr.n_tiles = static_cast<int>((N + BN - 1) / BN);
+  pr.tile_begin = 0;
+  p.num_problems = 1;
+  p.total_tiles = static_cast<int>(M / bl::kGemmBM) * pr.n_tiles;
+  return wide ? launch_gemm<256, 4>(p, dev, 1, s) : launch_gemm<128, 6>(p, dev, 0, s);
+}
+
+bitlinear_status bitlinear_device_error(int* status_out, int clear) {
+  if (!status_out) return BITLINEAR_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bl::g_device_error, sizeof v) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  *status_out = (v & bl::kDeviceTimeout) ? BITLINEAR_ERR_DEVICE_TIMEOUT : BITLINEAR_OK;
+  if (clear && v) {
+    unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(bl::g_device_error, &zero, sizeof zero) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+  }
+  return BITLINEAR_OK;
+}
+
+}  // extern "C"

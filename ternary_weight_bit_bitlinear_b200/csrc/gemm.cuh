@@ -1,0 +1,261 @@
+// gemm.cuh -- prefill mpGEMM on the 5th-generation tensor cores.
+//
+// For many tokens the ternary x int8 product is a dense contraction (the
+// reading notes, section 4.4, note that prefill turns compute-bound and is
+// left unoptimised by the CPU kernels).  Each CTA owns a 128-row weight block
+// and a BN-token block, accumulating D[128 x BN] (int32) in tensor memory:
+//
+//   warp 0      TMA producer: packed weight tile (128 rows x 32 bytes = 128
+//               weights per row) and int8 activation tile (BN x 128, 128-byte
+//               swizzle) into a STAGES-deep shared-memory ring;
+//   warps 2-5   unpackers: one weight row per thread, 2-bit fields -> int8
+//               codes+1 written in the 128-byte-swizzled K-major layout the
+//               MMA reads, then a proxy fence and an mbarrier arrive;
+//   warp 1      MMA issuer: 4 x tcgen05.mma kind::i8 (K = 32 each) per stage,
+//               tcgen05.commit frees the stage; accumulators double-buffered
+//               in tensor memory so the epilogue of tile i overlaps tile i+1;
+//   warps 6-9   epilogue: tcgen05.ld, acc - xsum (removes the +1 code offset),
+//               rescale by alpha * amax/127, coalesced fp32 stores.
+//
+// Several independent problems (e.g. the projections of a layer) can share one
+// persistent launch: tiles are numbered across problems.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace bl {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 128;                       // int8 elements per k-block
+constexpr int kGemmPackedRowBytes = kGemmBK / 4;   // 32 bytes of 2-bit fields
+constexpr int kGemmThreads = 320;                  // 10 warps
+constexpr int kGemmMaxProblems = 8;
+
+struct GemmProblem {
+  const float* alpha;
+  const float* amax;
+  const int32_t* xsum;
+  float* y;
+  int32_t* acc;
+  int M, K, N;
+  int n_tiles;      // ceil(N / BN)
+  int tile_begin;   // first global tile of this problem
+};
+
+struct GemmParams {
+  CUtensorMap tmA[kGemmMaxProblems];   // packed weights as uint8 [M][K/4], box 32 x 128
+  CUtensorMap tmB[kGemmMaxProblems];   // xq as uint8 [N][K], box 128 x BN, 128B swizzle
+  GemmProblem prob[kGemmMaxProblems];
+  int num_problems;
+  int total_tiles;
+};
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  uint8_t b[STAGES][BN * kGemmBK];                          // 1024-aligned stages
+  uint8_t a[STAGES][kGemmBM * kGemmBK];                     // unpacked codes+1
+  uint8_t apk[STAGES][kGemmBM * kGemmPackedRowBytes];       // packed tile
+  uint64_t full[STAGES];
+  uint64_t unpacked[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_slot;
+  int abort;
+};
+
+template <int BN>
+__device__ __forceinline__ void gemm_locate(const GemmParams& p, int tile, int& pi, int& m_blk,
+                                            int& n_blk) {
+  pi = 0;
+  while (pi + 1 < p.num_problems && tile >= p.prob[pi + 1].tile_begin) ++pi;
+  const int lt = tile - p.prob[pi].tile_begin;
+  m_blk = lt / p.prob[pi].n_tiles;
+  n_blk = lt - m_blk * p.prob[pi].n_tiles;
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  using Smem = GemmSmem<BN, STAGES>;
+  const uint32_t base = smem_u32(smem_raw);
+  Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr uint32_t kTmemCols = 2 * BN;
+  constexpr uint32_t kStageTx = kGemmBM * kGemmPackedRowBytes + BN * kGemmBK;
+  volatile int* abort = &s.abort;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.unpacked[i], 128);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], 128);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_mbar_init();
+    for (int i = 0; i < p.num_problems; ++i) {
+      tma_prefetch_desc(&p.tmA[i]);
+      tma_prefetch_desc(&p.tmB[i]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s.tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+        int pi, m_blk, n_blk;
+        gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+        const int kblocks = p.prob[pi].K / kGemmBK;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort)) goto producer_done;
+          mbar_arrive_expect_tx(&s.full[stage], kStageTx);
+          tma_load_2d(s.apk[stage], &p.tmA[pi], &s.full[stage], kb * kGemmPackedRowBytes,
+                      m_blk * kGemmBM);
+          tma_load_2d(s.b[stage], &p.tmB[pi], &s.full[stage], kb * kGemmBK, n_blk * BN);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
+      uint32_t stage = 0, phase = 0;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++it) {
+        int pi, m_blk, n_blk;
+        gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+        const int kblocks = p.prob[pi].K / kGemmBK;
+        const uint32_t ab = it & 1, ap = (it >> 1) & 1;
+        if (!mbar_wait(&s.tempty[ab], ap ^ 1u, abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + ab * BN;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&s.full[stage], phase, abort) ||
+              !mbar_wait(&s.unpacked[stage], phase, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(s.a[stage]);
+          const uint32_t b_addr = smem_u32(s.b[stage]);
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 32; ++kk) {
+            mma_i8_ss(d_tmem, smem_desc_k_sw128(a_addr + 32 * kk),
+                      smem_desc_k_sw128(b_addr + 32 * kk), idesc, (kb | kk) != 0);
+          }
+          mma_commit(&s.empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&s.tfull[ab]);
+      }
+      // Everything issued must finish before tensor memory is released.
+      mma_commit(&s.drain);
+      unsigned long long t0 = global_timer_ns();
+      while (!mbar_try_wait(&s.drain, 0)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          atomicOr(&g_device_error, kDeviceTimeout);
+          break;
+        }
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ unpackers
+    const int u = threadIdx.x - 64;   // weight row within the tile
+    const uint32_t sw = static_cast<uint32_t>(u & 7);
+    uint32_t stage = 0, phase = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+      int pi, m_blk, n_blk;
+      gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+      const int kblocks = p.prob[pi].K / kGemmBK;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!mbar_wait(&s.full[stage], phase, abort)) goto unpack_done;
+        const uint4* src = reinterpret_cast<const uint4*>(s.apk[stage] + u * kGemmPackedRowBytes);
+        const uint4 p0 = src[0], p1 = src[1];
+        const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        uint8_t* row = s.a[stage] + (u >> 3) * 1024 + (u & 7) * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t w = words[j];
+          uint4 v;
+          v.x = w & 0x03030303u;
+          v.y = (w >> 2) & 0x03030303u;
+          v.z = (w >> 4) & 0x03030303u;
+          v.w = (w >> 6) & 0x03030303u;
+          *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(j) ^ sw) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&s.unpacked[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  unpack_done:;
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t quarter = static_cast<uint32_t>(warp & 3);   // TMEM lanes 32q .. 32q+31
+    const int r_in_tile = static_cast<int>(quarter) * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++it) {
+      int pi, m_blk, n_blk;
+      gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+      const GemmProblem& pr = p.prob[pi];
+      const uint32_t ab = it & 1, ap = (it >> 1) & 1;
+      if (!mbar_wait(&s.tfull[ab], ap, abort)) break;
+      tc_fence_after();
+      const int m = m_blk * kGemmBM + r_in_tile;
+      const float alpha = *pr.alpha;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + ab * BN + cc * 32, r);
+        tmem_ld_wait();
+        const int n0 = n_blk * BN + cc * 32;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int n = n0 + j;
+          if (n < pr.N) {
+            const int a = static_cast<int>(r[j]) - __ldg(pr.xsum + n);
+            const float scale = __fmul_rn(alpha, __fdiv_rn(__ldg(pr.amax + n), 127.0f));
+            const int64_t o = static_cast<int64_t>(n) * pr.M + m;
+            pr.y[o] = __fmul_rn(__int2float_rn(a), scale);
+            if (pr.acc) pr.acc[o] = a;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s.tempty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace bl

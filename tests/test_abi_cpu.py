@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+Every call below fails argument validation before the library touches CUDA,
+so these tests are safe with or without a device present.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from ternary_weight_bit_bitlinear_b200 import _lib, build
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: every case fails validation first
+MISALIGNED = 0x10004
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.load()
+
+
+def test_library_exports_every_declared_symbol(L):
+    declared = _lib.header_symbols()
+    assert len(declared) >= 8
+    for name in declared:
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(declared) <= exported
+    assert {n for n in exported if n.startswith("bitlinear_")} == set(declared)
+
+
+def test_version_and_status_strings(L):
+    assert L.bitlinear_version() == 100
+    for code in range(7):
+        assert _lib.status_string(code)
+    assert _lib.status_string(0) == "ok"
+    assert _lib.status_string(99) == "unknown status"
+
+
+def test_missing_library_raises(tmp_path):
+    saved = _lib._lib
+    try:
+        _lib._lib = None
+        with pytest.raises(ImportError):
+            _lib.load(str(tmp_path / "nope.so"))
+    finally:
+        _lib._lib = saved
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_pack_argument_errors(L):
+    ws = L.bitlinear_pack_workspace_bytes(128, 128)
+    assert ws >= 256 * 8
+    f = L.bitlinear_pack_weights
+    ok = dict(W=FAKE, M=128, K=128, packed=FAKE, alpha=FAKE, ws=FAKE, wsb=ws)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(_p(a["W"]), a["M"], a["K"], _p(a["packed"]), _p(a["alpha"]), _p(a["ws"]),
+                 a["wsb"], None)
+
+    assert call(W=0) == _lib.ERR_INVALID_ARG
+    assert call(alpha=0) == _lib.ERR_INVALID_ARG
+    assert call(M=-1) == _lib.ERR_INVALID_ARG
+    assert call(K=100) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(K=0) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(K=131072 + 128) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(M=(1 << 40) // 128 + 1) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(ws=0) == _lib.ERR_WORKSPACE
+    assert call(wsb=ws - 1) == _lib.ERR_WORKSPACE
+    assert call(W=MISALIGNED) == _lib.ERR_MISALIGNED
+    assert call(packed=MISALIGNED) == _lib.ERR_MISALIGNED
+
+
+def test_quant_act_argument_errors(L):
+    f = L.bitlinear_quant_act
+    assert f(_p(FAKE), 1, 100, _p(FAKE), _p(FAKE), None, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert f(_p(FAKE), -1, 128, _p(FAKE), _p(FAKE), None, None) == _lib.ERR_INVALID_ARG
+    assert f(_p(0), 1, 128, _p(FAKE), _p(FAKE), None, None) == _lib.ERR_INVALID_ARG
+    assert f(_p(FAKE), 1, 128, _p(MISALIGNED), _p(FAKE), None, None) == _lib.ERR_MISALIGNED
+    assert f(_p(FAKE), 0, 128, _p(FAKE), _p(FAKE), None, None) == _lib.OK   # N = 0: no-op
+
+
+@pytest.mark.parametrize("name", ["bitlinear_gemv", "bitlinear_gemm"])
+def test_matmul_argument_errors(L, name):
+    f = getattr(L, name)
+    ok = dict(packed=FAKE, alpha=FAKE, M=128, K=256, xq=FAKE, amax=FAKE, xsum=FAKE, N=1,
+              y=FAKE, acc=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(_p(a["packed"]), _p(a["alpha"]), a["M"], a["K"], _p(a["xq"]), _p(a["amax"]),
+                 _p(a["xsum"]), a["N"], _p(a["y"]), _p(a["acc"]), None)
+
+    assert call(N=0) == _lib.OK
+    assert call(N=-1) == _lib.ERR_INVALID_ARG
+    assert call(packed=0) == _lib.ERR_INVALID_ARG
+    assert call(xsum=0) == _lib.ERR_INVALID_ARG
+    assert call(y=0) == _lib.ERR_INVALID_ARG
+    assert call(K=200) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(M=0) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(y=MISALIGNED) == _lib.ERR_MISALIGNED
+    assert call(acc=MISALIGNED) == _lib.ERR_MISALIGNED
+    assert call(xq=MISALIGNED) == _lib.ERR_MISALIGNED
+    if name == "bitlinear_gemv":
+        assert call(N=17) == _lib.ERR_UNSUPPORTED_SHAPE
+    else:
+        assert call(M=200) == _lib.ERR_UNSUPPORTED_SHAPE
+
+
+def test_header_is_self_contained(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "bitlinear.h"\nint main(void){return BITLINEAR_OK;}\n')
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, "-c", str(src), "-o",
+                    str(tmp_path / "t.o")], check=True)

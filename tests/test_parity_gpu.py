@@ -1,0 +1,204 @@
+"""GPU-vs-oracle parity through the C ABI (ctypes view in ternary_weight_bit_bitlinear_b200._lib).
+
+Inputs come from the seeded generators in ternary_weight_bit_bitlinear_b200.inputs;
+the oracle sees the same fp32 buffers on the host.  The bar: packed words,
+alpha, int8 activations, amax, activation sums and int32 accumulators
+bit-exact; fp32 outputs within 1e-6 relative (they are expected bit-exact,
+since both sides use the same fp32 operation order), zeros exactly zero.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ternary_weight_bit_bitlinear_b200 import _lib, api, build, inputs
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    _lib.load()
+    yield
+    assert _lib.bitlinear_device_error(clear=True) == _lib.OK
+
+
+def dev_t(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def words(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def assert_y_close(y_gpu, y_ref):
+    y_gpu = np.asarray(y_gpu, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    zero = y_ref == 0
+    assert (y_gpu[zero] == 0).all()
+    rel = np.abs(y_gpu[~zero] - y_ref[~zero]) / np.abs(y_ref[~zero])
+    assert rel.size == 0 or rel.max() <= REL_TOL, rel.max()
+
+
+# ----------------------------------------------------------------------------- pack
+
+PACK_SHAPES = [(128, 128), (7, 256), (300, 640), (1024, 1024), (640, 2560), (2560, 6912)]
+
+
+@pytest.mark.parametrize("M,K", PACK_SHAPES)
+def test_pack_parity(M, K):
+    W = inputs.latent_weights(M, K, seed=M * 7 + K)
+    packed, alpha = api.pack_weights(W.cuda())
+    a_ref = oracle.absmean(W.numpy())
+    p_ref = oracle.pack(oracle.ternarize(W.numpy(), a_ref))
+    assert alpha.cpu().numpy()[0] == a_ref
+    assert np.array_equal(words(packed), p_ref)
+
+
+def test_pack_edge_cases():
+    # all zero -> alpha 0, every code 0 (field 01)
+    z = torch.zeros(128, 256, device="cuda")
+    packed, alpha = api.pack_weights(z)
+    assert alpha.item() == 0.0 and (words(packed) == 0x55555555).all()
+    # exact ties: values +-0.5 and +-1.5 in equal numbers -> alpha = 1 exactly,
+    # 0.5 -> 0 (half to even), 1.5 -> clamp(2) = 1
+    base = np.array([0.5, -0.5, 1.5, -1.5], np.float32)
+    W = np.tile(base, (128, 64))
+    packed, alpha = api.pack_weights(dev_t(W))
+    assert alpha.item() == 1.0
+    codes = oracle.unpack(words(packed), 128, 256)
+    assert np.array_equal(codes, np.tile(np.array([0, 0, 1, -1], np.int8), (128, 64)))
+    assert np.array_equal(words(packed), oracle.pack(oracle.ternarize(W, np.float32(1.0))))
+    # subnormal-only weights
+    W = (np.arange(128 * 128, dtype=np.float32).reshape(128, 128) % 97 + 1) * np.float32(1e-45)
+    packed, alpha = api.pack_weights(dev_t(W))
+    a_ref = oracle.absmean(W)
+    assert alpha.cpu().numpy()[0] == a_ref
+    assert np.array_equal(words(packed), oracle.pack(oracle.ternarize(W, a_ref)))
+    # non-finite -> alpha NaN, codes 0
+    W = np.ones((128, 128), np.float32)
+    W[3, 5] = np.inf
+    packed, alpha = api.pack_weights(dev_t(W))
+    assert np.isnan(alpha.item()) and (words(packed) == 0x55555555).all()
+
+
+# ----------------------------------------------------------------------------- quant_act
+
+QUANT_SHAPES = [(1, 1024), (3, 2560), (16, 6912), (33, 4096), (2, 131072), (512, 128)]
+
+
+@pytest.mark.parametrize("N,K", QUANT_SHAPES)
+def test_quant_act_parity(N, K):
+    x = inputs.activations(N, K, seed=N * 13 + K, outlier_frac=0.01)
+    xq, amax, xsum = api.quant_act(x.cuda())
+    q_ref, a_ref, s_ref = oracle.quant_act(x.numpy())
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(amax.cpu().numpy(), a_ref)
+    assert np.array_equal(xsum.cpu().numpy(), s_ref)
+
+
+def test_quant_act_edge_cases():
+    x = np.zeros((4, 256), np.float32)
+    x[1, :] = np.linspace(-3, 3, 256)
+    x[2, :4] = [1e-44, -1e-44, 0.0, 5e-45]          # 127/amax overflows to inf
+    x[3, :] = 127.0
+    x[3, :6] = [0.5, 1.5, 2.5, -0.5, -1.5, -2.5]     # s == 1: ties to even
+    xq, amax, xsum = api.quant_act(dev_t(x))
+    q_ref, a_ref, s_ref = oracle.quant_act(x)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(amax.cpu().numpy(), a_ref)
+    assert np.array_equal(xsum.cpu().numpy(), s_ref)
+    assert xq[3, :6].tolist() == [0, 2, 2, 0, -2, -2]
+
+
+# ----------------------------------------------------------------------------- matmul
+
+def _layer(M, K, N, seed, outlier_frac=0.0):
+    W = inputs.latent_weights(M, K, seed=seed)
+    x = inputs.activations(N, K, seed=seed + 500, outlier_frac=outlier_frac)
+    ref = oracle.bitlinear(W.numpy(), x.numpy())
+    packed, alpha = api.pack_weights(W.cuda())
+    xq, amax, xsum = api.quant_act(x.cuda())
+    return ref, (packed, alpha, xq, amax, xsum)
+
+
+@pytest.mark.parametrize("N", list(range(1, 17)))
+def test_gemv_parity_all_token_counts(N):
+    M, K = 300, 640        # ragged row blocks
+    ref, (packed, alpha, xq, amax, xsum) = _layer(M, K, N, seed=100 + N)
+    y, acc = api.gemv(packed, alpha, xq, amax, xsum, with_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_y_close(y.cpu().numpy(), ref["y"])
+    assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("M,K,N", [(1024, 1024, 1), (2560, 6912, 1), (640, 2560, 4),
+                                   (6912, 2560, 16), (1, 128, 1), (129, 28672, 2)])
+def test_gemv_parity_shapes(M, K, N):
+    ref, (packed, alpha, xq, amax, xsum) = _layer(M, K, N, seed=M + K + N, outlier_frac=0.01)
+    y, acc = api.gemv(packed, alpha, xq, amax, xsum, with_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_y_close(y.cpu().numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("M,K,N", [(128, 128, 1), (256, 512, 200), (384, 1024, 129),
+                                   (128, 256, 16), (1024, 2560, 512), (512, 4096, 300),
+                                   (256, 6912, 77)])
+def test_gemm_parity(M, K, N):
+    ref, (packed, alpha, xq, amax, xsum) = _layer(M, K, N, seed=3 * M + K + N)
+    y, acc = api.gemm(packed, alpha, xq, amax, xsum, with_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert_y_close(y.cpu().numpy(), ref["y"])
+    assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
+def test_gemm_matches_gemv_small_n():
+    ref, (packed, alpha, xq, amax, xsum) = _layer(512, 1024, 9, seed=77)
+    y1, a1 = api.gemv(packed, alpha, xq, amax, xsum, with_acc=True)
+    y2, a2 = api.gemm(packed, alpha, xq, amax, xsum, with_acc=True)
+    assert torch.equal(a1, a2) and torch.equal(y1, y2)
+    assert np.array_equal(a1.cpu().numpy(), ref["acc"])
+
+
+def test_zero_token_and_zero_weights():
+    M, K, N = 256, 512, 3
+    W = inputs.latent_weights(M, K, seed=5)
+    x = inputs.activations(N, K, seed=6)
+    x[1] = 0
+    ref = oracle.bitlinear(W.numpy(), x.numpy())
+    packed, alpha = api.pack_weights(W.cuda())
+    xq, amax, xsum = api.quant_act(x.cuda())
+    for fn in (api.gemv, api.gemm):
+        y, acc = fn(packed, alpha, xq, amax, xsum, with_acc=True)
+        assert (y[1] == 0).all() and (acc[1] == 0).all()
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    zp, za = api.pack_weights(torch.zeros(M, K, device="cuda"))
+    for fn in (api.gemv, api.gemm):
+        y = fn(zp, za, xq, amax, xsum)
+        assert (y == 0).all()
+
+
+def test_empty_batch_is_noop():
+    packed, alpha = api.pack_weights(inputs.latent_weights(128, 128, seed=1).cuda())
+    xq = torch.empty(0, 128, dtype=torch.int8, device="cuda")
+    amax = torch.empty(0, dtype=torch.float32, device="cuda")
+    xsum = torch.empty(0, dtype=torch.int32, device="cuda")
+    for fn in (_lib.bitlinear_gemv, _lib.bitlinear_gemm):
+        y = torch.empty(1, 128, device="cuda")
+        # empty tensors may carry a NULL data pointer: N == 0 returns before any check
+        st = fn(packed, alpha, 128, 128, xq, amax, xsum, 0, y)
+        assert st == _lib.OK
+
+
+def test_rejects_bad_shapes_on_device():
+    ref, (packed, alpha, xq, amax, xsum) = _layer(256, 256, 17, seed=9)
+    y = torch.empty(17, 256, device="cuda")
+    assert _lib.bitlinear_gemv(packed, alpha, 256, 256, xq, amax, xsum, 17, y) == \
+        _lib.ERR_UNSUPPORTED_SHAPE
+    assert _lib.bitlinear_gemm(packed, alpha, 200, 256, xq, amax, xsum, 17, y) == \
+        _lib.ERR_UNSUPPORTED_SHAPE
