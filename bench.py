@@ -1,0 +1,627 @@
+#!/usr/bin/env python
+"""Benchmark of the ternary BitLinear path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (one JSON line on rank 0): effective packed-weight GB/s of the decode
+path at N=1 on the BitNet-b1.58-2B-shaped workload -- 30 decoder layers x 7
+BitLinear projections (q 2560x2560, k/v 640x2560, o 2560x2560, gate/up
+6912x2560, down 2560x6912), every linear fed one token.  One step:
+
+    quant_act(90 x 2560 activation rows)   quant_act(30 x 6912 rows)
+    gemv_grouped(180 layers, K=2560)       gemv_grouped(30 layers, K=6912)
+
+i.e. per-token absmax int8 quantisation of every layer input and the ternary x
+int8 GEMV with fused rescale of every projection; the 521 MB of packed weights
+exceed the 126 MB L2, so no flush is needed between steps.  The same JSON line
+carries the prefill measurement (7B-shaped layer, 7 projections, N=512 tokens,
+tensor-core GEMM, int8 TOPS), a dependent per-layer decode chain (the launch
+order a real decoder imposes, captured in a CUDA graph), the end-to-end number
+through host buffers, the roofline of the dominant kernel and the CPU oracle
+baseline.
+
+--impl reference times the CPU oracle (the reference arm of this project) on a
+bounded sample of the same workload, on rank 0 only.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from ternary_weight_bit_bitlinear_b200 import _lib, api, inputs  # noqa: E402
+
+METRIC = "ternary BitLinear GB/s (% HBM peak) at N=1; int8 TOPS (% peak) at N=512"
+DECODE_CFG = 2
+PREFILL_CFG = 3
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+INT8_PER_BF16 = 2.0          # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(PEAKS_FALLBACK)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index, interval_ms=50):
+        self.gpu, self.interval, self.proc = gpu_index, interval_ms, None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval)],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.out.flush()
+        self.out.seek(0)
+        sm, smax, reasons = [], None, set()
+        for line in self.out.read().splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.out.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def input_proj(p):
+    """Projection whose seed names the input of projection p (q,k,v share one
+    input, gate/up share one)."""
+    return 0 if p < 3 else 3 if p == 3 else 4 if p < 6 else 6
+
+
+class DecodeWorkload:
+    """30 layers x 7 projections of the 2B shape, one token per linear."""
+
+    def __init__(self, device, layers=None, cfg=DECODE_CFG):
+        wl = inputs.WORKLOADS[cfg]
+        self.shape = wl.model
+        self.layers = layers or wl.layers
+        h, f = self.shape.hidden, self.shape.ffn
+        L = self.layers
+        self.weights = []            # [layer][proj] -> (packed, alpha, M, K)
+        for l in range(L):
+            row = []
+            for p, (name, M, K) in enumerate(self.shape.projections()):
+                W = inputs.latent_weights(M, K, inputs.weight_seed(cfg, l, p), device=device)
+                packed, alpha = api.pack_weights(W)
+                del W
+                row.append((packed, alpha, M, K))
+            self.weights.append(row)
+        torch.cuda.synchronize()
+        # activation inputs: per layer x_qkv, x_o, x_ffn (K = hidden), x_down (K = ffn)
+        self.Xh = torch.empty((3 * L, h), device=device)
+        self.Xf = torch.empty((L, f), device=device)
+        for l in range(L):
+            for j, p in enumerate((0, 3, 4)):
+                self.Xh[3 * l + j] = inputs.activations(1, h, inputs.act_seed(cfg, l, p),
+                                                        device=device)[0]
+            self.Xf[l] = inputs.activations(1, f, inputs.act_seed(cfg, l, 6), device=device)[0]
+        self.XQh = torch.empty((3 * L, h), dtype=torch.int8, device=device)
+        self.XQf = torch.empty((L, f), dtype=torch.int8, device=device)
+        self.AMh = torch.empty(3 * L, device=device)
+        self.AMf = torch.empty(L, device=device)
+        self.XSh = torch.empty(3 * L, dtype=torch.int32, device=device)
+        self.XSf = torch.empty(L, dtype=torch.int32, device=device)
+        per_layer = sum(M for _, M, _ in self.shape.projections())
+        self.Y = torch.empty(L * per_layer, device=device)   # all outputs, one buffer
+        self.ys = []
+        off = 0
+        group_h, group_f = [], []
+        self.chain = []              # per layer: list of (kind, args) launch groups
+        for l in range(L):
+            ys_l = []
+            for p, (packed, alpha, M, K) in enumerate(self.weights[l]):
+                y = self.Y[off:off + M].view(1, M)
+                off += M
+                ys_l.append(y)
+                if K == h:
+                    r = 3 * l + (0 if p < 3 else 1 if p == 3 else 2)
+                    e = (packed, alpha, M, self.XQh[r:r + 1], self.AMh[r:r + 1],
+                         self.XSh[r:r + 1], y, None)
+                    group_h.append(e)
+                else:
+                    e = (packed, alpha, M, self.XQf[l:l + 1], self.AMf[l:l + 1],
+                         self.XSf[l:l + 1], y, None)
+                    group_f.append(e)
+            self.ys.append(ys_l)
+        self.prob_h = _lib.make_problems(group_h)
+        self.prob_f = _lib.make_problems(group_f)
+        self.n_h, self.n_f = len(group_h), len(group_f)
+        self.packed_bytes = sum(M * K // 4 for row in self.weights for _, _, M, K in row)
+        self.packed_bytes_h = sum(M * K // 4 for row in self.weights for _, _, M, K in row
+                                  if K == h)
+        # algorithmic bytes of each grouped GEMV launch: packed weights, the
+        # int8 activations, alpha/amax/xsum and the fp32 outputs of its layers
+        self.alg_bytes_h = sum(e[2] * h // 4 + h + 12 + 4 * e[2] for e in group_h)
+        self.alg_bytes_f = sum(e[2] * f // 4 + f + 12 + 4 * e[2] for e in group_f)
+        self._entries_h, self._entries_f = group_h, group_f
+
+    # each call launches exactly one kernel
+    def quant_h(self, s):
+        _lib.check(_lib.bitlinear_quant_act(self.Xh, self.Xh.shape[0], self.Xh.shape[1],
+                                            self.XQh, self.AMh, self.XSh, s), "quant_act")
+
+    def quant_f(self, s):
+        _lib.check(_lib.bitlinear_quant_act(self.Xf, self.Xf.shape[0], self.Xf.shape[1],
+                                            self.XQf, self.AMf, self.XSf, s), "quant_act")
+
+    def gemv_h(self, s):
+        _lib.check(_lib.bitlinear_gemv_grouped(self.prob_h, self.n_h, self.shape.hidden, 1, s),
+                   "gemv_grouped")
+
+    def gemv_f(self, s):
+        _lib.check(_lib.bitlinear_gemv_grouped(self.prob_f, self.n_f, self.shape.ffn, 1, s),
+                   "gemv_grouped")
+
+    def step(self, s):
+        self.quant_h(s)
+        self.quant_f(s)
+        self.gemv_h(s)
+        self.gemv_f(s)
+
+    def chain_step(self, s):
+        """The order a real decoder imposes: per layer, quantise an input, then
+        run the projections that read it, one group after the other."""
+        h = self.shape.hidden
+        for l in range(self.layers):
+            w = self.weights[l]
+            for (r, projs) in ((3 * l, (0, 1, 2)), (3 * l + 1, (3,)), (3 * l + 2, (4, 5))):
+                _lib.check(_lib.bitlinear_quant_act(self.Xh[r:r + 1], 1, h, self.XQh[r:r + 1],
+                                                    self.AMh[r:r + 1], self.XSh[r:r + 1], s),
+                           "quant_act")
+                ents = [(w[p][0], w[p][1], w[p][2], self.XQh[r:r + 1], self.AMh[r:r + 1],
+                         self.XSh[r:r + 1], self.ys[l][p], None) for p in projs]
+                arr = _lib.make_problems(ents)
+                _lib.check(_lib.bitlinear_gemv_grouped(arr, len(ents), h, 1, s), "gemv_grouped")
+            f = self.shape.ffn
+            _lib.check(_lib.bitlinear_quant_act(self.Xf[l:l + 1], 1, f, self.XQf[l:l + 1],
+                                                self.AMf[l:l + 1], self.XSf[l:l + 1], s),
+                       "quant_act")
+            arr = _lib.make_problems([(w[6][0], w[6][1], w[6][2], self.XQf[l:l + 1],
+                                       self.AMf[l:l + 1], self.XSf[l:l + 1], self.ys[l][6],
+                                       None)])
+            _lib.check(_lib.bitlinear_gemv_grouped(arr, 1, f, 1, s), "gemv_grouped")
+
+
+class PrefillWorkload:
+    """One 7B-shaped layer, 7 projections, N tokens through the tensor-core GEMM."""
+
+    def __init__(self, device, cfg=PREFILL_CFG):
+        wl = inputs.WORKLOADS[cfg]
+        self.shape = wl.model
+        self.N = wl.tokens[0]
+        h, f, N = self.shape.hidden, self.shape.ffn, self.N
+        self.weights = []
+        for p, (name, M, K) in enumerate(self.shape.projections()):
+            W = inputs.latent_weights(M, K, inputs.weight_seed(cfg, 0, p), device=device)
+            self.weights.append(api.pack_weights(W) + (M, K))
+            del W
+        self.X = [inputs.activations(N, h, inputs.act_seed(cfg, 0, p), device=device)
+                  for p in (0, 3, 4)]
+        self.X.append(inputs.activations(N, f, inputs.act_seed(cfg, 0, 6), device=device))
+        self.Q = [api.quant_act(x) for x in self.X]
+        self.src = [0, 0, 0, 1, 2, 2, 3]       # which input each projection reads
+        self.Y = [torch.empty((N, M), device=device) for (_, _, M, _) in self.weights]
+        self.flops = sum(2 * M * N * K for (_, _, M, K) in self.weights)
+
+    def quant(self, i, s):
+        x = self.X[i]
+        xq, am, xs = self.Q[i]
+        _lib.check(_lib.bitlinear_quant_act(x, x.shape[0], x.shape[1], xq, am, xs, s), "quant")
+
+    def gemm(self, p, s):
+        packed, alpha, M, K = self.weights[p]
+        xq, am, xs = self.Q[self.src[p]]
+        _lib.check(_lib.bitlinear_gemm(packed, alpha, M, K, xq, am, xs, self.N, self.Y[p],
+                                       None, s), "gemm")
+
+
+# ----------------------------------------------------------------------------- timing helpers
+
+def events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks = load_peaks()
+    s = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    dec = DecodeWorkload(dev)
+    for _ in range(args.warmup):
+        dec.step(s)
+    torch.cuda.synchronize()
+
+    # ---- headline: K timed decode steps, events around every launch
+    K = args.steps
+    ev = events(5 * K + 2)
+    for e in ev:              # create every event before the timed region
+        e.record(s)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    ev[-2].record(s)
+    for i in range(K):
+        e = ev[5 * i:5 * i + 5]
+        e[0].record(s)
+        dec.quant_h(s)
+        e[1].record(s)
+        dec.quant_f(s)
+        e[2].record(s)
+        dec.gemv_h(s)
+        e[3].record(s)
+        dec.gemv_f(s)
+        e[4].record(s)
+    ev[-1].record(s)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(ev[-2].elapsed_time(ev[-1]))
+    per = {k: 0.0 for k in ("quant_h", "quant_f", "gemv_h", "gemv_f")}
+    for i in range(K):
+        e = ev[5 * i:5 * i + 5]
+        for j, k in enumerate(("quant_h", "quant_f", "gemv_h", "gemv_f")):
+            per[k] += e[j].elapsed_time(e[j + 1])
+    per = {k: v / K for k, v in per.items()}
+    ms_per_step = total_ms / K
+    gbs = world * dec.packed_bytes / (ms_per_step * 1e-3) / 1e9
+    gemv_h_gbs = dec.alg_bytes_h / (per["gemv_h"] * 1e-3) / 1e9
+    hbm_peak = peaks["hbm_gbs"]
+
+    # ---- dependent per-layer chain, CUDA graph
+    chain_ms = None
+    try:
+        gs = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gs):
+            dec.chain_step(gs)          # warm
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=gs):
+            dec.chain_step(gs)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        reps = max(20, K // 50)
+        a, b = events(2)
+        a.record(s)
+        for _ in range(reps):
+            g.replay()
+        b.record(s)
+        torch.cuda.synchronize()
+        chain_ms = a.elapsed_time(b) / reps
+        del g
+    except Exception as exc:  # noqa: BLE001
+        chain_ms = "failed: %s" % exc
+
+    # ---- end to end through host buffers: H2D of every input, D2H of every output
+    hXh = torch.empty(dec.Xh.shape, pin_memory=True)
+    hXf = torch.empty(dec.Xf.shape, pin_memory=True)
+    hY = torch.empty(dec.Y.shape, pin_memory=True)
+    hXh.copy_(dec.Xh)
+    hXf.copy_(dec.Xf)
+    e2e_steps = max(50, K // 10)
+
+    def e2e_step():
+        dec.Xh.copy_(hXh, non_blocking=True)
+        dec.Xf.copy_(hXf, non_blocking=True)
+        dec.step(s)
+        hY.copy_(dec.Y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    a, b = events(2)
+    a.record(s)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(s)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps)
+    h2d = (dec.Xh.numel() + dec.Xf.numel()) * 4
+    d2h = dec.Y.numel() * 4
+
+    # ---- prefill: 7B-shaped layer at N=512 on the tensor cores
+    pre = PrefillWorkload(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        for i in range(4):
+            pre.quant(i, s)
+        for p in range(7):
+            pre.gemm(p, s)
+    torch.cuda.synchronize()
+    P = max(10, min(200, K // 50))
+    gemm_ms, quant_ms, step_ms = 0.0, 0.0, 0.0
+    per_proj = [0.0] * 7
+    for _ in range(P):
+        flush_l2(flush)
+        e = events(13)
+        e[0].record(s)
+        for i in range(4):
+            pre.quant(i, s)
+        e[1].record(s)
+        for p in range(7):
+            pre.gemm(p, s)
+            e[2 + p].record(s)
+        torch.cuda.synchronize()
+        quant_ms += e[0].elapsed_time(e[1])
+        prev = e[1]
+        for p in range(7):
+            per_proj[p] += prev.elapsed_time(e[2 + p])
+            prev = e[2 + p]
+        gemm_ms += e[1].elapsed_time(e[8])
+        step_ms += e[0].elapsed_time(e[8])
+    gemm_ms /= P
+    quant_ms /= P
+    step_ms /= P
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    tops = pre.flops / (gemm_ms * 1e-3) / 1e12
+    prefill = {
+        "workload": "7B-shaped layer, 7 projections (q,k,v,o 4096x4096; gate/up 11008x4096; "
+                    "down 4096x11008), N=512 tokens",
+        "value": round(tops, 1), "unit": "int8 TOPS",
+        "gemm_ms": round(gemm_ms, 4), "quant_ms": round(quant_ms, 4),
+        "step_tops_incl_quant": round(pre.flops / (step_ms * 1e-3) / 1e12, 1),
+        "per_projection_ms": [round(v / P, 4) for v in per_proj],
+        "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(int8_peak, 1),
+                     "unit": "TOPS", "frac": round(tops / int8_peak, 4),
+                     "peak_note": "int8 peak = measured bf16 burst x nominal int8:bf16 ratio 2 (%s)"
+                                  % peaks["source"],
+                     "frac_of_nominal_4500": round(tops / 4500.0, 4), "traffic": None},
+        "l2": "256 MB buffer written between timed steps (flush)",
+    }
+    del flush
+
+    # ---- CPU oracle baseline (rank 0, N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(dec, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        out = {
+            "metric": METRIC,
+            "value": round(gbs, 1),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "i8",
+            "data": "synthetic (seeded N(0,0.02) latent weights, N(0,1) activations)",
+            "config": {
+                "workload": "BitNet-b1.58-2B-shaped decode: 30 layers x 7 projections, N=1",
+                "layers": dec.layers, "tokens": 1,
+                "packed_bytes_per_step": dec.packed_bytes,
+                "launches_per_step": 4,
+                "l2": "no flush: 521 MB of packed weights per step > 126 MB L2",
+                "parallelism": "replicas" if world > 1 else "single GPU",
+            },
+            "pct_of_measured_hbm": round(100 * gbs / world / hbm_peak, 2),
+            "roofline": {
+                "bound": "hbm", "kernel": "gemv_stream (grouped, 180 layers, K=2560)",
+                "achieved": round(gemv_h_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(gemv_h_gbs / hbm_peak, 4),
+                "peak_note": "hbm_gbs %s (burst copy)" % peaks["source"],
+                "bytes_per_launch": dec.alg_bytes_h,
+                "avg_launch_ms": round(per["gemv_h"], 5),
+                "traffic": None,
+            },
+            "kernel_ms": {k: round(v, 5) for k, v in per.items()},
+            "decode_chain": {
+                "what": "same 210 linears, per-layer dependent launches (quant -> qkv, quant -> o,"
+                        " quant -> gate/up, quant -> down), one CUDA graph",
+                "ms_per_step": chain_ms if isinstance(chain_ms, str) else round(chain_ms, 4),
+                "gbs": None if isinstance(chain_ms, str) else
+                round(dec.packed_bytes / (chain_ms * 1e-3) / 1e9, 1),
+                "launches_per_step": 8 * dec.layers,
+            },
+            "prefill": prefill,
+            "e2e": {"value": round(world * dec.packed_bytes / (e2e_ms * 1e-3) / 1e9, 1),
+                    "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * K,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(out), flush=True)
+    assert _lib.bitlinear_device_error(clear=True) == _lib.OK
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def _oracle_layer_sample(dec, layer):
+    """Host copies of one layer for the oracle: codes (unpacked from the
+    oracle's own ternarisation of the seeded latent weights) and activations."""
+    import oracle
+    h = dec.shape.hidden
+    items = []
+    for p, (name, M, K) in enumerate(dec.shape.projections()):
+        W = inputs.latent_weights(M, K, inputs.weight_seed(DECODE_CFG, layer, p),
+                                  device="cuda").cpu().numpy()
+        alpha = oracle.absmean(W)
+        codes = oracle.ternarize(W, alpha)
+        del W
+        if K == h:
+            r = 3 * layer + (0 if p < 3 else 1 if p == 3 else 2)
+            x = dec.Xh[r:r + 1].cpu().numpy()
+        else:
+            x = dec.Xf[layer:layer + 1].cpu().numpy()
+        items.append((codes, alpha, x, M * K // 4))
+    return items
+
+
+def _oracle_time(items):
+    import oracle
+    t0 = time.perf_counter()
+    nbytes = 0
+    for codes, alpha, x, pb in items:
+        q, amax, _ = oracle.quant_act(x)
+        acc = oracle.matmul_i32(codes, q)
+        oracle.rescale(acc, alpha, amax)
+        nbytes += pb
+    return nbytes, time.perf_counter() - t0
+
+
+def cpu_baseline(dec, budget_s=15.0):
+    items = _oracle_layer_sample(dec, 0)
+    nbytes, secs, reps = 0, 0.0, 0
+    while secs < budget_s or reps == 0:
+        b, t = _oracle_time(items)
+        nbytes += b
+        secs += t
+        reps += 1
+    return {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": "layer 0 of the 2B-shaped stream (7 projections, N=1): quant_act + int32 "
+                      "triple-loop matmul + rescale, x%d (%.1f s)" % (reps, secs)}
+
+
+def run_reference(args, rank, world):
+    """CPU oracle on bounded samples of the decode workload (rank 0 only)."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    cfg = inputs.WORKLOADS[DECODE_CFG]
+    h = cfg.model.hidden
+    projs = cfg.model.projections()
+    # one step = rows [r0, r0+R) of one projection of layer 0 (rotating), N=1;
+    # R sized so that warmup + steps stay within ~90 s of CPU time
+    data = []
+    for p, (name, M, K) in enumerate(projs):
+        W = inputs.latent_weights(M, K, inputs.weight_seed(DECODE_CFG, 0, p)).numpy()
+        alpha = oracle.absmean(W)
+        codes = oracle.ternarize(W, alpha)
+        x = inputs.activations(1, K, inputs.act_seed(DECODE_CFG, 0, input_proj(p))).numpy()
+        data.append((codes, alpha, x))
+    t0 = time.perf_counter()
+    c, a, x = data[0]
+    q, amax, _ = oracle.quant_act(x)
+    oracle.matmul_i32(c[:256], q)
+    rate = 256 * c.shape[1] / max(time.perf_counter() - t0, 1e-6)     # weights per second
+    total = max(1, args.steps + args.warmup)
+    per_step_w = max(128 * 2560, int(rate * 90.0 / total))
+    nbytes, secs = 0, 0.0
+    for i in range(args.warmup + args.steps):
+        codes, alpha, x = data[i % 7]
+        rows = max(1, min(codes.shape[0], per_step_w // codes.shape[1]))
+        r0 = (i * 131) % max(1, codes.shape[0] - rows + 1)
+        t = time.perf_counter()
+        q, amax, _ = oracle.quant_act(x)
+        acc = oracle.matmul_i32(np.ascontiguousarray(codes[r0:r0 + rows]), q)
+        oracle.rescale(acc, alpha, amax)
+        dt = time.perf_counter() - t
+        if i >= args.warmup:
+            nbytes += rows * codes.shape[1] // 4
+            secs += dt
+    v = nbytes / secs / 1e9
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(1e3 * secs / max(1, args.steps), 4), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+           "config": {"workload": "BitNet-b1.58-2B-shaped decode: 30 layers x 7 projections, N=1",
+                      "layers": 30, "tokens": 1},
+           "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                            "sample": "per step: a row block of one projection of layer 0 "
+                                      "(rotating over the 7), quant_act + matmul + rescale"},
+           "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", args.gpus if args.gpus == 1 else 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -28,7 +28,9 @@
  * Conventions for every entry point:
  *   - Ownership: the caller owns every buffer.  The library allocates no
  *     device or host memory and keeps no per-call state.
- *   - Pointers are DEVICE pointers unless stated otherwise, 16-byte aligned.
+ *   - Pointers are DEVICE pointers unless stated otherwise.  Array pointers
+ *     (W, packed, x, xq, y, acc, workspace) must be 16-byte aligned; the
+ *     scalar-per-token pointers (alpha, amax, xsum) 4-byte aligned.
  *   - Shapes: K must be a positive multiple of 128 and at most 131072; M >= 1
  *     (a multiple of 128 for bitlinear_gemm); M*K <= 2^40.  N = 0 is a no-op.
  *   - Every call is asynchronous on `stream` (NULL = the legacy default
@@ -143,6 +145,33 @@ BITLINEAR_API bitlinear_status bitlinear_gemm(const uint32_t* packed, const floa
                                 const int8_t* xq, const float* amax, const int32_t* xsum,
                                 int64_t N, float* y, int32_t* acc,
                                 bitlinear_stream_t stream);
+
+/*
+ * One linear layer of a grouped decode call.  Every pointer follows the
+ * conventions above; all problems of one call share K and N.
+ */
+typedef struct {
+    const uint32_t* packed;   /* [M, K/16] words */
+    const float* alpha;       /* [1] */
+    int64_t M;
+    const int8_t* xq;         /* [N, K] */
+    const float* amax;        /* [N] */
+    const int32_t* xsum;      /* [N] */
+    float* y;                 /* [N, M] output */
+    int32_t* acc;             /* [N, M] output, or NULL */
+} bitlinear_problem;
+
+/*
+ * Decode GEMV over a list of independent layers in as few launches as
+ * possible (one per 256 problems): the same arithmetic as bitlinear_gemv for
+ * each entry.  Meant for layers that read activations known at the same time
+ * -- the q/k/v or gate/up projections of one decoder layer, or a stream of
+ * layers whose inputs are all available.  `problems` is a HOST array of
+ * `count` entries, read during the call only.  1 <= N <= 16.
+ */
+BITLINEAR_API bitlinear_status bitlinear_gemv_grouped(const bitlinear_problem* problems,
+                                                      int64_t count, int64_t K, int64_t N,
+                                                      bitlinear_stream_t stream);
 
 /* ------------------------------------------------------------ diagnostics */
 

@@ -72,6 +72,34 @@ def gemv(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out
                    with_acc, stream, out)
 
 
+def gemv_grouped(layers, xq, amax, xsum, with_acc=False, stream=None, outs=None):
+    """One grouped decode call over several layers that share K and the token
+    count.  layers: list of (packed, alpha); xq/amax/xsum: one tensor for all
+    layers, or a list with one entry per layer.  Returns a list of y (and acc)."""
+    n = len(layers)
+    xqs = xq if isinstance(xq, (list, tuple)) else [xq] * n
+    amaxs = amax if isinstance(amax, (list, tuple)) else [amax] * n
+    xsums = xsum if isinstance(xsum, (list, tuple)) else [xsum] * n
+    N, K = xqs[0].shape
+    ys, accs, entries = [], [], []
+    for i, (packed, alpha) in enumerate(layers):
+        _need(packed, torch.int32, "packed")
+        _need(alpha, torch.float32, "alpha")
+        _need(xqs[i], torch.int8, "xq")
+        if tuple(xqs[i].shape) != (N, K) or packed.shape[1] != K // 16:
+            raise ValueError("all layers of a grouped call share K and N")
+        M = packed.shape[0]
+        y = outs[i] if outs is not None else torch.empty((N, M), dtype=torch.float32,
+                                                           device=packed.device)
+        acc = torch.empty((N, M), dtype=torch.int32, device=packed.device) if with_acc else None
+        ys.append(y)
+        accs.append(acc)
+        entries.append((packed, alpha, M, xqs[i], amaxs[i], xsums[i], y, acc))
+    arr = _lib.make_problems(entries)
+    _lib.check(_lib.bitlinear_gemv_grouped(arr, n, K, N, stream), "bitlinear_gemv_grouped")
+    return (ys, accs) if with_acc else ys
+
+
 def gemm(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out=None):
     """Tensor-core GEMM (any N, M % 128 == 0): y[N,M] fp32 (and int32 acc)."""
     M = packed.shape[0] if M is None else M

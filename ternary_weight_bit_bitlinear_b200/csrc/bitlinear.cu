@@ -20,6 +20,7 @@ constexpr int64_t kMaxElems = int64_t(1) << 40;
 constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bitlinear_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
@@ -36,6 +37,7 @@ bitlinear_status check_mk(int64_t M, int64_t K) {
 struct DeviceInfo {
   int sms = 0;
   bool gemm_attr_set[2] = {false, false};
+  bool stream_attr_set[bl::kStreamMaxTokens + 1][17] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -85,14 +87,144 @@ bool encode_u8_2d(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t row
 }
 
 template <int NT>
-void launch_gemv(const uint32_t* packed, const float* alpha, int M, int K, const int8_t* xq,
-                 const float* amax, const int32_t* xsum, float* y, int32_t* acc,
-                 cudaStream_t s) {
+void launch_gemv_generic(const bitlinear_problem& q, int K, cudaStream_t s) {
+  const int M = static_cast<int>(q.M);
   const int rows_per_block = (bl::kGemvThreads / 32) * bl::kGemvRows;
   const int grid = (M + rows_per_block - 1) / rows_per_block;
-  bl::gemv_kernel<NT><<<grid, bl::kGemvThreads, 0, s>>>(
-      reinterpret_cast<const uint4*>(packed), M, K / 64, reinterpret_cast<const uint4*>(xq),
-      alpha, amax, xsum, y, acc);
+  bl::gemv_generic_kernel<NT><<<grid, bl::kGemvThreads, 0, s>>>(
+      reinterpret_cast<const uint4*>(q.packed), M, K / 64, reinterpret_cast<const uint4*>(q.xq),
+      q.alpha, q.amax, q.xsum, q.y, q.acc);
+}
+
+void launch_gemv_generic_n(const bitlinear_problem& q, int K, int N, cudaStream_t s) {
+  switch (N) {
+#define BL_GEMV_CASE(n) \
+  case n: launch_gemv_generic<n>(q, K, s); break;
+    BL_GEMV_CASE(1) BL_GEMV_CASE(2) BL_GEMV_CASE(3) BL_GEMV_CASE(4)
+    BL_GEMV_CASE(5) BL_GEMV_CASE(6) BL_GEMV_CASE(7) BL_GEMV_CASE(8)
+    BL_GEMV_CASE(9) BL_GEMV_CASE(10) BL_GEMV_CASE(11) BL_GEMV_CASE(12)
+    BL_GEMV_CASE(13) BL_GEMV_CASE(14) BL_GEMV_CASE(15) BL_GEMV_CASE(16)
+#undef BL_GEMV_CASE
+    default: break;
+  }
+}
+
+// Streaming GEMV plan for one K: k-slices per row and spans (32 words) per
+// slice, with spans * N <= 12 so a lane's activations fit in 48 registers.
+struct StreamPlan {
+  bool ok = false;
+  int ksplit = 1, spans = 1, rows_per_stage = 1;
+};
+
+StreamPlan stream_plan(int64_t K, int64_t N) {
+  StreamPlan pl;
+  if (N < 1 || N > bl::kStreamMaxTokens) return pl;
+  const int64_t W = K / 16;
+  if (W * 4 > bl::kStreamStageBytes) return pl;
+  const int64_t nspan = (W + 31) / 32;
+  const int64_t cap = 12 / N;
+  int ks = 1;
+  while (ks * cap < nspan) ks *= 2;
+  if (ks > bl::kStreamConsumerWarps) return pl;
+  pl.ksplit = ks;
+  pl.spans = static_cast<int>((nspan + ks - 1) / ks);
+  pl.rows_per_stage = static_cast<int>(bl::kStreamStageBytes / (W * 4));
+  pl.ok = true;
+  return pl;
+}
+
+template <int NT, int S>
+bitlinear_status launch_stream_ns(const bl::GemvParams& p, int grid, DeviceInfo* dev,
+                                  cudaStream_t s) {
+  auto kernel = bl::gemv_stream_kernel<NT, S>;
+  constexpr int smem = static_cast<int>(bl::stream_smem_bytes());
+  if (!dev->stream_attr_set[NT][S]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    dev->stream_attr_set[NT][S] = true;
+  }
+  kernel<<<grid, bl::kStreamThreads, smem, s>>>(p);
+  return launch_status();
+}
+
+template <int NT, int S>
+bitlinear_status launch_stream_s(int spans, const bl::GemvParams& p, int grid, DeviceInfo* dev,
+                                 cudaStream_t s) {
+  if constexpr (S > 12 / NT) {
+    return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  } else {
+    if (spans == S) return launch_stream_ns<NT, S>(p, grid, dev, s);
+    return launch_stream_s<NT, S + 1>(spans, p, grid, dev, s);
+  }
+}
+
+bitlinear_status launch_stream(int N, int spans, const bl::GemvParams& p, int grid,
+                               DeviceInfo* dev, cudaStream_t s) {
+  switch (N) {
+    case 1: return launch_stream_s<1, 1>(spans, p, grid, dev, s);
+    case 2: return launch_stream_s<2, 1>(spans, p, grid, dev, s);
+    case 3: return launch_stream_s<3, 1>(spans, p, grid, dev, s);
+    case 4: return launch_stream_s<4, 1>(spans, p, grid, dev, s);
+    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
+// Decode GEMV over problems that share K and N (all validated).
+bitlinear_status gemv_group(const bitlinear_problem* probs, int64_t count, int64_t K, int64_t N,
+                            cudaStream_t s) {
+  const StreamPlan pl = stream_plan(K, N);
+  if (!pl.ok) {
+    for (int64_t i = 0; i < count; ++i)
+      launch_gemv_generic_n(probs[i], static_cast<int>(K), static_cast<int>(N), s);
+    return launch_status();
+  }
+  DeviceInfo* dev = nullptr;
+  bitlinear_status st = device_info(&dev);
+  if (st != BITLINEAR_OK) return st;
+  const int grid_cap = dev->sms * 2;
+  int64_t total_rows = 0;
+  for (int64_t i = 0; i < count; ++i) total_rows += probs[i].M;
+  // Units of consecutive rows: about 8 per resident CTA for balance, a whole
+  // number of stages when longer than one stage.
+  const int RS = pl.rows_per_stage;
+  int64_t ur = (total_rows + 8 * grid_cap - 1) / (8 * grid_cap);
+  if (ur > RS) ur = (ur + RS - 1) / RS * RS;
+  const int64_t ur_cap = bl::kStreamMaxUnitRows / RS * RS;
+  if (ur > ur_cap) ur = ur_cap;
+  if (ur < 1) ur = 1;
+  for (int64_t base = 0; base < count; base += bl::kStreamMaxProblems) {
+    const int n = static_cast<int>(count - base < bl::kStreamMaxProblems
+                                       ? count - base : bl::kStreamMaxProblems);
+    bl::GemvParams p;
+    memset(&p, 0, sizeof p);
+    int units = 0;
+    for (int i = 0; i < n; ++i) {
+      const bitlinear_problem& q = probs[base + i];
+      bl::GemvProblem& g = p.prob[i];
+      g.packed = q.packed;
+      g.alpha = q.alpha;
+      g.xq = q.xq;
+      g.amax = q.amax;
+      g.xsum = q.xsum;
+      g.y = q.y;
+      g.acc = q.acc;
+      g.M = static_cast<int>(q.M);
+      g.unit_begin = units;
+      units += static_cast<int>((q.M + ur - 1) / ur);
+    }
+    p.num_problems = n;
+    p.total_units = units;
+    p.K = static_cast<int>(K);
+    p.W = static_cast<int>(K / 16);
+    p.rows_per_stage = RS;
+    p.unit_rows = static_cast<int>(ur);
+    p.ksplit = pl.ksplit;
+    const int grid = units < grid_cap ? units : grid_cap;
+    st = launch_stream(static_cast<int>(N), pl.spans, p, grid, dev, s);
+    if (st != BITLINEAR_OK) return st;
+  }
+  return BITLINEAR_OK;
 }
 
 template <int BN, int STAGES>
@@ -121,7 +253,7 @@ bitlinear_status check_matmul_args(const uint32_t* packed, const float* alpha, i
   if (!packed || !alpha || !xq || !amax || !xsum || !y) return BITLINEAR_ERR_INVALID_ARG;
   if (!aligned16(packed) || !aligned16(xq) || !aligned16(y) || (acc && !aligned16(acc)))
     return BITLINEAR_ERR_MISALIGNED;
-  if (!aligned16(alpha) || !aligned16(amax) || !aligned16(xsum)) return BITLINEAR_ERR_MISALIGNED;
+  if (!aligned4(alpha) || !aligned4(amax) || !aligned4(xsum)) return BITLINEAR_ERR_MISALIGNED;
   return BITLINEAR_OK;
 }
 
@@ -157,7 +289,7 @@ bitlinear_status bitlinear_pack_weights(const float* W, int64_t M, int64_t K, ui
   if (st != BITLINEAR_OK) return st;
   if (!W || !packed || !alpha) return BITLINEAR_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < bl::kPackWorkspaceBytes) return BITLINEAR_ERR_WORKSPACE;
-  if (!aligned16(W) || !aligned16(packed) || !aligned16(workspace) || !aligned16(alpha))
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(workspace) || !aligned4(alpha))
     return BITLINEAR_ERR_MISALIGNED;
   DeviceInfo* dev = nullptr;
   if ((st = device_info(&dev)) != BITLINEAR_OK) return st;
@@ -185,7 +317,7 @@ bitlinear_status bitlinear_quant_act(const float* x, int64_t N, int64_t K, int8_
   if (K == 0 || K % 128 != 0 || K > kMaxK || N > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   if (N == 0) return BITLINEAR_OK;
   if (!x || !xq || !amax) return BITLINEAR_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(xq) || !aligned16(amax) || (xsum && !aligned16(xsum)))
+  if (!aligned16(x) || !aligned16(xq) || !aligned4(amax) || (xsum && !aligned4(xsum)))
     return BITLINEAR_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   bl::quant_act_kernel<<<static_cast<int>(N), bl::kQuantThreads, 0, s>>>(x, static_cast<int>(K),
@@ -199,19 +331,22 @@ bitlinear_status bitlinear_gemv(const uint32_t* packed, const float* alpha, int6
   bitlinear_status st = check_matmul_args(packed, alpha, M, K, xq, amax, xsum, N, y, acc);
   if (st != BITLINEAR_OK || N == 0) return st;
   if (N > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int m = static_cast<int>(M), k = static_cast<int>(K);
-  switch (N) {
-#define BL_GEMV_CASE(n) \
-  case n: launch_gemv<n>(packed, alpha, m, k, xq, amax, xsum, y, acc, s); break;
-    BL_GEMV_CASE(1) BL_GEMV_CASE(2) BL_GEMV_CASE(3) BL_GEMV_CASE(4)
-    BL_GEMV_CASE(5) BL_GEMV_CASE(6) BL_GEMV_CASE(7) BL_GEMV_CASE(8)
-    BL_GEMV_CASE(9) BL_GEMV_CASE(10) BL_GEMV_CASE(11) BL_GEMV_CASE(12)
-    BL_GEMV_CASE(13) BL_GEMV_CASE(14) BL_GEMV_CASE(15) BL_GEMV_CASE(16)
-#undef BL_GEMV_CASE
-    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  const bitlinear_problem q = {packed, alpha, M, xq, amax, xsum, y, acc};
+  return gemv_group(&q, 1, K, N, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitlinear_status bitlinear_gemv_grouped(const bitlinear_problem* problems, int64_t count,
+                                        int64_t K, int64_t N, bitlinear_stream_t stream) {
+  if (count < 0 || N < 0 || (count > 0 && !problems)) return BITLINEAR_ERR_INVALID_ARG;
+  if (count == 0 || N == 0) return BITLINEAR_OK;
+  if (N > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  for (int64_t i = 0; i < count; ++i) {
+    const bitlinear_problem& q = problems[i];
+    bitlinear_status st = check_matmul_args(q.packed, q.alpha, q.M, K, q.xq, q.amax, q.xsum, N,
+                                            q.y, q.acc);
+    if (st != BITLINEAR_OK) return st;
   }
-  return launch_status();
+  return gemv_group(problems, count, K, N, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bitlinear_status bitlinear_gemm(const uint32_t* packed, const float* alpha, int64_t M, int64_t K,

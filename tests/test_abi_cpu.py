@@ -121,3 +121,22 @@ def test_header_is_self_contained(tmp_path):
     inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, "-c", str(src), "-o",
                     str(tmp_path / "t.o")], check=True)
+
+
+def test_gemv_grouped_argument_errors(L):
+    f = L.bitlinear_gemv_grouped
+    P = _lib.Problem
+    good = P(FAKE, FAKE, 128, FAKE, FAKE, FAKE, FAKE, 0)
+    arr = (P * 2)(good, good)
+    assert f(arr, -1, 256, 1, None) == _lib.ERR_INVALID_ARG
+    assert f(None, 2, 256, 1, None) == _lib.ERR_INVALID_ARG
+    assert f(arr, 0, 256, 1, None) == _lib.OK
+    assert f(arr, 2, 256, 0, None) == _lib.OK
+    assert f(arr, 2, 256, 17, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert f(arr, 2, 200, 1, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    bad = (P * 2)(good, P(FAKE, FAKE, 128, FAKE, FAKE, FAKE, MISALIGNED, 0))
+    assert f(bad, 2, 256, 1, None) == _lib.ERR_MISALIGNED
+    bad = (P * 2)(good, P(FAKE, 0, 128, FAKE, FAKE, FAKE, FAKE, 0))
+    assert f(bad, 2, 256, 1, None) == _lib.ERR_INVALID_ARG
+    bad = (P * 2)(good, P(FAKE, FAKE + 2, 128, FAKE, FAKE, FAKE, FAKE, 0))
+    assert f(bad, 2, 256, 1, None) == _lib.ERR_MISALIGNED

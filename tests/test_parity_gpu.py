@@ -146,6 +146,40 @@ def test_gemv_parity_shapes(M, K, N):
     assert_y_close(y.cpu().numpy(), ref["y"])
 
 
+@pytest.mark.parametrize("N", [1, 2, 3, 4, 7])
+@pytest.mark.parametrize("K", [1024, 2560, 6912, 28672])
+def test_gemv_grouped_parity(K, N):
+    Ms = [640, 128, 2560, 300]
+    layers, refs = [], []
+    x = inputs.activations(N, K, seed=K + N, outlier_frac=0.01)
+    for i, M in enumerate(Ms):
+        W = inputs.latent_weights(M, K, seed=1000 * i + K + N)
+        refs.append(oracle.bitlinear(W.numpy(), x.numpy()))
+        layers.append(api.pack_weights(W.cuda()))
+    xq, amax, xsum = api.quant_act(x.cuda())
+    ys, accs = api.gemv_grouped(layers, xq, amax, xsum, with_acc=True)
+    for y, acc, ref in zip(ys, accs, refs):
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+        assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
+def test_gemv_grouped_many_problems_and_row_views():
+    # 150 problems (more than one launch's table), activations as row views of
+    # one stacked buffer (4-byte aligned amax/xsum pointers)
+    K, M = 512, 256
+    X = inputs.activations(150, K, seed=31)
+    xq, amax, xsum = api.quant_act(X.cuda())
+    W = inputs.latent_weights(M, K, seed=32)
+    packed, alpha = api.pack_weights(W.cuda())
+    ys, accs = api.gemv_grouped([(packed, alpha)] * 150, [xq[i:i + 1] for i in range(150)],
+                                [amax[i:i + 1] for i in range(150)],
+                                [xsum[i:i + 1] for i in range(150)], with_acc=True)
+    ref = oracle.bitlinear(W.numpy(), X.numpy())
+    got = torch.cat(accs).cpu().numpy()
+    assert np.array_equal(got, ref["acc"])
+    assert np.array_equal(torch.cat(ys).cpu().numpy(), ref["y"])
+
+
 @pytest.mark.parametrize("M,K,N", [(128, 128, 1), (256, 512, 200), (384, 1024, 129),
                                    (128, 256, 16), (1024, 2560, 512), (512, 4096, 300),
                                    (256, 6912, 77)])
