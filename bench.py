@@ -269,6 +269,61 @@ def flush_l2(buf):
     buf.zero_()
 
 
+def measure_prefill(dev, s, peaks, K):
+    """7B-shaped layer at N=512 on the tensor cores: GEMM time from events
+    around the seven launches, L2 flushed before every timed step."""
+    pre = PrefillWorkload(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        for i in range(4):
+            pre.quant(i, s)
+        for p in range(7):
+            pre.gemm(p, s)
+    torch.cuda.synchronize()
+    P = max(10, min(200, K // 50))
+    gemm_ms, quant_ms, step_ms = 0.0, 0.0, 0.0
+    per_proj = [0.0] * 7
+    for _ in range(P):
+        flush_l2(flush)
+        e = events(13)
+        e[0].record(s)
+        for i in range(4):
+            pre.quant(i, s)
+        e[1].record(s)
+        for p in range(7):
+            pre.gemm(p, s)
+            e[2 + p].record(s)
+        torch.cuda.synchronize()
+        quant_ms += e[0].elapsed_time(e[1])
+        prev = e[1]
+        for p in range(7):
+            per_proj[p] += prev.elapsed_time(e[2 + p])
+            prev = e[2 + p]
+        gemm_ms += e[1].elapsed_time(e[8])
+        step_ms += e[0].elapsed_time(e[8])
+    gemm_ms /= P
+    quant_ms /= P
+    step_ms /= P
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    tops = pre.flops / (gemm_ms * 1e-3) / 1e12
+    prefill = {
+        "workload": "7B-shaped layer, 7 projections (q,k,v,o 4096x4096; gate/up 11008x4096; "
+                    "down 4096x11008), N=512 tokens",
+        "value": round(tops, 1), "unit": "int8 TOPS",
+        "gemm_ms": round(gemm_ms, 4), "quant_ms": round(quant_ms, 4),
+        "step_tops_incl_quant": round(pre.flops / (step_ms * 1e-3) / 1e12, 1),
+        "per_projection_ms": [round(v / P, 4) for v in per_proj],
+        "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(int8_peak, 1),
+                     "unit": "TOPS", "frac": round(tops / int8_peak, 4),
+                     "peak_note": "int8 peak = measured bf16 burst x nominal int8:bf16 ratio 2 (%s)"
+                                  % peaks["source"],
+                     "frac_of_nominal_4500": round(tops / 4500.0, 4), "traffic": None},
+        "l2": "256 MB buffer written between timed steps (flush)",
+    }
+    del flush
+    return prefill
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -294,6 +349,10 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return t.item()
 
+    if args.only == "prefill":
+        print(json.dumps({"partial_run": "prefill", "prefill": measure_prefill(dev, s, peaks,
+                                                                              args.steps)}))
+        return
     dec = DecodeWorkload(dev)
     for _ in range(args.warmup):
         dec.step(s)
@@ -336,6 +395,10 @@ def run_ours(args, rank, world, local_rank):
     gbs = world * dec.packed_bytes / (ms_per_step * 1e-3) / 1e9
     gemv_h_gbs = dec.alg_bytes_h / (per["gemv_h"] * 1e-3) / 1e9
     hbm_peak = peaks["hbm_gbs"]
+    if args.only == "decode":
+        print(json.dumps({"partial_run": "decode", "value": round(gbs, 1), "unit": "GB/s",
+                          "kernel_ms": per, "gemv_h_gbs": round(gemv_h_gbs, 1), "clocks": clk}))
+        return
 
     # ---- dependent per-layer chain, CUDA graph
     chain_ms = None
@@ -389,56 +452,7 @@ def run_ours(args, rank, world, local_rank):
     h2d = (dec.Xh.numel() + dec.Xf.numel()) * 4
     d2h = dec.Y.numel() * 4
 
-    # ---- prefill: 7B-shaped layer at N=512 on the tensor cores
-    pre = PrefillWorkload(dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    for _ in range(3):
-        for i in range(4):
-            pre.quant(i, s)
-        for p in range(7):
-            pre.gemm(p, s)
-    torch.cuda.synchronize()
-    P = max(10, min(200, K // 50))
-    gemm_ms, quant_ms, step_ms = 0.0, 0.0, 0.0
-    per_proj = [0.0] * 7
-    for _ in range(P):
-        flush_l2(flush)
-        e = events(13)
-        e[0].record(s)
-        for i in range(4):
-            pre.quant(i, s)
-        e[1].record(s)
-        for p in range(7):
-            pre.gemm(p, s)
-            e[2 + p].record(s)
-        torch.cuda.synchronize()
-        quant_ms += e[0].elapsed_time(e[1])
-        prev = e[1]
-        for p in range(7):
-            per_proj[p] += prev.elapsed_time(e[2 + p])
-            prev = e[2 + p]
-        gemm_ms += e[1].elapsed_time(e[8])
-        step_ms += e[0].elapsed_time(e[8])
-    gemm_ms /= P
-    quant_ms /= P
-    step_ms /= P
-    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
-    tops = pre.flops / (gemm_ms * 1e-3) / 1e12
-    prefill = {
-        "workload": "7B-shaped layer, 7 projections (q,k,v,o 4096x4096; gate/up 11008x4096; "
-                    "down 4096x11008), N=512 tokens",
-        "value": round(tops, 1), "unit": "int8 TOPS",
-        "gemm_ms": round(gemm_ms, 4), "quant_ms": round(quant_ms, 4),
-        "step_tops_incl_quant": round(pre.flops / (step_ms * 1e-3) / 1e12, 1),
-        "per_projection_ms": [round(v / P, 4) for v in per_proj],
-        "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(int8_peak, 1),
-                     "unit": "TOPS", "frac": round(tops / int8_peak, 4),
-                     "peak_note": "int8 peak = measured bf16 burst x nominal int8:bf16 ratio 2 (%s)"
-                                  % peaks["source"],
-                     "frac_of_nominal_4500": round(tops / 4500.0, 4), "traffic": None},
-        "l2": "256 MB buffer written between timed steps (flush)",
-    }
-    del flush
+    prefill = measure_prefill(dev, s, peaks, K)
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
     cpu = None
@@ -611,6 +625,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "decode", "prefill"], default="all",
+                    help="profiling runs: time only one part and print a partial line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
