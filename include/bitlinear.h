@@ -173,6 +173,38 @@ BITLINEAR_API bitlinear_status bitlinear_gemv_grouped(const bitlinear_problem* p
                                                       int64_t count, int64_t K, int64_t N,
                                                       bitlinear_stream_t stream);
 
+/* ------------------------------------------------- weights, no allocation */
+
+/*
+ * bitlinear_pack_weights for callers that cannot allocate device memory at
+ * all -- not even the small workspace the entry point above asks for.  Typical
+ * cases: a plugin inside a host process (an inference server, a game engine)
+ * that owns the whole device memory budget through its own pool and forbids
+ * its libraries from calling cudaMalloc; or a latency-critical path where
+ * cudaMalloc/cudaFree are unacceptable because they can synchronise the
+ * device.  The pages describe no such entry point; it exists only for these
+ * callers.
+ *
+ * Same arguments, results and errors as bitlinear_pack_weights minus the
+ * workspace: the exponent bins live in a fixed 2064-byte array that the
+ * library keeps in device global memory (one copy per GPU that loads the
+ * library, held until the process exits).  That array bounds nothing but the
+ * element count: M*K must not exceed 2^40 (BITLINEAR_ERR_UNSUPPORTED_SHAPE
+ * otherwise), the same limit as the workspace version.  The array is cleared
+ * on the stream at the start of every call.
+ *
+ * The first call on each device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  The call
+ * allocates nothing, host or device.  All calls on one device share the array:
+ * calls whose work may overlap on the GPU (different streams without ordering
+ * between them) race and give wrong results; order them on one stream, or use
+ * bitlinear_pack_weights with separate workspaces.
+ */
+BITLINEAR_API bitlinear_status bitlinear_pack_weights_noalloc(const float* W, int64_t M,
+                                                              int64_t K, uint32_t* packed,
+                                                              float* alpha,
+                                                              bitlinear_stream_t stream);
+
 /* ------------------------------------------------------------ diagnostics */
 
 /*

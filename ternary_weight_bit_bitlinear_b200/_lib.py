@@ -55,6 +55,8 @@ def load(path: str = LIB_PATH):
     L.bitlinear_pack_workspace_bytes.restype = sz
     L.bitlinear_pack_weights.argtypes = [p, i64, i64, p, p, p, sz, p]
     L.bitlinear_pack_weights.restype = st
+    L.bitlinear_pack_weights_noalloc.argtypes = [p, i64, i64, p, p, p]
+    L.bitlinear_pack_weights_noalloc.restype = st
     L.bitlinear_quant_act.argtypes = [p, i64, i64, p, p, p, p]
     L.bitlinear_quant_act.restype = st
     for name in ("bitlinear_gemv", "bitlinear_gemm"):
@@ -102,6 +104,11 @@ def _stream(stream):
 def bitlinear_pack_weights(W, M, K, packed, alpha, workspace, workspace_bytes, stream=None):
     return load().bitlinear_pack_weights(_p(W), M, K, _p(packed), _p(alpha), _p(workspace),
                                          workspace_bytes, _stream(stream))
+
+
+def bitlinear_pack_weights_noalloc(W, M, K, packed, alpha, stream=None):
+    return load().bitlinear_pack_weights_noalloc(_p(W), M, K, _p(packed), _p(alpha),
+                                                 _stream(stream))
 
 
 def bitlinear_quant_act(x, N, K, xq, amax, xsum, stream=None):

@@ -399,3 +399,46 @@ bitlinear_status bitlinear_device_error(int* status_out, int clear) {
 }
 
 }  // extern "C"
+// ---------------------------------------------------------------- no-alloc pack
+// Scratch of bitlinear_pack_weights_noalloc: the exponent bins and flag word
+// that bitlinear_pack_weights otherwise takes as workspace.  One copy per
+// device, shared by every call on that device.
+static __device__ __align__(256) unsigned char g_noalloc_pack_scratch[bl::kPackWorkspaceBytes];
+
+namespace {
+void* g_noalloc_pack_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array for the current device.  Host code may
+// not pass the symbol itself to a kernel: on the host it names a stand-in,
+// not device memory.  Looked up once per device, with that device current.
+bitlinear_status noalloc_pack_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return BITLINEAR_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_pack_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_pack_scratch) != cudaSuccess || !p)
+      return BITLINEAR_ERR_CUDA;
+    g_noalloc_pack_ptr[dev] = p;
+  }
+  *out = g_noalloc_pack_ptr[dev];
+  return BITLINEAR_OK;
+}
+}  // namespace
+
+extern "C" bitlinear_status bitlinear_pack_weights_noalloc(const float* W, int64_t M, int64_t K,
+                                                           uint32_t* packed, float* alpha,
+                                                           bitlinear_stream_t stream) {
+  // Argument checks first, so a bad call touches no CUDA state.  check_mk
+  // rejects M*K > 2^40, beyond which the fixed bins could overflow.
+  bitlinear_status st = check_mk(M, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!W || !packed || !alpha) return BITLINEAR_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(packed) || !aligned4(alpha)) return BITLINEAR_ERR_MISALIGNED;
+  void* scratch = nullptr;
+  if ((st = noalloc_pack_scratch(&scratch)) != BITLINEAR_OK) return st;
+  return bitlinear_pack_weights(W, M, K, packed, alpha, scratch, sizeof(g_noalloc_pack_scratch),
+                                stream);
+}
