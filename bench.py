@@ -9,7 +9,7 @@ BitLinear projections (q 2560x2560, k/v 640x2560, o 2560x2560, gate/up
 6912x2560, down 2560x6912), every linear fed one token.  One step:
 
     quant_act(90 x 2560 activation rows)   quant_act(30 x 6912 rows)
-    gemv_grouped(180 layers, K=2560)       gemv_grouped(30 layers, K=6912)
+    gemv_grouped(all 210 layers, one launch)
 
 i.e. per-token absmax int8 quantisation of every layer input and the ternary x
 int8 GEMV with fused rescale of every projection; the 521 MB of packed weights
@@ -149,35 +149,28 @@ class DecodeWorkload:
         self.Y = torch.empty(L * per_layer, device=device)   # all outputs, one buffer
         self.ys = []
         off = 0
-        group_h, group_f = [], []
-        self.chain = []              # per layer: list of (kind, args) launch groups
+        entries = []
         for l in range(L):
             ys_l = []
             for p, (packed, alpha, M, K) in enumerate(self.weights[l]):
                 y = self.Y[off:off + M].view(1, M)
                 off += M
                 ys_l.append(y)
-                if K == h:
-                    r = 3 * l + (0 if p < 3 else 1 if p == 3 else 2)
-                    e = (packed, alpha, M, self.XQh[r:r + 1], self.AMh[r:r + 1],
-                         self.XSh[r:r + 1], y, None)
-                    group_h.append(e)
-                else:
-                    e = (packed, alpha, M, self.XQf[l:l + 1], self.AMf[l:l + 1],
-                         self.XSf[l:l + 1], y, None)
-                    group_f.append(e)
+                entries.append((packed, alpha, M, K) + self._act(l, p) + (y, None))
             self.ys.append(ys_l)
-        self.prob_h = _lib.make_problems(group_h)
-        self.prob_f = _lib.make_problems(group_f)
-        self.n_h, self.n_f = len(group_h), len(group_f)
+        self.prob = _lib.make_problems(entries)
+        self.n_prob = len(entries)
         self.packed_bytes = sum(M * K // 4 for row in self.weights for _, _, M, K in row)
-        self.packed_bytes_h = sum(M * K // 4 for row in self.weights for _, _, M, K in row
-                                  if K == h)
-        # algorithmic bytes of each grouped GEMV launch: packed weights, the
-        # int8 activations, alpha/amax/xsum and the fp32 outputs of its layers
-        self.alg_bytes_h = sum(e[2] * h // 4 + h + 12 + 4 * e[2] for e in group_h)
-        self.alg_bytes_f = sum(e[2] * f // 4 + f + 12 + 4 * e[2] for e in group_f)
-        self._entries_h, self._entries_f = group_h, group_f
+        # algorithmic bytes of the grouped GEMV launch: packed weights, the int8
+        # activations and alpha/amax/xsum each layer reads, and its fp32 outputs
+        self.alg_bytes = sum(M * K // 4 + K + 12 + 4 * M for (_, _, M, K, *_r) in entries)
+
+    def _act(self, l, p):
+        """(xq, amax, xsum) row views of the input projection p of layer l reads."""
+        if p == 6:
+            return (self.XQf[l:l + 1], self.AMf[l:l + 1], self.XSf[l:l + 1])
+        r = 3 * l + (0 if p < 3 else 1 if p == 3 else 2)
+        return (self.XQh[r:r + 1], self.AMh[r:r + 1], self.XSh[r:r + 1])
 
     # each call launches exactly one kernel
     def quant_h(self, s):
@@ -188,42 +181,32 @@ class DecodeWorkload:
         _lib.check(_lib.bitlinear_quant_act(self.Xf, self.Xf.shape[0], self.Xf.shape[1],
                                             self.XQf, self.AMf, self.XSf, s), "quant_act")
 
-    def gemv_h(self, s):
-        _lib.check(_lib.bitlinear_gemv_grouped(self.prob_h, self.n_h, self.shape.hidden, 1, s),
-                   "gemv_grouped")
-
-    def gemv_f(self, s):
-        _lib.check(_lib.bitlinear_gemv_grouped(self.prob_f, self.n_f, self.shape.ffn, 1, s),
-                   "gemv_grouped")
+    def gemv(self, s):
+        _lib.check(_lib.bitlinear_gemv_grouped(self.prob, self.n_prob, 1, s), "gemv_grouped")
 
     def step(self, s):
         self.quant_h(s)
         self.quant_f(s)
-        self.gemv_h(s)
-        self.gemv_f(s)
+        self.gemv(s)
 
     def chain_step(self, s):
         """The order a real decoder imposes: per layer, quantise an input, then
         run the projections that read it, one group after the other."""
-        h = self.shape.hidden
+        h, f = self.shape.hidden, self.shape.ffn
         for l in range(self.layers):
             w = self.weights[l]
-            for (r, projs) in ((3 * l, (0, 1, 2)), (3 * l + 1, (3,)), (3 * l + 2, (4, 5))):
-                _lib.check(_lib.bitlinear_quant_act(self.Xh[r:r + 1], 1, h, self.XQh[r:r + 1],
-                                                    self.AMh[r:r + 1], self.XSh[r:r + 1], s),
-                           "quant_act")
-                ents = [(w[p][0], w[p][1], w[p][2], self.XQh[r:r + 1], self.AMh[r:r + 1],
-                         self.XSh[r:r + 1], self.ys[l][p], None) for p in projs]
+            for projs in ((0, 1, 2), (3,), (4, 5), (6,)):
+                K = w[projs[0]][3]
+                if projs[0] == 6:
+                    x, xq, am, xs = self.Xf[l:l + 1], *self._act(l, 6)
+                else:
+                    r = 3 * l + (0 if projs[0] < 3 else 1 if projs[0] == 3 else 2)
+                    x, xq, am, xs = self.Xh[r:r + 1], *self._act(l, projs[0])
+                _lib.check(_lib.bitlinear_quant_act(x, 1, K, xq, am, xs, s), "quant_act")
+                ents = [(w[p][0], w[p][1], w[p][2], K, xq, am, xs, self.ys[l][p], None)
+                        for p in projs]
                 arr = _lib.make_problems(ents)
-                _lib.check(_lib.bitlinear_gemv_grouped(arr, len(ents), h, 1, s), "gemv_grouped")
-            f = self.shape.ffn
-            _lib.check(_lib.bitlinear_quant_act(self.Xf[l:l + 1], 1, f, self.XQf[l:l + 1],
-                                                self.AMf[l:l + 1], self.XSf[l:l + 1], s),
-                       "quant_act")
-            arr = _lib.make_problems([(w[6][0], w[6][1], w[6][2], self.XQf[l:l + 1],
-                                       self.AMf[l:l + 1], self.XSf[l:l + 1], self.ys[l][6],
-                                       None)])
-            _lib.check(_lib.bitlinear_gemv_grouped(arr, 1, f, 1, s), "gemv_grouped")
+                _lib.check(_lib.bitlinear_gemv_grouped(arr, len(ents), 1, s), "gemv_grouped")
 
 
 class PrefillWorkload:
@@ -246,6 +229,14 @@ class PrefillWorkload:
         self.src = [0, 0, 0, 1, 2, 2, 3]       # which input each projection reads
         self.Y = [torch.empty((N, M), device=device) for (_, _, M, _) in self.weights]
         self.flops = sum(2 * M * N * K for (_, _, M, K) in self.weights)
+        self._make_problems()
+
+    def _make_problems(self):
+        ents = []
+        for p, (packed, alpha, M, K) in enumerate(self.weights):
+            xq, am, xs = self.Q[self.src[p]]
+            ents.append((packed, alpha, M, K, xq, am, xs, self.Y[p], None))
+        self.prob = _lib.make_problems(ents)
 
     def quant(self, i, s):
         x = self.X[i]
@@ -253,10 +244,15 @@ class PrefillWorkload:
         _lib.check(_lib.bitlinear_quant_act(x, x.shape[0], x.shape[1], xq, am, xs, s), "quant")
 
     def gemm(self, p, s):
+        """One projection alone (for the per-projection breakdown)."""
         packed, alpha, M, K = self.weights[p]
         xq, am, xs = self.Q[self.src[p]]
         _lib.check(_lib.bitlinear_gemm(packed, alpha, M, K, xq, am, xs, self.N, self.Y[p],
                                        None, s), "gemm")
+
+    def gemm_all(self, s):
+        """All seven projections in one grouped launch."""
+        _lib.check(_lib.bitlinear_gemm_grouped(self.prob, 7, self.N, s), "gemm_grouped")
 
 
 # ----------------------------------------------------------------------------- timing helpers
@@ -270,50 +266,54 @@ def flush_l2(buf):
 
 
 def measure_prefill(dev, s, peaks, K):
-    """7B-shaped layer at N=512 on the tensor cores: GEMM time from events
-    around the seven launches, L2 flushed before every timed step."""
+    """7B-shaped layer at N=512 on the tensor cores: the seven projections in
+    one grouped GEMM launch, timed with events around it; L2 flushed before
+    every timed step.  A per-projection breakdown (one launch each) follows."""
     pre = PrefillWorkload(dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(3):
         for i in range(4):
             pre.quant(i, s)
-        for p in range(7):
-            pre.gemm(p, s)
+        pre.gemm_all(s)
     torch.cuda.synchronize()
     P = max(10, min(200, K // 50))
-    gemm_ms, quant_ms, step_ms = 0.0, 0.0, 0.0
-    per_proj = [0.0] * 7
+    gemm_ms, quant_ms = 0.0, 0.0
     for _ in range(P):
         flush_l2(flush)
-        e = events(13)
+        e = events(3)
         e[0].record(s)
         for i in range(4):
             pre.quant(i, s)
         e[1].record(s)
-        for p in range(7):
-            pre.gemm(p, s)
-            e[2 + p].record(s)
+        pre.gemm_all(s)
+        e[2].record(s)
         torch.cuda.synchronize()
         quant_ms += e[0].elapsed_time(e[1])
-        prev = e[1]
-        for p in range(7):
-            per_proj[p] += prev.elapsed_time(e[2 + p])
-            prev = e[2 + p]
-        gemm_ms += e[1].elapsed_time(e[8])
-        step_ms += e[0].elapsed_time(e[8])
+        gemm_ms += e[1].elapsed_time(e[2])
     gemm_ms /= P
     quant_ms /= P
-    step_ms /= P
+    per_proj = [0.0] * 7
+    for _ in range(P):
+        flush_l2(flush)
+        e = events(8)
+        e[0].record(s)
+        for p in range(7):
+            pre.gemm(p, s)
+            e[1 + p].record(s)
+        torch.cuda.synchronize()
+        for p in range(7):
+            per_proj[p] += e[p].elapsed_time(e[1 + p])
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
     tops = pre.flops / (gemm_ms * 1e-3) / 1e12
     prefill = {
         "workload": "7B-shaped layer, 7 projections (q,k,v,o 4096x4096; gate/up 11008x4096; "
-                    "down 4096x11008), N=512 tokens",
+                    "down 4096x11008), N=512 tokens, one grouped GEMM launch",
         "value": round(tops, 1), "unit": "int8 TOPS",
         "gemm_ms": round(gemm_ms, 4), "quant_ms": round(quant_ms, 4),
-        "step_tops_incl_quant": round(pre.flops / (step_ms * 1e-3) / 1e12, 1),
-        "per_projection_ms": [round(v / P, 4) for v in per_proj],
-        "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(int8_peak, 1),
+        "step_tops_incl_quant": round(pre.flops / ((gemm_ms + quant_ms) * 1e-3) / 1e12, 1),
+        "per_projection_ms_separate_launches": [round(v / P, 4) for v in per_proj],
+        "roofline": {"bound": "tensor", "kernel": "gemm_i8_tcgen05 (grouped, 7 layers)",
+                     "achieved": round(tops, 1), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(tops / int8_peak, 4),
                      "peak_note": "int8 peak = measured bf16 burst x nominal int8:bf16 ratio 2 (%s)"
                                   % peaks["source"],
@@ -360,7 +360,8 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- headline: K timed decode steps, events around every launch
     K = args.steps
-    ev = events(5 * K + 2)
+    names = ("quant_h", "quant_f", "gemv")
+    ev = events(4 * K + 2)
     for e in ev:              # create every event before the timed region
         e.record(s)
     torch.cuda.synchronize()
@@ -370,34 +371,32 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ev[-2].record(s)
     for i in range(K):
-        e = ev[5 * i:5 * i + 5]
+        e = ev[4 * i:4 * i + 4]
         e[0].record(s)
         dec.quant_h(s)
         e[1].record(s)
         dec.quant_f(s)
         e[2].record(s)
-        dec.gemv_h(s)
+        dec.gemv(s)
         e[3].record(s)
-        dec.gemv_f(s)
-        e[4].record(s)
     ev[-1].record(s)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     total_ms = max_over_ranks(ev[-2].elapsed_time(ev[-1]))
-    per = {k: 0.0 for k in ("quant_h", "quant_f", "gemv_h", "gemv_f")}
+    per = {k: 0.0 for k in names}
     for i in range(K):
-        e = ev[5 * i:5 * i + 5]
-        for j, k in enumerate(("quant_h", "quant_f", "gemv_h", "gemv_f")):
+        e = ev[4 * i:4 * i + 4]
+        for j, k in enumerate(names):
             per[k] += e[j].elapsed_time(e[j + 1])
     per = {k: v / K for k, v in per.items()}
     ms_per_step = total_ms / K
     gbs = world * dec.packed_bytes / (ms_per_step * 1e-3) / 1e9
-    gemv_h_gbs = dec.alg_bytes_h / (per["gemv_h"] * 1e-3) / 1e9
+    gemv_gbs = dec.alg_bytes / (per["gemv"] * 1e-3) / 1e9
     hbm_peak = peaks["hbm_gbs"]
     if args.only == "decode":
         print(json.dumps({"partial_run": "decode", "value": round(gbs, 1), "unit": "GB/s",
-                          "kernel_ms": per, "gemv_h_gbs": round(gemv_h_gbs, 1), "clocks": clk}))
+                          "kernel_ms": per, "gemv_gbs": round(gemv_gbs, 1), "clocks": clk}))
         return
 
     # ---- dependent per-layer chain, CUDA graph
@@ -477,18 +476,18 @@ def run_ours(args, rank, world, local_rank):
                 "workload": "BitNet-b1.58-2B-shaped decode: 30 layers x 7 projections, N=1",
                 "layers": dec.layers, "tokens": 1,
                 "packed_bytes_per_step": dec.packed_bytes,
-                "launches_per_step": 4,
+                "launches_per_step": 3,
                 "l2": "no flush: 521 MB of packed weights per step > 126 MB L2",
                 "parallelism": "replicas" if world > 1 else "single GPU",
             },
             "pct_of_measured_hbm": round(100 * gbs / world / hbm_peak, 2),
             "roofline": {
-                "bound": "hbm", "kernel": "gemv_stream (grouped, 180 layers, K=2560)",
-                "achieved": round(gemv_h_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(gemv_h_gbs / hbm_peak, 4),
+                "bound": "hbm", "kernel": "gemv_tile (grouped, 210 layers, K=2560 and 6912)",
+                "achieved": round(gemv_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(gemv_gbs / hbm_peak, 4),
                 "peak_note": "hbm_gbs %s (burst copy)" % peaks["source"],
-                "bytes_per_launch": dec.alg_bytes_h,
-                "avg_launch_ms": round(per["gemv_h"], 5),
+                "bytes_per_launch": dec.alg_bytes,
+                "avg_launch_ms": round(per["gemv"], 5),
                 "traffic": None,
             },
             "kernel_ms": {k: round(v, 5) for k, v in per.items()},
@@ -504,7 +503,7 @@ def run_ours(args, rank, world, local_rank):
             "e2e": {"value": round(world * dec.packed_bytes / (e2e_ms * 1e-3) / 1e9, 1),
                     "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 4 * K,
+            "gpu_launches": 3 * K,
             "clocks": clk,
             "cpu_baseline": cpu,
         }

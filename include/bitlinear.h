@@ -147,13 +147,15 @@ BITLINEAR_API bitlinear_status bitlinear_gemm(const uint32_t* packed, const floa
                                 bitlinear_stream_t stream);
 
 /*
- * One linear layer of a grouped decode call.  Every pointer follows the
- * conventions above; all problems of one call share K and N.
+ * One linear layer of a grouped call.  Every pointer follows the conventions
+ * above; M and K are this layer's shape (K a multiple of 128; for the GEMM, M a
+ * multiple of 128).  All layers of one call share the token count N.
  */
 typedef struct {
     const uint32_t* packed;   /* [M, K/16] words */
     const float* alpha;       /* [1] */
     int64_t M;
+    int64_t K;
     const int8_t* xq;         /* [N, K] */
     const float* amax;        /* [N] */
     const int32_t* xsum;      /* [N] */
@@ -163,14 +165,24 @@ typedef struct {
 
 /*
  * Decode GEMV over a list of independent layers in as few launches as
- * possible (one per 256 problems): the same arithmetic as bitlinear_gemv for
- * each entry.  Meant for layers that read activations known at the same time
+ * possible (one per 256 layers): the same arithmetic as bitlinear_gemv for
+ * each entry.  Meant for layers whose activations are known at the same time
  * -- the q/k/v or gate/up projections of one decoder layer, or a stream of
  * layers whose inputs are all available.  `problems` is a HOST array of
  * `count` entries, read during the call only.  1 <= N <= 16.
  */
 BITLINEAR_API bitlinear_status bitlinear_gemv_grouped(const bitlinear_problem* problems,
-                                                      int64_t count, int64_t K, int64_t N,
+                                                      int64_t count, int64_t N,
+                                                      bitlinear_stream_t stream);
+
+/*
+ * Tensor-core GEMM over a list of independent layers in one persistent
+ * launch per 8 layers (tiles of all layers share the grid, the layers with the
+ * largest K first): the same arithmetic as bitlinear_gemm for each entry.
+ * `problems` is a HOST array read during the call only.  N >= 1.
+ */
+BITLINEAR_API bitlinear_status bitlinear_gemm_grouped(const bitlinear_problem* problems,
+                                                      int64_t count, int64_t N,
                                                       bitlinear_stream_t stream);
 
 /* ------------------------------------------------- weights, no allocation */

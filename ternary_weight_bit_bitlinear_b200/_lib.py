@@ -24,7 +24,7 @@ ERR_DEVICE_TIMEOUT = 6
 class Problem(ctypes.Structure):
     """Mirror of bitlinear_problem (include/bitlinear.h)."""
     _fields_ = [("packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("M", ctypes.c_int64),
-                ("xq", ctypes.c_void_p), ("amax", ctypes.c_void_p), ("xsum", ctypes.c_void_p),
+                ("K", ctypes.c_int64), ("xq", ctypes.c_void_p), ("amax", ctypes.c_void_p), ("xsum", ctypes.c_void_p),
                 ("y", ctypes.c_void_p), ("acc", ctypes.c_void_p)]
 
 
@@ -63,8 +63,10 @@ def load(path: str = LIB_PATH):
         f = getattr(L, name)
         f.argtypes = [p, p, i64, i64, p, p, p, i64, p, p, p]
         f.restype = st
-    L.bitlinear_gemv_grouped.argtypes = [ctypes.POINTER(Problem), i64, i64, i64, p]
-    L.bitlinear_gemv_grouped.restype = st
+    for name in ("bitlinear_gemv_grouped", "bitlinear_gemm_grouped"):
+        f = getattr(L, name)
+        f.argtypes = [ctypes.POINTER(Problem), i64, i64, p]
+        f.restype = st
     L.bitlinear_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
     L.bitlinear_device_error.restype = st
     _lib = L
@@ -126,19 +128,26 @@ def bitlinear_gemm(packed, alpha, M, K, xq, amax, xsum, N, y, acc=None, stream=N
 
 
 def make_problems(entries):
-    """entries: iterable of (packed, alpha, M, xq, amax, xsum, y, acc-or-None) tensors.
-    Returns a ctypes array of Problem (keep it alive while the call runs)."""
+    """entries: iterable of (packed, alpha, M, K, xq, amax, xsum, y, acc-or-None);
+    tensors for the pointers.  Returns a ctypes array of Problem (keep it alive
+    while the call runs)."""
     entries = list(entries)
     arr = (Problem * max(1, len(entries)))()
-    for i, (packed, alpha, M, xq, amax, xsum, y, acc) in enumerate(entries):
-        arr[i] = Problem(packed.data_ptr(), alpha.data_ptr(), M, xq.data_ptr(), amax.data_ptr(),
-                         xsum.data_ptr(), y.data_ptr(), 0 if acc is None else acc.data_ptr())
+    for i, (packed, alpha, M, K, xq, amax, xsum, y, acc) in enumerate(entries):
+        arr[i] = Problem(packed.data_ptr(), alpha.data_ptr(), M, K, xq.data_ptr(),
+                         amax.data_ptr(), xsum.data_ptr(), y.data_ptr(),
+                         0 if acc is None else acc.data_ptr())
     return arr
 
 
-def bitlinear_gemv_grouped(problems, count, K, N, stream=None):
+def bitlinear_gemv_grouped(problems, count, N, stream=None):
     """problems: a ctypes array from make_problems()."""
-    return load().bitlinear_gemv_grouped(problems, count, K, N, _stream(stream))
+    return load().bitlinear_gemv_grouped(problems, count, N, _stream(stream))
+
+
+def bitlinear_gemm_grouped(problems, count, N, stream=None):
+    """problems: a ctypes array from make_problems()."""
+    return load().bitlinear_gemm_grouped(problems, count, N, _stream(stream))
 
 
 def bitlinear_pack_workspace_bytes(M, K):

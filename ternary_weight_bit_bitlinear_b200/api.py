@@ -72,32 +72,45 @@ def gemv(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out
                    with_acc, stream, out)
 
 
-def gemv_grouped(layers, xq, amax, xsum, with_acc=False, stream=None, outs=None):
-    """One grouped decode call over several layers that share K and the token
-    count.  layers: list of (packed, alpha); xq/amax/xsum: one tensor for all
-    layers, or a list with one entry per layer.  Returns a list of y (and acc)."""
+def _grouped(fn, name, layers, xq, amax, xsum, with_acc, stream, outs):
     n = len(layers)
     xqs = xq if isinstance(xq, (list, tuple)) else [xq] * n
     amaxs = amax if isinstance(amax, (list, tuple)) else [amax] * n
     xsums = xsum if isinstance(xsum, (list, tuple)) else [xsum] * n
-    N, K = xqs[0].shape
+    N = xqs[0].shape[0]
     ys, accs, entries = [], [], []
     for i, (packed, alpha) in enumerate(layers):
         _need(packed, torch.int32, "packed")
         _need(alpha, torch.float32, "alpha")
         _need(xqs[i], torch.int8, "xq")
-        if tuple(xqs[i].shape) != (N, K) or packed.shape[1] != K // 16:
-            raise ValueError("all layers of a grouped call share K and N")
-        M = packed.shape[0]
+        M, K = packed.shape[0], xqs[i].shape[1]
+        if xqs[i].shape[0] != N or packed.shape[1] != K // 16:
+            raise ValueError("layer %d: packed [M, K/16] must match xq [N, K]; N shared" % i)
         y = outs[i] if outs is not None else torch.empty((N, M), dtype=torch.float32,
                                                            device=packed.device)
         acc = torch.empty((N, M), dtype=torch.int32, device=packed.device) if with_acc else None
         ys.append(y)
         accs.append(acc)
-        entries.append((packed, alpha, M, xqs[i], amaxs[i], xsums[i], y, acc))
+        entries.append((packed, alpha, M, K, xqs[i], amaxs[i], xsums[i], y, acc))
     arr = _lib.make_problems(entries)
-    _lib.check(_lib.bitlinear_gemv_grouped(arr, n, K, N, stream), "bitlinear_gemv_grouped")
+    _lib.check(fn(arr, n, N, stream), name)
     return (ys, accs) if with_acc else ys
+
+
+def gemv_grouped(layers, xq, amax, xsum, with_acc=False, stream=None, outs=None):
+    """One grouped decode call over several layers sharing the token count.
+    layers: list of (packed, alpha); xq/amax/xsum: one tensor for all layers or
+    a list with one entry per layer (K may differ between layers).  Returns a
+    list of y (and of acc)."""
+    return _grouped(_lib.bitlinear_gemv_grouped, "bitlinear_gemv_grouped", layers, xq, amax,
+                    xsum, with_acc, stream, outs)
+
+
+def gemm_grouped(layers, xq, amax, xsum, with_acc=False, stream=None, outs=None):
+    """Tensor-core GEMM over several layers in one persistent launch (M % 128
+    == 0 for each); same arguments as gemv_grouped."""
+    return _grouped(_lib.bitlinear_gemm_grouped, "bitlinear_gemm_grouped", layers, xq, amax,
+                    xsum, with_acc, stream, outs)
 
 
 def gemm(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out=None):

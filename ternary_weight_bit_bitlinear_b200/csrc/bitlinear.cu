@@ -37,7 +37,7 @@ bitlinear_status check_mk(int64_t M, int64_t K) {
 struct DeviceInfo {
   int sms = 0;
   bool gemm_attr_set[2] = {false, false};
-  bool stream_attr_set[bl::kStreamMaxTokens + 1][17] = {};
+  int gemv_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};   // 0: not set up yet
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -87,118 +87,56 @@ bool encode_u8_2d(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t row
 }
 
 template <int NT>
-void launch_gemv_generic(const bitlinear_problem& q, int K, cudaStream_t s) {
-  const int M = static_cast<int>(q.M);
-  const int rows_per_block = (bl::kGemvThreads / 32) * bl::kGemvRows;
-  const int grid = (M + rows_per_block - 1) / rows_per_block;
-  bl::gemv_generic_kernel<NT><<<grid, bl::kGemvThreads, 0, s>>>(
-      reinterpret_cast<const uint4*>(q.packed), M, K / 64, reinterpret_cast<const uint4*>(q.xq),
-      q.alpha, q.amax, q.xsum, q.y, q.acc);
+bitlinear_status launch_gemv_tile(const bl::GemvParams& p, DeviceInfo* dev, cudaStream_t s) {
+  auto kernel = bl::gemv_tile_kernel<NT>;
+  constexpr int smem = bl::GemvCfg<NT>::kSmemBytes;
+  int& per_sm = dev->gemv_blocks_per_sm[NT];
+  if (per_sm == 0) {
+    int nb = 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, bl::kGemvThreads, smem) !=
+            cudaSuccess ||
+        nb < 1)
+      return BITLINEAR_ERR_CUDA;
+    per_sm = nb;
+  }
+  // Every warp resident at once, with the same number of units (give or take
+  // one) per warp: units per warp first, then just enough warps.
+  const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm * bl::kGemvWarps;
+  const int64_t upw = (p.total_units + cap - 1) / cap;
+  const int64_t warps = (p.total_units + upw - 1) / upw;
+  const int grid = static_cast<int>((warps + bl::kGemvWarps - 1) / bl::kGemvWarps);
+  kernel<<<grid, bl::kGemvThreads, smem, s>>>(p);
+  return launch_status();
 }
 
-void launch_gemv_generic_n(const bitlinear_problem& q, int K, int N, cudaStream_t s) {
+bitlinear_status launch_gemv_n(int N, const bl::GemvParams& p, DeviceInfo* dev, cudaStream_t s) {
   switch (N) {
 #define BL_GEMV_CASE(n) \
-  case n: launch_gemv_generic<n>(q, K, s); break;
+  case n: return launch_gemv_tile<n>(p, dev, s);
     BL_GEMV_CASE(1) BL_GEMV_CASE(2) BL_GEMV_CASE(3) BL_GEMV_CASE(4)
     BL_GEMV_CASE(5) BL_GEMV_CASE(6) BL_GEMV_CASE(7) BL_GEMV_CASE(8)
     BL_GEMV_CASE(9) BL_GEMV_CASE(10) BL_GEMV_CASE(11) BL_GEMV_CASE(12)
     BL_GEMV_CASE(13) BL_GEMV_CASE(14) BL_GEMV_CASE(15) BL_GEMV_CASE(16)
 #undef BL_GEMV_CASE
-    default: break;
-  }
-}
-
-// Streaming GEMV plan for one K: k-slices per row and spans (32 words) per
-// slice, with spans * N <= 12 so a lane's activations fit in 48 registers.
-struct StreamPlan {
-  bool ok = false;
-  int ksplit = 1, spans = 1, rows_per_stage = 1;
-};
-
-StreamPlan stream_plan(int64_t K, int64_t N) {
-  StreamPlan pl;
-  if (N < 1 || N > bl::kStreamMaxTokens) return pl;
-  const int64_t W = K / 16;
-  if (W * 4 > bl::kStreamStageBytes) return pl;
-  const int64_t nspan = (W + 31) / 32;
-  const int64_t cap = 12 / N;
-  int ks = 1;
-  while (ks * cap < nspan) ks *= 2;
-  if (ks > bl::kStreamConsumerWarps) return pl;
-  pl.ksplit = ks;
-  pl.spans = static_cast<int>((nspan + ks - 1) / ks);
-  pl.rows_per_stage = static_cast<int>(bl::kStreamStageBytes / (W * 4));
-  pl.ok = true;
-  return pl;
-}
-
-template <int NT, int S>
-bitlinear_status launch_stream_ns(const bl::GemvParams& p, int grid, DeviceInfo* dev,
-                                  cudaStream_t s) {
-  auto kernel = bl::gemv_stream_kernel<NT, S>;
-  constexpr int smem = static_cast<int>(bl::stream_smem_bytes());
-  if (!dev->stream_attr_set[NT][S]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
-    dev->stream_attr_set[NT][S] = true;
-  }
-  kernel<<<grid, bl::kStreamThreads, smem, s>>>(p);
-  return launch_status();
-}
-
-template <int NT, int S>
-bitlinear_status launch_stream_s(int spans, const bl::GemvParams& p, int grid, DeviceInfo* dev,
-                                 cudaStream_t s) {
-  if constexpr (S > 12 / NT) {
-    return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  } else {
-    if (spans == S) return launch_stream_ns<NT, S>(p, grid, dev, s);
-    return launch_stream_s<NT, S + 1>(spans, p, grid, dev, s);
-  }
-}
-
-bitlinear_status launch_stream(int N, int spans, const bl::GemvParams& p, int grid,
-                               DeviceInfo* dev, cudaStream_t s) {
-  switch (N) {
-    case 1: return launch_stream_s<1, 1>(spans, p, grid, dev, s);
-    case 2: return launch_stream_s<2, 1>(spans, p, grid, dev, s);
-    case 3: return launch_stream_s<3, 1>(spans, p, grid, dev, s);
-    case 4: return launch_stream_s<4, 1>(spans, p, grid, dev, s);
     default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   }
 }
 
-// Decode GEMV over problems that share K and N (all validated).
-bitlinear_status gemv_group(const bitlinear_problem* probs, int64_t count, int64_t K, int64_t N,
+// Decode GEMV over problems that share N (all validated): one launch
+// per kGemvMaxProblems problems, units of 32 rows numbered across problems.
+bitlinear_status gemv_group(const bitlinear_problem* probs, int64_t count, int64_t N,
                             cudaStream_t s) {
-  const StreamPlan pl = stream_plan(K, N);
-  if (!pl.ok) {
-    for (int64_t i = 0; i < count; ++i)
-      launch_gemv_generic_n(probs[i], static_cast<int>(K), static_cast<int>(N), s);
-    return launch_status();
-  }
   DeviceInfo* dev = nullptr;
   bitlinear_status st = device_info(&dev);
   if (st != BITLINEAR_OK) return st;
-  const int grid_cap = dev->sms * 2;
-  int64_t total_rows = 0;
-  for (int64_t i = 0; i < count; ++i) total_rows += probs[i].M;
-  // Units of consecutive rows: about 8 per resident CTA for balance, a whole
-  // number of stages when longer than one stage.
-  const int RS = pl.rows_per_stage;
-  int64_t ur = (total_rows + 8 * grid_cap - 1) / (8 * grid_cap);
-  if (ur > RS) ur = (ur + RS - 1) / RS * RS;
-  const int64_t ur_cap = bl::kStreamMaxUnitRows / RS * RS;
-  if (ur > ur_cap) ur = ur_cap;
-  if (ur < 1) ur = 1;
-  for (int64_t base = 0; base < count; base += bl::kStreamMaxProblems) {
-    const int n = static_cast<int>(count - base < bl::kStreamMaxProblems
-                                       ? count - base : bl::kStreamMaxProblems);
+  for (int64_t base = 0; base < count; base += bl::kGemvMaxProblems) {
+    const int n = static_cast<int>(count - base < bl::kGemvMaxProblems
+                                       ? count - base : bl::kGemvMaxProblems);
     bl::GemvParams p;
     memset(&p, 0, sizeof p);
-    int units = 0;
+    int64_t units = 0;
     for (int i = 0; i < n; ++i) {
       const bitlinear_problem& q = probs[base + i];
       bl::GemvProblem& g = p.prob[i];
@@ -210,18 +148,15 @@ bitlinear_status gemv_group(const bitlinear_problem* probs, int64_t count, int64
       g.y = q.y;
       g.acc = q.acc;
       g.M = static_cast<int>(q.M);
-      g.unit_begin = units;
-      units += static_cast<int>((q.M + ur - 1) / ur);
+      g.K = static_cast<int>(q.K);
+      g.W = static_cast<int>(q.K / 16);
+      g.unit_begin = static_cast<int>(units);
+      units += (q.M + bl::kGemvTileRows - 1) / bl::kGemvTileRows;
     }
+    if (units > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     p.num_problems = n;
-    p.total_units = units;
-    p.K = static_cast<int>(K);
-    p.W = static_cast<int>(K / 16);
-    p.rows_per_stage = RS;
-    p.unit_rows = static_cast<int>(ur);
-    p.ksplit = pl.ksplit;
-    const int grid = units < grid_cap ? units : grid_cap;
-    st = launch_stream(static_cast<int>(N), pl.spans, p, grid, dev, s);
+    p.total_units = static_cast<int>(units);
+    st = launch_gemv_n(static_cast<int>(N), p, dev, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;
@@ -254,6 +189,66 @@ bitlinear_status check_matmul_args(const uint32_t* packed, const float* alpha, i
   if (!aligned16(packed) || !aligned16(xq) || !aligned16(y) || (acc && !aligned16(acc)))
     return BITLINEAR_ERR_MISALIGNED;
   if (!aligned4(alpha) || !aligned4(amax) || !aligned4(xsum)) return BITLINEAR_ERR_MISALIGNED;
+  return BITLINEAR_OK;
+}
+
+bitlinear_status check_problem(const bitlinear_problem& q, int64_t N) {
+  return check_matmul_args(q.packed, q.alpha, q.M, q.K, q.xq, q.amax, q.xsum, N, q.y, q.acc);
+}
+
+// Tensor-core GEMM over problems that share N (all validated, M % 128 == 0):
+// one persistent launch per kGemmMaxProblems problems, tiles numbered across
+// problems with the largest K first so the longest tiles start in the first
+// wave.
+bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64_t N,
+                            cudaStream_t s) {
+  DeviceInfo* dev = nullptr;
+  bitlinear_status st = device_info(&dev);
+  if (st != BITLINEAR_OK) return st;
+  const bool wide = N > 128;
+  const int BN = wide ? 256 : 128;
+  const int64_t n_tiles = (N + BN - 1) / BN;
+  for (int64_t base = 0; base < count; base += bl::kGemmMaxProblems) {
+    const int n = static_cast<int>(count - base < bl::kGemmMaxProblems
+                                       ? count - base : bl::kGemmMaxProblems);
+    int order[bl::kGemmMaxProblems];
+    for (int i = 0; i < n; ++i) order[i] = i;
+    for (int i = 1; i < n; ++i)   // insertion sort by K, descending (stable)
+      for (int j = i; j > 0 && probs[base + order[j]].K > probs[base + order[j - 1]].K; --j) {
+        const int t = order[j];
+        order[j] = order[j - 1];
+        order[j - 1] = t;
+      }
+    bl::GemmParams p;
+    memset(&p, 0, sizeof p);
+    int64_t tiles = 0;
+    for (int i = 0; i < n; ++i) {
+      const bitlinear_problem& q = probs[base + order[i]];
+      if (!encode_u8_2d(&p.tmA[i], q.packed, static_cast<uint64_t>(q.K / 4),
+                        static_cast<uint64_t>(q.M), bl::kGemmPackedRowBytes, bl::kGemmBM,
+                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
+          !encode_u8_2d(&p.tmB[i], q.xq, static_cast<uint64_t>(q.K), static_cast<uint64_t>(N),
+                        bl::kGemmBK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BITLINEAR_ERR_CUDA;
+      bl::GemmProblem& g = p.prob[i];
+      g.alpha = q.alpha;
+      g.amax = q.amax;
+      g.xsum = q.xsum;
+      g.y = q.y;
+      g.acc = q.acc;
+      g.M = static_cast<int>(q.M);
+      g.K = static_cast<int>(q.K);
+      g.N = static_cast<int>(N);
+      g.n_tiles = static_cast<int>(n_tiles);
+      g.tile_begin = static_cast<int>(tiles);
+      tiles += (q.M / bl::kGemmBM) * n_tiles;
+    }
+    if (tiles > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    p.num_problems = n;
+    p.total_tiles = static_cast<int>(tiles);
+    st = wide ? launch_gemm<256, 4>(p, dev, 1, s) : launch_gemm<128, 6>(p, dev, 0, s);
+    if (st != BITLINEAR_OK) return st;
+  }
   return BITLINEAR_OK;
 }
 
@@ -330,23 +325,21 @@ bitlinear_status bitlinear_gemv(const uint32_t* packed, const float* alpha, int6
                                 int64_t N, float* y, int32_t* acc, bitlinear_stream_t stream) {
   bitlinear_status st = check_matmul_args(packed, alpha, M, K, xq, amax, xsum, N, y, acc);
   if (st != BITLINEAR_OK || N == 0) return st;
-  if (N > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  const bitlinear_problem q = {packed, alpha, M, xq, amax, xsum, y, acc};
-  return gemv_group(&q, 1, K, N, reinterpret_cast<cudaStream_t>(stream));
+  if (N > bl::kGemvMaxTokens) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  const bitlinear_problem q = {packed, alpha, M, K, xq, amax, xsum, y, acc};
+  return gemv_group(&q, 1, N, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bitlinear_status bitlinear_gemv_grouped(const bitlinear_problem* problems, int64_t count,
-                                        int64_t K, int64_t N, bitlinear_stream_t stream) {
+                                        int64_t N, bitlinear_stream_t stream) {
   if (count < 0 || N < 0 || (count > 0 && !problems)) return BITLINEAR_ERR_INVALID_ARG;
   if (count == 0 || N == 0) return BITLINEAR_OK;
-  if (N > 16) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  if (N > bl::kGemvMaxTokens) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   for (int64_t i = 0; i < count; ++i) {
-    const bitlinear_problem& q = problems[i];
-    bitlinear_status st = check_matmul_args(q.packed, q.alpha, q.M, K, q.xq, q.amax, q.xsum, N,
-                                            q.y, q.acc);
+    bitlinear_status st = check_problem(problems[i], N);
     if (st != BITLINEAR_OK) return st;
   }
-  return gemv_group(problems, count, K, N, reinterpret_cast<cudaStream_t>(stream));
+  return gemv_group(problems, count, N, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bitlinear_status bitlinear_gemm(const uint32_t* packed, const float* alpha, int64_t M, int64_t K,
@@ -355,32 +348,20 @@ bitlinear_status bitlinear_gemm(const uint32_t* packed, const float* alpha, int6
   bitlinear_status st = check_matmul_args(packed, alpha, M, K, xq, amax, xsum, N, y, acc);
   if (st != BITLINEAR_OK || N == 0) return st;
   if (M % 128 != 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  DeviceInfo* dev = nullptr;
-  if ((st = device_info(&dev)) != BITLINEAR_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool wide = N > 128;
-  const int BN = wide ? 256 : 128;
-  bl::GemmParams p;
-  memset(&p, 0, sizeof p);
-  if (!encode_u8_2d(&p.tmA[0], packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(M),
-                    bl::kGemmPackedRowBytes, bl::kGemmBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_u8_2d(&p.tmB[0], xq, static_cast<uint64_t>(K), static_cast<uint64_t>(N),
-                    bl::kGemmBK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
-    return BITLINEAR_ERR_CUDA;
-  bl::GemmProblem& pr = p.prob[0];
-  pr.alpha = alpha;
-  pr.amax = amax;
-  pr.xsum = xsum;
-  pr.y = y;
-  pr.acc = acc;
-  pr.M = static_cast<int>(M);
-  pr.K = static_cast<int>(K);
-  pr.N = static_cast<int>(N);
-  pr.n_tiles = static_cast<int>((N + BN - 1) / BN);
-  pr.tile_begin = 0;
-  p.num_problems = 1;
-  p.total_tiles = static_cast<int>(M / bl::kGemmBM) * pr.n_tiles;
-  return wide ? launch_gemm<256, 4>(p, dev, 1, s) : launch_gemm<128, 6>(p, dev, 0, s);
+  const bitlinear_problem q = {packed, alpha, M, K, xq, amax, xsum, y, acc};
+  return gemm_group(&q, 1, N, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitlinear_status bitlinear_gemm_grouped(const bitlinear_problem* problems, int64_t count,
+                                        int64_t N, bitlinear_stream_t stream) {
+  if (count < 0 || N < 0 || (count > 0 && !problems)) return BITLINEAR_ERR_INVALID_ARG;
+  if (count == 0 || N == 0) return BITLINEAR_OK;
+  for (int64_t i = 0; i < count; ++i) {
+    bitlinear_status st = check_problem(problems[i], N);
+    if (st != BITLINEAR_OK) return st;
+    if (problems[i].M % 128 != 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  }
+  return gemm_group(problems, count, N, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bitlinear_status bitlinear_device_error(int* status_out, int clear) {

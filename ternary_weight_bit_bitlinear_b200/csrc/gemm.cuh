@@ -61,6 +61,8 @@ struct GemmSmem {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
+  float ep_scale[4][BN];   // per epilogue warp: alpha * amax/127 of the tile's tokens
+  int ep_xsum[4][BN];      // per epilogue warp: activation sums of the tile's tokens
   uint32_t tmem_slot;
   int abort;
 };
@@ -224,7 +226,25 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       if (!mbar_wait(&s.tfull[ab], ap, abort)) break;
       tc_fence_after();
       const int m = m_blk * kGemmBM + r_in_tile;
-      const float alpha = *pr.alpha;
+      // this warp's copy of the tile's per-token scale and sum
+      float* sc = s.ep_scale[quarter];
+      int* xs = s.ep_xsum[quarter];
+      {
+        const float alpha = *pr.alpha;
+        __syncwarp();
+        for (int i = lane; i < BN; i += 32) {
+          const int n = n_blk * BN + i;
+          float v = 0.0f;
+          int x = 0;
+          if (n < pr.N) {
+            v = __fmul_rn(alpha, __fdiv_rn(__ldg(pr.amax + n), 127.0f));
+            x = __ldg(pr.xsum + n);
+          }
+          sc[i] = v;
+          xs[i] = x;
+        }
+        __syncwarp();
+      }
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t r[32];
@@ -236,10 +256,9 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         for (int j = 0; j < 32; ++j) {
           const int n = n0 + j;
           if (n < pr.N) {
-            const int a = static_cast<int>(r[j]) - __ldg(pr.xsum + n);
-            const float scale = __fmul_rn(alpha, __fdiv_rn(__ldg(pr.amax + n), 127.0f));
+            const int a = static_cast<int>(r[j]) - xs[cc * 32 + j];
             const int64_t o = static_cast<int64_t>(n) * pr.M + m;
-            pr.y[o] = __fmul_rn(__int2float_rn(a), scale);
+            pr.y[o] = __fmul_rn(__int2float_rn(a), sc[cc * 32 + j]);
             if (pr.acc) pr.acc[o] = a;
           }
         }

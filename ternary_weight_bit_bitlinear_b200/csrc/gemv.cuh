@@ -2,123 +2,48 @@
 //
 // The reading notes' I2_S kernel is MAD-based: int8 multiply-adds of
 // activations against ternary weights ("Bitnet.cpp" reading notes, section 4.1
-// item 3); the FairyFuse "fused kernel design" unpacks the bit-packed codes
-// and accumulates in the same loop with no intermediate writes.  Here each
-// 16-byte load brings 64 weights; (word >> 2j) & 0x03030303 puts four codes+1
-// in byte lanes that line up with four int8 activations, so one dp4a does four
-// multiply-adds.  The +1 offset is removed once per output with the token's
-// activation sum: acc = dp4a_total - xsum.
+// item 3); the FairyFuse "fused kernel design" unpacks the bit-packed codes and
+// accumulates in the same loop, with no intermediate writes.
+//
+// Work unit: 32 consecutive rows of one layer, one row per lane, all of its K
+// (layers of one launch may differ in K).
+// Each warp runs its own pipeline of k-chunks (512 weights = 128 bytes per row,
+// plus the matching 512 int8 activations of every token), brought in with
+// 16-byte cp.async copies into a STAGES-deep ring in shared memory.  A row's
+// 16-byte chunks are stored XOR-swizzled by row (chunk c of row r at c ^ r%8),
+// so the per-lane 16-byte reads of 8 consecutive lanes hit all 32 banks once.
+// Activations are read as broadcasts (every lane wants the same k).
+//
+// Arithmetic per 32-bit packed word (16 weights): byte lane b of field j
+// (bits 2j..2j+1) holds code+1 of weight 4j+b, so
+//   w & (0x03030303 << 2j)  =  4^j * (codes+1 of weights 4j..4j+3, one per byte)
+// and one dp4a (unsigned bytes x signed int8) against activations 4j..4j+3
+// accumulates 4^j times their dot product.  Four accumulators, one per j, are
+// combined exactly at the end (acc_j is a multiple of 4^j), and the +1 offset
+// is removed with the token's activation sum: acc = sum - xsum.  No shifts in
+// the inner loop and no cross-lane reduction at all.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace bl {
 
-// ---------------------------------------------------------------- generic
-// Any N <= 16 and any K: each warp takes 4 rows; lanes stride over 16-byte
-// chunks (64 weights) and read the matching activations through L1.
-
-constexpr int kGemvThreads = 256;
-constexpr int kGemvRows = 4;   // rows per warp
-
-__device__ __forceinline__ uint4 ld_stream_u4(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+constexpr int kGemvTileRows = 32;        // rows per unit: one per lane
+constexpr int kGemvChunkBytes = 128;     // packed bytes per row per k-chunk (512 weights)
+constexpr int kGemvChunkK = 512;
+constexpr int kGemvWarps = 4;            // warps per CTA
+constexpr int kGemvThreads = kGemvWarps * 32;
+constexpr int kGemvMaxTokens = 16;
+constexpr int kGemvMaxProblems = 256;
 
 template <int NT>
-__global__ void __launch_bounds__(kGemvThreads)
-gemv_generic_kernel(const uint4* __restrict__ wq, int M, int cpr,      // cpr = K / 64 chunks per row
-            const uint4* __restrict__ xq4,                       // [N, 4*cpr] uint4
-            const float* __restrict__ alpha_ptr, const float* __restrict__ amax,
-            const int32_t* __restrict__ xsum, float* __restrict__ y,
-            int32_t* __restrict__ acc_out) {
-  constexpr int R = kGemvRows;
-  const int lane = threadIdx.x & 31;
-  const int warp_global = (blockIdx.x * kGemvThreads + threadIdx.x) >> 5;
-  const int row0 = warp_global * R;
-  if (row0 >= M) return;
-
-  int acc[R][NT];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[r][t] = 0;
-
-  for (int c = lane; c < cpr; c += 32) {
-    uint32_t u[R][16];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      uint4 w = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
-      if (row0 + r < M) w = ld_stream_u4(wq + static_cast<int64_t>(row0 + r) * cpr + c);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) u[r][4 * i + j] = (ws[i] >> (2 * j)) & 0x03030303u;
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const uint4* xa = xq4 + static_cast<int64_t>(t) * 4 * cpr + 4 * c;
-      int a[16];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint4 v = __ldg(xa + i);
-        a[4 * i + 0] = static_cast<int>(v.x);
-        a[4 * i + 1] = static_cast<int>(v.y);
-        a[4 * i + 2] = static_cast<int>(v.z);
-        a[4 * i + 3] = static_cast<int>(v.w);
-      }
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[r][t] = __dp4a(static_cast<int>(u[r][e]), a[e], acc[r][t]);
-    }
-  }
-
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[r][t] += __shfl_xor_sync(0xFFFFFFFFu, acc[r][t], o);
-
-  const float alpha = *alpha_ptr;
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      if (lane == ((r * NT + t) & 31) && row0 + r < M) {
-        const int a = acc[r][t] - xsum[t];
-        const float scale = __fmul_rn(alpha, __fdiv_rn(amax[t], 127.0f));
-        const int64_t o = static_cast<int64_t>(t) * M + row0 + r;
-        y[o] = __fmul_rn(__int2float_rn(a), scale);
-        if (acc_out) acc_out[o] = a;
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- streaming
-// N <= 4.  One launch covers a group of problems that share K (and N).  Work
-// is cut into units of consecutive rows of one problem; since rows are stored
-// back to back, a unit is one contiguous byte range, copied into a 4-stage
-// shared-memory ring by one producer thread with bulk async copies.  Eight
-// consumer warps read it: warp w owns k-slice (w % ksplit) -- every lane keeps
-// the int8 activations of its 32-word-strided slice in registers for the whole
-// unit -- and rows w / ksplit, + 8/ksplit, ...; a row's partial dot product is
-// reduced over the warp, and with ksplit > 1 combined in shared memory.
-
-constexpr int kStreamStages = 4;
-constexpr int kStreamStageBytes = 16384;
-constexpr int kStreamConsumerWarps = 8;
-constexpr int kStreamThreads = (kStreamConsumerWarps + 1) * 32;
-constexpr int kStreamMaxUnitRows = 1024;
-constexpr int kStreamMaxTokens = 4;
-constexpr int kStreamMaxProblems = 256;
+struct GemvCfg {
+  static constexpr int kStages = NT <= 4 ? 4 : (NT <= 8 ? 3 : 2);
+  static constexpr int kWeightBytes = kGemvTileRows * kGemvChunkBytes;    // 4 KB
+  static constexpr int kStageBytes = kWeightBytes + NT * kGemvChunkK;
+  static constexpr int kWarpBytes = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kGemvWarps * kWarpBytes;
+};
 
 struct GemvProblem {
   const uint32_t* packed;
@@ -128,26 +53,17 @@ struct GemvProblem {
   const int32_t* xsum;
   float* y;
   int32_t* acc;
-  int M;
+  int M, K, W;      // W = K / 16 words per row
   int unit_begin;   // first unit of this problem
 };
 
 struct GemvParams {
-  GemvProblem prob[kStreamMaxProblems];
+  GemvProblem prob[kGemvMaxProblems];
   int num_problems;
   int total_units;
-  int K, W;              // W = K / 16 words per row
-  int rows_per_stage;    // RS
-  int unit_rows;         // RS * stages per unit
-  int ksplit;            // 1, 2, 4 or 8 k-slices
 };
 
-constexpr size_t stream_smem_bytes() {
-  return kStreamStages * kStreamStageBytes + 2 * kStreamStages * sizeof(uint64_t) +
-         kStreamMaxUnitRows * kStreamMaxTokens * sizeof(int) + 16;
-}
-
-__device__ __forceinline__ int stream_locate(const GemvParams& p, int unit) {
+__device__ __forceinline__ int gemv_locate(const GemvParams& p, int unit) {
   int lo = 0, hi = p.num_problems - 1;
   while (lo < hi) {   // last problem whose unit_begin <= unit
     const int mid = (lo + hi + 1) >> 1;
@@ -156,158 +72,105 @@ __device__ __forceinline__ int stream_locate(const GemvParams& p, int unit) {
   return lo;
 }
 
-template <int NT, int S>
-__global__ void __launch_bounds__(kStreamThreads, 2)
-gemv_stream_kernel(const __grid_constant__ GemvParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint32_t* ring = reinterpret_cast<uint32_t*>(smem);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStreamStages * kStreamStageBytes);
-  uint64_t* empty = full + kStreamStages;
-  int* part = reinterpret_cast<int*>(empty + kStreamStages);
-  __shared__ int abort_flag;
-  volatile int* abort = &abort_flag;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kStageWords = kStreamStageBytes / 4;
-  const int W = p.W, RS = p.rows_per_stage, UR = p.unit_rows;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStreamStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kStreamConsumerWarps);
-    }
-    abort_flag = 0;
-    fence_mbar_init();
+// Issue the copies of k-chunk `kc` of the unit starting at row0 into `st`.
+template <int NT>
+__device__ __forceinline__ void gemv_issue(const GemvProblem& pr, int row0, int kc, uint8_t* st,
+                                           int lane) {
+  // weights: 32 rows x 8 sixteen-byte chunks; a warp instruction copies 4
+  // whole 128-byte row segments (coalesced)
+  const int c = lane & 7;
+  const int word = kc * (kGemvChunkBytes / 4) + c * 4;
+  const bool kval = word < pr.W;
+#pragma unroll
+  for (int i = 0; i < kGemvTileRows / 4; ++i) {
+    const int r = i * 4 + (lane >> 3);
+    const int row = row0 + r;
+    const bool ok = kval && row < pr.M;
+    const uint32_t* src = ok ? pr.packed + static_cast<int64_t>(row) * pr.W + word : pr.packed;
+    cp_async16(st + r * kGemvChunkBytes + ((c ^ (r & 7)) << 4), src, ok ? 16u : 0u);
   }
-  __syncthreads();
+  // activations: 512 bytes per token, 16 per lane
+  const int k0 = kc * kGemvChunkK + lane * 16;
+  const bool xval = k0 < pr.K;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int8_t* src = xval ? pr.xq + static_cast<int64_t>(t) * pr.K + k0 : pr.xq;
+    cp_async16(st + GemvCfg<NT>::kWeightBytes + t * kGemvChunkK + lane * 16, src,
+               xval ? 16u : 0u);
+  }
+}
 
-  if (warp == kStreamConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t slot = 0, phase = 0;
-      for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
-        const GemvProblem& pr = p.prob[stream_locate(p, u)];
-        const int r0 = (u - pr.unit_begin) * UR;
-        const int r1 = min(r0 + UR, pr.M);
-        for (int rs = r0; rs < r1; rs += RS) {
-          const int nrows = min(RS, r1 - rs);
-          if (!mbar_wait(&empty[slot], phase ^ 1u, abort)) return;
-          const uint32_t bytes = static_cast<uint32_t>(nrows) * W * 4u;
-          mbar_arrive_expect_tx(&full[slot], bytes);
-          bulk_load(ring + slot * kStageWords, pr.packed + static_cast<int64_t>(rs) * W, bytes,
-                    &full[slot]);
-          if (++slot == kStreamStages) { slot = 0; phase ^= 1u; }
+template <int NT>
+__global__ void __launch_bounds__(kGemvThreads)
+gemv_tile_kernel(const __grid_constant__ GemvParams p) {
+  using C = GemvCfg<NT>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = smem + warp * C::kWarpBytes;
+  const int total_warps = gridDim.x * kGemvWarps;
+  const uint32_t sw = static_cast<uint32_t>(lane & 7);
+
+  for (int u = blockIdx.x * kGemvWarps + warp; u < p.total_units; u += total_warps) {
+    const GemvProblem& pr = p.prob[gemv_locate(p, u)];
+    const int row0 = (u - pr.unit_begin) * kGemvTileRows;
+    const int nchunks = (pr.K + kGemvChunkK - 1) / kGemvChunkK;
+
+    int acc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[t][j] = 0;
+
+#pragma unroll
+    for (int s = 0; s < C::kStages - 1; ++s) {
+      if (s < nchunks) gemv_issue<NT>(pr, row0, s, ring + s * C::kStageBytes, lane);
+      cp_async_commit();
+    }
+    for (int kc = 0; kc < nchunks; ++kc) {
+      const int nxt = kc + C::kStages - 1;
+      if (nxt < nchunks)
+        gemv_issue<NT>(pr, row0, nxt, ring + (nxt % C::kStages) * C::kStageBytes, lane);
+      cp_async_commit();
+      cp_async_wait<C::kStages - 1>();
+      __syncwarp();
+      const uint8_t* st = ring + (kc % C::kStages) * C::kStageBytes;
+      const uint8_t* wrow = st + lane * kGemvChunkBytes;
+      const uint8_t* xs = st + C::kWeightBytes;
+#pragma unroll
+      for (int c = 0; c < kGemvChunkBytes / 16; ++c) {
+        const uint4 w = *reinterpret_cast<const uint4*>(wrow + ((static_cast<uint32_t>(c) ^ sw) << 4));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const uint4* xp = reinterpret_cast<const uint4*>(xs + t * kGemvChunkK + c * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 xa = xp[i];
+            acc[t][0] = dp4a_us(ws[i] & 0x03030303u, xa.x, acc[t][0]);
+            acc[t][1] = dp4a_us(ws[i] & 0x0C0C0C0Cu, xa.y, acc[t][1]);
+            acc[t][2] = dp4a_us(ws[i] & 0x30303030u, xa.z, acc[t][2]);
+            acc[t][3] = dp4a_us(ws[i] & 0xC0C0C0C0u, xa.w, acc[t][3]);
+          }
         }
       }
+      __syncwarp();   // every lane is done with this stage before it is refilled
     }
-    return;
-  }
 
-  // ------------------------------------------------------------ consumers
-  const int ks = p.ksplit;
-  const int slice = warp % ks, group = warp / ks, groups = kStreamConsumerWarps / ks;
-  const int word0 = slice * S * 32 + lane;   // this lane's first word within a row
-  uint32_t slot = 0, phase = 0;
-  int cur = -1;
-  uint32_t xr[NT][S][4];
-  float scale = 0.0f;   // lane t < NT: alpha * (amax_t / 127)
-  int xs = 0;           // lane t < NT: sum of token t's activations
-
-  for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
-    const int pi = stream_locate(p, u);
-    const GemvProblem& pr = p.prob[pi];
-    const int r0 = (u - pr.unit_begin) * UR;
-    const int r1 = min(r0 + UR, pr.M);
-    if (pi != cur) {
-      cur = pi;
+    const int row = row0 + lane;
+    if (row < pr.M) {
+      const float alpha = *pr.alpha;
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-#pragma unroll
-        for (int j = 0; j < S; ++j) {
-          const int wi = word0 + 32 * j;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (wi < W)
-            v = __ldg(reinterpret_cast<const uint4*>(pr.xq + static_cast<int64_t>(t) * p.K) + wi);
-          xr[t][j][0] = v.x;
-          xr[t][j][1] = v.y;
-          xr[t][j][2] = v.z;
-          xr[t][j][3] = v.w;
-        }
-      }
-      if (lane < NT) {
-        scale = __fmul_rn(*pr.alpha, __fdiv_rn(pr.amax[lane], 127.0f));
-        xs = pr.xsum[lane];
-      }
-    }
-    if (ks > 1) {
-      for (int i = threadIdx.x; i < (r1 - r0) * NT; i += kStreamConsumerWarps * 32) part[i] = 0;
-      named_barrier(1, kStreamConsumerWarps * 32);
-    }
-    for (int rs = r0; rs < r1; rs += RS) {
-      const int nrows = min(RS, r1 - rs);
-      // On a timeout the stage is skipped but the loop (and its named
-      // barriers) still runs to the end, so no warp is left waiting.
-      const bool ready = mbar_wait(&full[slot], phase, abort);
-      const uint32_t* st = ring + slot * kStageWords;
-      for (int i = group; ready && i < nrows; i += groups) {
-        int acc[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = 0;
-        const uint32_t* row = st + i * W;
-#pragma unroll
-        for (int j = 0; j < S; ++j) {
-          const int wi = word0 + 32 * j;
-          if (wi < W) {
-            const uint32_t w = row[wi];
-            const uint32_t q0 = w & 0x03030303u, q1 = (w >> 2) & 0x03030303u,
-                           q2 = (w >> 4) & 0x03030303u, q3 = (w >> 6) & 0x03030303u;
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-              acc[t] = __dp4a(static_cast<int>(q0), static_cast<int>(xr[t][j][0]), acc[t]);
-              acc[t] = __dp4a(static_cast<int>(q1), static_cast<int>(xr[t][j][1]), acc[t]);
-              acc[t] = __dp4a(static_cast<int>(q2), static_cast<int>(xr[t][j][2]), acc[t]);
-              acc[t] = __dp4a(static_cast<int>(q3), static_cast<int>(xr[t][j][3]), acc[t]);
-            }
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xFFFFFFFFu, acc[t], o);
-        int mine = acc[0];
-#pragma unroll
-        for (int t = 1; t < NT; ++t)
-          if (lane == t) mine = acc[t];
-        if (lane < NT) {
-          const int row_idx = rs + i;
-          if (ks == 1) {
-            const int a = mine - xs;
-            const int64_t o = static_cast<int64_t>(lane) * pr.M + row_idx;
-            pr.y[o] = __fmul_rn(__int2float_rn(a), scale);
-            if (pr.acc) pr.acc[o] = a;
-          } else {
-            atomicAdd(&part[(row_idx - r0) * NT + lane], mine);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
-      if (++slot == kStreamStages) { slot = 0; phase ^= 1u; }
-    }
-    if (ks > 1) {
-      named_barrier(1, kStreamConsumerWarps * 32);
-      const float alpha = *pr.alpha;
-      for (int i = threadIdx.x; i < (r1 - r0) * NT; i += kStreamConsumerWarps * 32) {
-        const int t = i % NT, row_idx = r0 + i / NT;
-        const int a = part[i] - pr.xsum[t];
-        const float sc = __fmul_rn(alpha, __fdiv_rn(pr.amax[t], 127.0f));
-        const int64_t o = static_cast<int64_t>(t) * pr.M + row_idx;
-        pr.y[o] = __fmul_rn(__int2float_rn(a), sc);
+        const int a = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) -
+                      pr.xsum[t];
+        const float scale = __fmul_rn(alpha, __fdiv_rn(pr.amax[t], 127.0f));
+        const int64_t o = static_cast<int64_t>(t) * pr.M + row;
+        pr.y[o] = __fmul_rn(__int2float_rn(a), scale);
         if (pr.acc) pr.acc[o] = a;
       }
-      named_barrier(1, kStreamConsumerWarps * 32);
     }
   }
+  cp_async_wait<0>();
 }
 
 }  // namespace bl

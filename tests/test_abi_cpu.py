@@ -123,20 +123,30 @@ def test_header_is_self_contained(tmp_path):
                     str(tmp_path / "t.o")], check=True)
 
 
-def test_gemv_grouped_argument_errors(L):
-    f = L.bitlinear_gemv_grouped
+@pytest.mark.parametrize("name", ["bitlinear_gemv_grouped", "bitlinear_gemm_grouped"])
+def test_grouped_argument_errors(L, name):
+    f = getattr(L, name)
     P = _lib.Problem
-    good = P(FAKE, FAKE, 128, FAKE, FAKE, FAKE, FAKE, 0)
+
+    def prob(**kw):
+        a = dict(packed=FAKE, alpha=FAKE, M=128, K=256, xq=FAKE, amax=FAKE, xsum=FAKE, y=FAKE,
+                 acc=0)
+        a.update(kw)
+        return P(a["packed"], a["alpha"], a["M"], a["K"], a["xq"], a["amax"], a["xsum"], a["y"],
+                 a["acc"])
+
+    good = prob()
     arr = (P * 2)(good, good)
-    assert f(arr, -1, 256, 1, None) == _lib.ERR_INVALID_ARG
-    assert f(None, 2, 256, 1, None) == _lib.ERR_INVALID_ARG
-    assert f(arr, 0, 256, 1, None) == _lib.OK
-    assert f(arr, 2, 256, 0, None) == _lib.OK
-    assert f(arr, 2, 256, 17, None) == _lib.ERR_UNSUPPORTED_SHAPE
-    assert f(arr, 2, 200, 1, None) == _lib.ERR_UNSUPPORTED_SHAPE
-    bad = (P * 2)(good, P(FAKE, FAKE, 128, FAKE, FAKE, FAKE, MISALIGNED, 0))
-    assert f(bad, 2, 256, 1, None) == _lib.ERR_MISALIGNED
-    bad = (P * 2)(good, P(FAKE, 0, 128, FAKE, FAKE, FAKE, FAKE, 0))
-    assert f(bad, 2, 256, 1, None) == _lib.ERR_INVALID_ARG
-    bad = (P * 2)(good, P(FAKE, FAKE + 2, 128, FAKE, FAKE, FAKE, FAKE, 0))
-    assert f(bad, 2, 256, 1, None) == _lib.ERR_MISALIGNED
+    assert f(arr, -1, 1, None) == _lib.ERR_INVALID_ARG
+    assert f(None, 2, 1, None) == _lib.ERR_INVALID_ARG
+    assert f(arr, 0, 1, None) == _lib.OK
+    assert f(arr, 2, 0, None) == _lib.OK
+    assert f(arr, 2, -3, None) == _lib.ERR_INVALID_ARG
+    assert f((P * 2)(good, prob(K=200)), 2, 1, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert f((P * 2)(good, prob(y=MISALIGNED)), 2, 1, None) == _lib.ERR_MISALIGNED
+    assert f((P * 2)(good, prob(alpha=0)), 2, 1, None) == _lib.ERR_INVALID_ARG
+    assert f((P * 2)(good, prob(alpha=FAKE + 2)), 2, 1, None) == _lib.ERR_MISALIGNED
+    if name == "bitlinear_gemv_grouped":
+        assert f(arr, 2, 17, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    else:
+        assert f((P * 2)(good, prob(M=200)), 2, 1, None) == _lib.ERR_UNSUPPORTED_SHAPE

@@ -180,6 +180,47 @@ def test_gemv_grouped_many_problems_and_row_views():
     assert np.array_equal(torch.cat(ys).cpu().numpy(), ref["y"])
 
 
+def _mixed_layers(shapes, N, seed):
+    layers, refs, qs = [], [], []
+    for i, (M, K) in enumerate(shapes):
+        W = inputs.latent_weights(M, K, seed=seed + 7 * i)
+        x = inputs.activations(N, K, seed=seed + 7 * i + 500, outlier_frac=0.01)
+        refs.append(oracle.bitlinear(W.numpy(), x.numpy()))
+        layers.append(api.pack_weights(W.cuda()))
+        qs.append(api.quant_act(x.cuda()))
+    return layers, refs, [q[0] for q in qs], [q[1] for q in qs], [q[2] for q in qs]
+
+
+@pytest.mark.parametrize("N", [1, 3, 16])
+def test_gemv_grouped_mixed_k(N):
+    shapes = [(2560, 2560), (640, 2560), (2560, 6912), (96, 11008), (33, 128)]
+    layers, refs, xq, amax, xsum = _mixed_layers(shapes, N, seed=300 + N)
+    ys, accs = api.gemv_grouped(layers, xq, amax, xsum, with_acc=True)
+    for y, acc, ref in zip(ys, accs, refs):
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+        assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("N", [1, 100, 512])
+def test_gemm_grouped_mixed_k(N):
+    shapes = [(512, 1024), (256, 4096), (384, 2816), (128, 128)]
+    layers, refs, xq, amax, xsum = _mixed_layers(shapes, N, seed=400 + N)
+    ys, accs = api.gemm_grouped(layers, xq, amax, xsum, with_acc=True)
+    for y, acc, ref in zip(ys, accs, refs):
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+        assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
+def test_gemm_grouped_more_than_one_launch():
+    # 10 layers > 8 per launch
+    shapes = [(128 * (1 + i % 3), 256 * (1 + i % 2)) for i in range(10)]
+    layers, refs, xq, amax, xsum = _mixed_layers(shapes, 40, seed=500)
+    ys, accs = api.gemm_grouped(layers, xq, amax, xsum, with_acc=True)
+    for y, acc, ref in zip(ys, accs, refs):
+        assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+        assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
 @pytest.mark.parametrize("M,K,N", [(128, 128, 1), (256, 512, 200), (384, 1024, 129),
                                    (128, 256, 16), (1024, 2560, 512), (512, 4096, 300),
                                    (256, 6912, 77)])
