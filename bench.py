@@ -8,7 +8,7 @@ path at N=1 on the BitNet-b1.58-2B-shaped workload -- 30 decoder layers x 7
 BitLinear projections (q 2560x2560, k/v 640x2560, o 2560x2560, gate/up
 6912x2560, down 2560x6912), every linear fed one token.  One step:
 
-    quant_act(90 x 2560 activation rows)   quant_act(30 x 6912 rows)
+    quant_act_grouped(90 x 2560 and 30 x 6912 activation rows, one launch)
     gemv_grouped(all 210 layers, one launch)
 
 i.e. per-token absmax int8 quantisation of every layer input and the ternary x
@@ -160,6 +160,8 @@ class DecodeWorkload:
             self.ys.append(ys_l)
         self.prob = _lib.make_problems(entries)
         self.n_prob = len(entries)
+        self.acts = _lib.make_acts([(self.Xh, self.XQh, self.AMh, self.XSh),
+                                    (self.Xf, self.XQf, self.AMf, self.XSf)])
         self.packed_bytes = sum(M * K // 4 for row in self.weights for _, _, M, K in row)
         # algorithmic bytes of the grouped GEMV launch: packed weights, the int8
         # activations and alpha/amax/xsum each layer reads, and its fp32 outputs
@@ -173,20 +175,14 @@ class DecodeWorkload:
         return (self.XQh[r:r + 1], self.AMh[r:r + 1], self.XSh[r:r + 1])
 
     # each call launches exactly one kernel
-    def quant_h(self, s):
-        _lib.check(_lib.bitlinear_quant_act(self.Xh, self.Xh.shape[0], self.Xh.shape[1],
-                                            self.XQh, self.AMh, self.XSh, s), "quant_act")
-
-    def quant_f(self, s):
-        _lib.check(_lib.bitlinear_quant_act(self.Xf, self.Xf.shape[0], self.Xf.shape[1],
-                                            self.XQf, self.AMf, self.XSf, s), "quant_act")
+    def quant(self, s):
+        _lib.check(_lib.bitlinear_quant_act_grouped(self.acts, 2, s), "quant_act_grouped")
 
     def gemv(self, s):
         _lib.check(_lib.bitlinear_gemv_grouped(self.prob, self.n_prob, 1, s), "gemv_grouped")
 
     def step(self, s):
-        self.quant_h(s)
-        self.quant_f(s)
+        self.quant(s)
         self.gemv(s)
 
     def chain_step(self, s):
@@ -237,11 +233,11 @@ class PrefillWorkload:
             xq, am, xs = self.Q[self.src[p]]
             ents.append((packed, alpha, M, K, xq, am, xs, self.Y[p], None))
         self.prob = _lib.make_problems(ents)
+        self.acts = _lib.make_acts([(x,) + tuple(q) for x, q in zip(self.X, self.Q)])
 
-    def quant(self, i, s):
-        x = self.X[i]
-        xq, am, xs = self.Q[i]
-        _lib.check(_lib.bitlinear_quant_act(x, x.shape[0], x.shape[1], xq, am, xs, s), "quant")
+    def quant_all(self, s):
+        """The four distinct layer inputs in one launch."""
+        _lib.check(_lib.bitlinear_quant_act_grouped(self.acts, 4, s), "quant_act_grouped")
 
     def gemm(self, p, s):
         """One projection alone (for the per-projection breakdown)."""
@@ -272,8 +268,7 @@ def measure_prefill(dev, s, peaks, K):
     pre = PrefillWorkload(dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(3):
-        for i in range(4):
-            pre.quant(i, s)
+        pre.quant_all(s)
         pre.gemm_all(s)
     torch.cuda.synchronize()
     P = max(10, min(200, K // 50))
@@ -282,8 +277,7 @@ def measure_prefill(dev, s, peaks, K):
         flush_l2(flush)
         e = events(3)
         e[0].record(s)
-        for i in range(4):
-            pre.quant(i, s)
+        pre.quant_all(s)
         e[1].record(s)
         pre.gemm_all(s)
         e[2].record(s)
@@ -360,8 +354,8 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- headline: K timed decode steps, events around every launch
     K = args.steps
-    names = ("quant_h", "quant_f", "gemv")
-    ev = events(4 * K + 2)
+    names = ("quant", "gemv")
+    ev = events(3 * K + 2)
     for e in ev:              # create every event before the timed region
         e.record(s)
     torch.cuda.synchronize()
@@ -371,14 +365,12 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ev[-2].record(s)
     for i in range(K):
-        e = ev[4 * i:4 * i + 4]
+        e = ev[3 * i:3 * i + 3]
         e[0].record(s)
-        dec.quant_h(s)
+        dec.quant(s)
         e[1].record(s)
-        dec.quant_f(s)
-        e[2].record(s)
         dec.gemv(s)
-        e[3].record(s)
+        e[2].record(s)
     ev[-1].record(s)
     torch.cuda.synchronize()
     barrier()
@@ -386,7 +378,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = max_over_ranks(ev[-2].elapsed_time(ev[-1]))
     per = {k: 0.0 for k in names}
     for i in range(K):
-        e = ev[4 * i:4 * i + 4]
+        e = ev[3 * i:3 * i + 3]
         for j, k in enumerate(names):
             per[k] += e[j].elapsed_time(e[j + 1])
     per = {k: v / K for k, v in per.items()}
@@ -476,7 +468,7 @@ def run_ours(args, rank, world, local_rank):
                 "workload": "BitNet-b1.58-2B-shaped decode: 30 layers x 7 projections, N=1",
                 "layers": dec.layers, "tokens": 1,
                 "packed_bytes_per_step": dec.packed_bytes,
-                "launches_per_step": 3,
+                "launches_per_step": 2,
                 "l2": "no flush: 521 MB of packed weights per step > 126 MB L2",
                 "parallelism": "replicas" if world > 1 else "single GPU",
             },
@@ -503,7 +495,7 @@ def run_ours(args, rank, world, local_rank):
             "e2e": {"value": round(world * dec.packed_bytes / (e2e_ms * 1e-3) / 1e9, 1),
                     "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * K,
+            "gpu_launches": 2 * K,
             "clocks": clk,
             "cpu_baseline": cpu,
         }

@@ -112,6 +112,26 @@ BITLINEAR_API bitlinear_status bitlinear_quant_act(const float* x, int64_t N, in
                                      int8_t* xq, float* amax, int32_t* xsum,
                                      bitlinear_stream_t stream);
 
+/* One activation matrix of a grouped quantisation call (same conventions and
+ * results as bitlinear_quant_act, per matrix). */
+typedef struct {
+    const float* x;           /* [N, K] fp32 */
+    int64_t N;
+    int64_t K;
+    int8_t* xq;               /* [N, K] output */
+    float* amax;              /* [N] output */
+    int32_t* xsum;            /* [N] output, or NULL */
+} bitlinear_act;
+
+/*
+ * Quantise several activation matrices (e.g. every layer input of a decode
+ * step) in one launch per 64 matrices.  `acts` is a HOST array of `count`
+ * entries, read during the call only.
+ */
+BITLINEAR_API bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* acts,
+                                                           int64_t count,
+                                                           bitlinear_stream_t stream);
+
 /* ----------------------------------------------------------------- matmul */
 
 /*

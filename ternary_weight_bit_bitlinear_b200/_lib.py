@@ -28,6 +28,12 @@ class Problem(ctypes.Structure):
                 ("y", ctypes.c_void_p), ("acc", ctypes.c_void_p)]
 
 
+class Act(ctypes.Structure):
+    """Mirror of bitlinear_act (include/bitlinear.h)."""
+    _fields_ = [("x", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("xq", ctypes.c_void_p), ("amax", ctypes.c_void_p), ("xsum", ctypes.c_void_p)]
+
+
 class BitLinearError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -57,6 +63,8 @@ def load(path: str = LIB_PATH):
     L.bitlinear_pack_weights.restype = st
     L.bitlinear_pack_weights_noalloc.argtypes = [p, i64, i64, p, p, p]
     L.bitlinear_pack_weights_noalloc.restype = st
+    L.bitlinear_quant_act_grouped.argtypes = [ctypes.POINTER(Act), i64, p]
+    L.bitlinear_quant_act_grouped.restype = st
     L.bitlinear_quant_act.argtypes = [p, i64, i64, p, p, p, p]
     L.bitlinear_quant_act.restype = st
     for name in ("bitlinear_gemv", "bitlinear_gemm"):
@@ -115,6 +123,22 @@ def bitlinear_pack_weights_noalloc(W, M, K, packed, alpha, stream=None):
 
 def bitlinear_quant_act(x, N, K, xq, amax, xsum, stream=None):
     return load().bitlinear_quant_act(_p(x), N, K, _p(xq), _p(amax), _p(xsum), _stream(stream))
+
+
+def make_acts(entries):
+    """entries: iterable of (x, xq, amax, xsum-or-None) tensors.  Returns a
+    ctypes array of Act."""
+    entries = list(entries)
+    arr = (Act * max(1, len(entries)))()
+    for i, (x, xq, amax, xsum) in enumerate(entries):
+        arr[i] = Act(x.data_ptr(), x.shape[0], x.shape[1], xq.data_ptr(), amax.data_ptr(),
+                     0 if xsum is None else xsum.data_ptr())
+    return arr
+
+
+def bitlinear_quant_act_grouped(acts, count, stream=None):
+    """acts: a ctypes array from make_acts()."""
+    return load().bitlinear_quant_act_grouped(acts, count, _stream(stream))
 
 
 def bitlinear_gemv(packed, alpha, M, K, xq, amax, xsum, N, y, acc=None, stream=None):

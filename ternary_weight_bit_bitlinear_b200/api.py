@@ -49,6 +49,24 @@ def quant_act(x, stream=None, with_sum=True):
     return xq, amax, xsum
 
 
+def quant_act_grouped(xs, stream=None):
+    """Quantise several fp32 activation matrices in one launch; returns a list
+    of (xq, amax, xsum)."""
+    outs, entries = [], []
+    for x in xs:
+        _need(x, torch.float32, "x")
+        N, K = x.shape
+        o = (torch.empty((N, K), dtype=torch.int8, device=x.device),
+             torch.empty(N, dtype=torch.float32, device=x.device),
+             torch.empty(N, dtype=torch.int32, device=x.device))
+        outs.append(o)
+        entries.append((x,) + o)
+    arr = _lib.make_acts(entries)
+    _lib.check(_lib.bitlinear_quant_act_grouped(arr, len(entries), stream),
+               "bitlinear_quant_act_grouped")
+    return outs
+
+
 def _matmul(fn, name, packed, alpha, xq, amax, xsum, M, with_acc, stream, out=None):
     _need(packed, torch.int32, "packed")
     _need(alpha, torch.float32, "alpha")

@@ -308,16 +308,51 @@ bitlinear_status bitlinear_pack_weights(const float* W, int64_t M, int64_t K, ui
 
 bitlinear_status bitlinear_quant_act(const float* x, int64_t N, int64_t K, int8_t* xq,
                                      float* amax, int32_t* xsum, bitlinear_stream_t stream) {
-  if (N < 0 || K < 0) return BITLINEAR_ERR_INVALID_ARG;
-  if (K == 0 || K % 128 != 0 || K > kMaxK || N > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  if (N == 0) return BITLINEAR_OK;
-  if (!x || !xq || !amax) return BITLINEAR_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(xq) || !aligned4(amax) || (xsum && !aligned4(xsum)))
-    return BITLINEAR_ERR_MISALIGNED;
+  const bitlinear_act a = {x, N, K, xq, amax, xsum};
+  return bitlinear_quant_act_grouped(&a, 1, stream);
+}
+
+bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* acts, int64_t count,
+                                             bitlinear_stream_t stream) {
+  if (count < 0 || (count > 0 && !acts)) return BITLINEAR_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < count; ++i) {
+    const bitlinear_act& a = acts[i];
+    if (a.N < 0 || a.K < 0) return BITLINEAR_ERR_INVALID_ARG;
+    if (a.K == 0 || a.K % 128 != 0 || a.K > kMaxK || a.N > INT_MAX)
+      return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    if (a.N == 0) continue;
+    if (!a.x || !a.xq || !a.amax) return BITLINEAR_ERR_INVALID_ARG;
+    if (!aligned16(a.x) || !aligned16(a.xq) || !aligned4(a.amax) || (a.xsum && !aligned4(a.xsum)))
+      return BITLINEAR_ERR_MISALIGNED;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  bl::quant_act_kernel<<<static_cast<int>(N), bl::kQuantThreads, 0, s>>>(x, static_cast<int>(K),
-                                                                          xq, amax, xsum);
-  return launch_status();
+  bl::QuantParams p;
+  memset(&p, 0, sizeof p);
+  int64_t rows = 0;
+  auto flush = [&]() -> bitlinear_status {
+    if (p.count == 0) return BITLINEAR_OK;
+    bl::quant_rows_kernel<<<static_cast<int>(rows), bl::kQuantThreads, 0, s>>>(p);
+    memset(&p, 0, sizeof p);
+    rows = 0;
+    return launch_status();
+  };
+  for (int64_t i = 0; i < count; ++i) {
+    const bitlinear_act& a = acts[i];
+    if (a.N == 0) continue;
+    if (p.count == bl::kQuantMaxMatrices || rows + a.N > INT_MAX) {
+      bitlinear_status st = flush();
+      if (st != BITLINEAR_OK) return st;
+    }
+    bl::QuantMatrix& m = p.m[p.count++];
+    m.x = a.x;
+    m.xq = a.xq;
+    m.amax = a.amax;
+    m.xsum = a.xsum;
+    m.K = static_cast<int>(a.K);
+    m.row_begin = static_cast<int>(rows);
+    rows += a.N;
+  }
+  return flush();
 }
 
 bitlinear_status bitlinear_gemv(const uint32_t* packed, const float* alpha, int64_t M, int64_t K,

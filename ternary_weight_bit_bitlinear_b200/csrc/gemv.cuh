@@ -38,7 +38,7 @@ constexpr int kGemvMaxProblems = 256;
 
 template <int NT>
 struct GemvCfg {
-  static constexpr int kStages = NT <= 4 ? 4 : (NT <= 8 ? 3 : 2);
+  static constexpr int kStages = NT <= 4 ? 4 : 2;   // powers of two: the ring index is a mask
   static constexpr int kWeightBytes = kGemvTileRows * kGemvChunkBytes;    // 4 KB
   static constexpr int kStageBytes = kWeightBytes + NT * kGemvChunkK;
   static constexpr int kWarpBytes = kStages * kStageBytes;
@@ -72,24 +72,46 @@ __device__ __forceinline__ int gemv_locate(const GemvParams& p, int unit) {
   return lo;
 }
 
-// Issue the copies of k-chunk `kc` of the unit starting at row0 into `st`.
+// Per-lane copy plan of one unit, fixed for all its k-chunks.  Lane l copies
+// the 16-byte chunk (l % 8) of rows row0 + 4i + l/8, i = 0..7.
+struct GemvCopyPlan {
+  const uint8_t* wsrc;     // chunk (l % 8) of row row0 + l/8 at k-chunk 0
+  int64_t wstep;           // bytes from one of this lane's rows to the next (4 rows)
+  uint32_t dst_even;       // stage offset of copy i = 0 (even i add i * 512)
+  uint32_t dst_odd;        // stage offset of copy i = 1 minus 512 (odd i add (i-1) * 512)
+  int vrows;               // copies i < vrows have a row inside the layer
+  int wword;               // word index of this lane's chunk within a k-chunk
+};
+
+__device__ __forceinline__ GemvCopyPlan gemv_plan(const GemvProblem& pr, int row0, int lane) {
+  GemvCopyPlan cp;
+  const int rr = lane >> 3, c = lane & 7;
+  cp.wsrc = reinterpret_cast<const uint8_t*>(pr.packed) +
+            static_cast<int64_t>(row0 + rr) * pr.W * 4 + c * 16;
+  cp.wstep = static_cast<int64_t>(pr.W) * 16;
+  cp.dst_even = rr * kGemvChunkBytes + ((c ^ rr) << 4);
+  cp.dst_odd = 512 + rr * kGemvChunkBytes + ((c ^ (rr + 4)) << 4);
+  cp.vrows = max(0, min(8, (pr.M - row0 - rr + 3) / 4));
+  cp.wword = 4 * c;
+  return cp;
+}
+
+// Issue the copies of k-chunk `kc` into stage buffer `st`.  Weight chunks
+// outside the layer are skipped (rows past M are never stored; past the last
+// word, the activations are zero, so stale bytes multiply zeros).
 template <int NT>
-__device__ __forceinline__ void gemv_issue(const GemvProblem& pr, int row0, int kc, uint8_t* st,
-                                           int lane) {
-  // weights: 32 rows x 8 sixteen-byte chunks; a warp instruction copies 4
-  // whole 128-byte row segments (coalesced)
-  const int c = lane & 7;
-  const int word = kc * (kGemvChunkBytes / 4) + c * 4;
-  const bool kval = word < pr.W;
+__device__ __forceinline__ void gemv_issue(const GemvProblem& pr, const GemvCopyPlan& cp, int kc,
+                                           uint8_t* st, int lane) {
+  if (kc * (kGemvChunkBytes / 4) + cp.wword < pr.W) {
+    const uint8_t* src = cp.wsrc + kc * kGemvChunkBytes;
 #pragma unroll
-  for (int i = 0; i < kGemvTileRows / 4; ++i) {
-    const int r = i * 4 + (lane >> 3);
-    const int row = row0 + r;
-    const bool ok = kval && row < pr.M;
-    const uint32_t* src = ok ? pr.packed + static_cast<int64_t>(row) * pr.W + word : pr.packed;
-    cp_async16(st + r * kGemvChunkBytes + ((c ^ (r & 7)) << 4), src, ok ? 16u : 0u);
+    for (int i = 0; i < kGemvTileRows / 4; ++i) {
+      if (i < cp.vrows)
+        cp_async16(st + ((i & 1) ? cp.dst_odd + (i - 1) * 512 : cp.dst_even + i * 512), src, 16u);
+      src += cp.wstep;
+    }
   }
-  // activations: 512 bytes per token, 16 per lane
+  // activations: 512 bytes per token, 16 per lane, zero-filled past K
   const int k0 = kc * kGemvChunkK + lane * 16;
   const bool xval = k0 < pr.K;
 #pragma unroll
@@ -114,6 +136,7 @@ gemv_tile_kernel(const __grid_constant__ GemvParams p) {
     const GemvProblem& pr = p.prob[gemv_locate(p, u)];
     const int row0 = (u - pr.unit_begin) * kGemvTileRows;
     const int nchunks = (pr.K + kGemvChunkK - 1) / kGemvChunkK;
+    const GemvCopyPlan cp = gemv_plan(pr, row0, lane);
 
     int acc[NT][4];
 #pragma unroll
@@ -123,13 +146,13 @@ gemv_tile_kernel(const __grid_constant__ GemvParams p) {
 
 #pragma unroll
     for (int s = 0; s < C::kStages - 1; ++s) {
-      if (s < nchunks) gemv_issue<NT>(pr, row0, s, ring + s * C::kStageBytes, lane);
+      if (s < nchunks) gemv_issue<NT>(pr, cp, s, ring + s * C::kStageBytes, lane);
       cp_async_commit();
     }
     for (int kc = 0; kc < nchunks; ++kc) {
       const int nxt = kc + C::kStages - 1;
       if (nxt < nchunks)
-        gemv_issue<NT>(pr, row0, nxt, ring + (nxt % C::kStages) * C::kStageBytes, lane);
+        gemv_issue<NT>(pr, cp, nxt, ring + (nxt % C::kStages) * C::kStageBytes, lane);
       cp_async_commit();
       cp_async_wait<C::kStages - 1>();
       __syncwarp();

@@ -3,36 +3,77 @@
 // The I2_S setting quantises activations to int8 with an absmax scale
 // ("Bitnet.cpp" reading notes, section 2.3 and section 4.1); here one scale
 // per token row.  q = clamp(rint(x * (127/amax)), -128, 127), ties to even.
-// One CTA per token: a warp-shuffle max reduction, then a second pass that
-// quantises, stores four int8 per 32-bit word and reduces the row sum.
+//
+// One CTA per token row, rows of several matrices numbered across one launch.
+// Each thread loads its float4s of the row once and keeps up to kQuantRegF4 of
+// them in registers (rows up to 8192 wide are read exactly once); the maximum
+// is reduced with warp shuffles and one shared-memory exchange, the row is
+// quantised from registers, stored four int8 per 32-bit word, and the row sum
+// reduced the same way.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace bl {
 
-constexpr int kQuantThreads = 512;
+constexpr int kQuantThreads = 256;
+constexpr int kQuantRegF4 = 8;             // float4 per thread kept in registers
+constexpr int kQuantMaxMatrices = 64;
+
+struct QuantMatrix {
+  const float* x;
+  int8_t* xq;
+  float* amax;
+  int32_t* xsum;   // may be null
+  int K;
+  int row_begin;   // first global row of this matrix
+};
+
+struct QuantParams {
+  QuantMatrix m[kQuantMaxMatrices];
+  int count;
+};
 
 __device__ __forceinline__ int quant_one(float x, float s) {
   int v = __float2int_rn(__fmul_rn(x, s));   // NaN (0 * inf) -> 0; +-inf saturate
   return max(-128, min(127, v));
 }
 
+__device__ __forceinline__ uint32_t quant_pack4(float4 v, float s, int& sum) {
+  const int a = quant_one(v.x, s), b = quant_one(v.y, s), c = quant_one(v.z, s),
+            d = quant_one(v.w, s);
+  sum += a + b + c + d;
+  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | (static_cast<uint32_t>(d) << 24);
+}
+
+__device__ __forceinline__ float absmax4(float4 v) {
+  return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+}
+
 __global__ void __launch_bounds__(kQuantThreads)
-quant_act_kernel(const float* __restrict__ x, int K, int8_t* __restrict__ xq,
-                 float* __restrict__ amax_out, int32_t* __restrict__ xsum_out) {
+quant_rows_kernel(const __grid_constant__ QuantParams p) {
   __shared__ float red_f[kQuantThreads / 32];
   __shared__ int red_i[kQuantThreads / 32];
-  const int n = blockIdx.x;
-  const float4* row = reinterpret_cast<const float4*>(x + static_cast<int64_t>(n) * K);
-  const int K4 = K / 4;
+  const int g = blockIdx.x;
+  int mi = 0;
+  while (mi + 1 < p.count && g >= p.m[mi + 1].row_begin) ++mi;
+  const QuantMatrix& A = p.m[mi];
+  const int n = g - A.row_begin;
+  const int K4 = A.K / 4;
+  const float4* row = reinterpret_cast<const float4*>(A.x + static_cast<int64_t>(n) * A.K);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
+  float4 v[kQuantRegF4];
   float m = 0.0f;
-  for (int i = threadIdx.x; i < K4; i += blockDim.x) {
-    float4 v = __ldg(row + i);
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+#pragma unroll
+  for (int j = 0; j < kQuantRegF4; ++j) {
+    const int i = threadIdx.x + j * kQuantThreads;
+    v[j] = i < K4 ? __ldg(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    m = fmaxf(m, absmax4(v[j]));
   }
+  for (int i = threadIdx.x + kQuantRegF4 * kQuantThreads; i < K4; i += kQuantThreads)
+    m = fmaxf(m, absmax4(__ldg(row + i)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   if (lane == 0) red_f[warp] = m;
@@ -41,23 +82,22 @@ quant_act_kernel(const float* __restrict__ x, int K, int8_t* __restrict__ xq,
 #pragma unroll
   for (int w = 0; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, red_f[w]);
 
-  uint32_t* out = reinterpret_cast<uint32_t*>(xq + static_cast<int64_t>(n) * K);
+  uint32_t* out = reinterpret_cast<uint32_t*>(A.xq + static_cast<int64_t>(n) * A.K);
   int sum = 0;
   if (amax == 0.0f) {
-    for (int i = threadIdx.x; i < K4; i += blockDim.x) out[i] = 0u;
+    for (int i = threadIdx.x; i < K4; i += kQuantThreads) out[i] = 0u;
   } else {
     const float s = __fdiv_rn(127.0f, amax);
-    for (int i = threadIdx.x; i < K4; i += blockDim.x) {
-      float4 v = __ldg(row + i);
-      int a = quant_one(v.x, s), b = quant_one(v.y, s), c = quant_one(v.z, s),
-          d = quant_one(v.w, s);
-      sum += a + b + c + d;
-      out[i] = (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-               ((static_cast<uint32_t>(c) & 0xFFu) << 16) | (static_cast<uint32_t>(d) << 24);
+#pragma unroll
+    for (int j = 0; j < kQuantRegF4; ++j) {
+      const int i = threadIdx.x + j * kQuantThreads;
+      if (i < K4) out[i] = quant_pack4(v[j], s, sum);
     }
+    for (int i = threadIdx.x + kQuantRegF4 * kQuantThreads; i < K4; i += kQuantThreads)
+      out[i] = quant_pack4(__ldg(row + i), s, sum);
   }
-  if (threadIdx.x == 0) amax_out[n] = amax;
-  if (xsum_out) {
+  if (threadIdx.x == 0) A.amax[n] = amax;
+  if (A.xsum) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
     if (lane == 0) red_i[warp] = sum;
@@ -66,7 +106,7 @@ quant_act_kernel(const float* __restrict__ x, int K, int8_t* __restrict__ xq,
       int t = 0;
 #pragma unroll
       for (int w = 0; w < kQuantThreads / 32; ++w) t += red_i[w];
-      xsum_out[n] = t;
+      A.xsum[n] = t;
     }
   }
 }

@@ -150,3 +150,20 @@ def test_grouped_argument_errors(L, name):
         assert f(arr, 2, 17, None) == _lib.ERR_UNSUPPORTED_SHAPE
     else:
         assert f((P * 2)(good, prob(M=200)), 2, 1, None) == _lib.ERR_UNSUPPORTED_SHAPE
+
+
+def test_quant_act_grouped_argument_errors(L):
+    f = L.bitlinear_quant_act_grouped
+    A = _lib.Act
+    good = A(FAKE, 4, 256, FAKE, FAKE, FAKE)
+    assert f(None, 1, None) == _lib.ERR_INVALID_ARG
+    assert f((A * 1)(good), -1, None) == _lib.ERR_INVALID_ARG
+    assert f((A * 1)(good), 0, None) == _lib.OK
+    assert f((A * 2)(good, A(FAKE, 4, 100, FAKE, FAKE, FAKE)), 2, None) == \
+        _lib.ERR_UNSUPPORTED_SHAPE
+    assert f((A * 2)(good, A(FAKE, -1, 256, FAKE, FAKE, FAKE)), 2, None) == _lib.ERR_INVALID_ARG
+    assert f((A * 2)(good, A(0, 4, 256, FAKE, FAKE, FAKE)), 2, None) == _lib.ERR_INVALID_ARG
+    assert f((A * 2)(good, A(FAKE, 4, 256, MISALIGNED, FAKE, FAKE)), 2, None) == \
+        _lib.ERR_MISALIGNED
+    assert f((A * 2)(good, A(FAKE, 4, 256, FAKE, FAKE + 1, FAKE)), 2, None) == \
+        _lib.ERR_MISALIGNED

@@ -116,6 +116,17 @@ def test_quant_act_edge_cases():
     assert xq[3, :6].tolist() == [0, 2, 2, 0, -2, -2]
 
 
+def test_quant_act_grouped_parity():
+    shapes = [(90, 2560), (30, 6912), (0, 1024), (5, 131072), (1, 128), (64, 8192), (3, 8320)]
+    xs = [inputs.activations(N, K, seed=N + K, outlier_frac=0.01) for N, K in shapes]
+    outs = api.quant_act_grouped([x.cuda() for x in xs])
+    for x, (xq, amax, xsum) in zip(xs, outs):
+        q_ref, a_ref, s_ref = oracle.quant_act(x.numpy())
+        assert np.array_equal(xq.cpu().numpy(), q_ref)
+        assert np.array_equal(amax.cpu().numpy(), a_ref)
+        assert np.array_equal(xsum.cpu().numpy(), s_ref)
+
+
 # ----------------------------------------------------------------------------- matmul
 
 def _layer(M, K, N, seed, outlier_frac=0.0):
