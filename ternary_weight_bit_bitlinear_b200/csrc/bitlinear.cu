@@ -162,6 +162,21 @@ bitlinear_status gemv_group(const bitlinear_problem* probs, int64_t count, int64
   return BITLINEAR_OK;
 }
 
+// 2-D fp32 tensor [rows][cols], box {box_cols, box_rows}, no swizzle.
+bool encode_f32_2d(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows,
+                   uint32_t box_cols, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int BN, int STAGES>
 bitlinear_status launch_gemm(const bl::GemmParams& p, DeviceInfo* dev, int slot, cudaStream_t s) {
   auto kernel = bl::gemm_i8_tcgen05_kernel<BN, STAGES>;
@@ -228,7 +243,9 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
                         static_cast<uint64_t>(q.M), bl::kGemmPackedRowBytes, bl::kGemmBM,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
           !encode_u8_2d(&p.tmB[i], q.xq, static_cast<uint64_t>(q.K), static_cast<uint64_t>(N),
-                        bl::kGemmBK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+                        bl::kGemmBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !encode_f32_2d(&p.tmY[i], q.y, static_cast<uint64_t>(q.M), static_cast<uint64_t>(N),
+                         32, 32))
         return BITLINEAR_ERR_CUDA;
       bl::GemmProblem& g = p.prob[i];
       g.alpha = q.alpha;
@@ -246,7 +263,7 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     if (tiles > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     p.num_problems = n;
     p.total_tiles = static_cast<int>(tiles);
-    st = wide ? launch_gemm<256, 4>(p, dev, 1, s) : launch_gemm<128, 6>(p, dev, 0, s);
+    st = wide ? launch_gemm<256, 3>(p, dev, 1, s) : launch_gemm<128, 5>(p, dev, 0, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;

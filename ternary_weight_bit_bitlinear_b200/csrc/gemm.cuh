@@ -15,7 +15,8 @@
 //               tcgen05.commit frees the stage; accumulators double-buffered
 //               in tensor memory so the epilogue of tile i overlaps tile i+1;
 //   warps 6-9   epilogue: tcgen05.ld, acc - xsum (removes the +1 code offset),
-//               rescale by alpha * amax/127, coalesced fp32 stores.
+//               rescale by alpha * amax/127, staged in shared memory per 32 x 32
+//               block and written by bulk tensor stores.
 //
 // Several independent problems (e.g. the projections of a layer) can share one
 // persistent launch: tiles are numbered across problems.
@@ -45,6 +46,7 @@ struct GemmProblem {
 struct GemmParams {
   CUtensorMap tmA[kGemmMaxProblems];   // packed weights as uint8 [M][K/4], box 32 x 128
   CUtensorMap tmB[kGemmMaxProblems];   // xq as uint8 [N][K], box 128 x BN, 128B swizzle
+  CUtensorMap tmY[kGemmMaxProblems];   // y as fp32 [N][M], box 32 x 32
   GemmProblem prob[kGemmMaxProblems];
   int num_problems;
   int total_tiles;
@@ -52,9 +54,12 @@ struct GemmParams {
 
 template <int BN, int STAGES>
 struct GemmSmem {
-  uint8_t b[STAGES][BN * kGemmBK];                          // 1024-aligned stages
+  // every array below up to ep_out is a multiple of 1024 bytes, so all of
+  // them start 1024-byte aligned
+  uint8_t b[STAGES][BN * kGemmBK];
   uint8_t a[STAGES][kGemmBM * kGemmBK];                     // unpacked codes+1
   uint8_t apk[STAGES][kGemmBM * kGemmPackedRowBytes];       // packed tile
+  float ep_out[4][2][32 * 32];   // per epilogue warp: two 32 (n) x 32 (m) fp32 blocks
   uint64_t full[STAGES];
   uint64_t unpacked[STAGES];
   uint64_t empty[STAGES];
@@ -218,10 +223,12 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     const uint32_t quarter = static_cast<uint32_t>(warp & 3);   // TMEM lanes 32q .. 32q+31
     const int r_in_tile = static_cast<int>(quarter) * 32 + lane;
     int it = 0;
+    int ep_buf = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++it) {
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
-      const GemmProblem& pr = p.prob[pi];
+      // by value: registers, not re-read from parameter space after each store
+      const GemmProblem pr = p.prob[pi];
       const uint32_t ab = it & 1, ap = (it >> 1) & 1;
       if (!mbar_wait(&s.tfull[ab], ap, abort)) break;
       tc_fence_after();
@@ -230,21 +237,26 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       float* sc = s.ep_scale[quarter];
       int* xs = s.ep_xsum[quarter];
       {
-        const float alpha = *pr.alpha;
+        // all loads in flight at once, then the divisions
+        const float alpha = __ldg(pr.alpha);
+        float am[BN / 32];
+        int xv[BN / 32];
+#pragma unroll
+        for (int k = 0; k < BN / 32; ++k) {
+          const int n = n_blk * BN + k * 32 + lane;
+          am[k] = n < pr.N ? __ldg(pr.amax + n) : 0.0f;
+          xv[k] = n < pr.N ? __ldg(pr.xsum + n) : 0;
+        }
         __syncwarp();
-        for (int i = lane; i < BN; i += 32) {
-          const int n = n_blk * BN + i;
-          float v = 0.0f;
-          int x = 0;
-          if (n < pr.N) {
-            v = __fmul_rn(alpha, __fdiv_rn(__ldg(pr.amax + n), 127.0f));
-            x = __ldg(pr.xsum + n);
-          }
-          sc[i] = v;
-          xs[i] = x;
+#pragma unroll
+        for (int k = 0; k < BN / 32; ++k) {
+          sc[k * 32 + lane] = __fmul_rn(alpha, __fdiv_rn(am[k], 127.0f));
+          xs[k * 32 + lane] = xv[k];
         }
         __syncwarp();
       }
+      // Each 32 (token) x 32 (row) block is staged in shared memory, [n][m],
+      // and written with one bulk tensor store; two staging buffers per warp.
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t r[32];
@@ -252,20 +264,29 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + ab * BN + cc * 32, r);
         tmem_ld_wait();
         const int n0 = n_blk * BN + cc * 32;
+        if (n0 >= pr.N) continue;          // tokens past N: nothing to store
+        float* blk = s.ep_out[quarter][ep_buf];
+        if (lane == 0) bulk_wait_group_read<1>();   // this buffer's previous store has read it
+        __syncwarp();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const int n = n0 + j;
-          if (n < pr.N) {
-            const int a = static_cast<int>(r[j]) - xs[cc * 32 + j];
-            const int64_t o = static_cast<int64_t>(n) * pr.M + m;
-            pr.y[o] = __fmul_rn(__int2float_rn(a), sc[cc * 32 + j]);
-            if (pr.acc) pr.acc[o] = a;
-          }
+          const int a = static_cast<int>(r[j]) - xs[cc * 32 + j];
+          blk[j * 32 + lane] = __fmul_rn(__int2float_rn(a), sc[cc * 32 + j]);
+          if (pr.acc && n0 + j < pr.N)
+            pr.acc[static_cast<int64_t>(n0 + j) * pr.M + m] = a;
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&p.tmY[pi], blk, m_blk * kGemmBM + static_cast<int>(quarter) * 32, n0);
+          bulk_commit_group();
+        }
+        ep_buf ^= 1;
       }
       tc_fence_before();
       mbar_arrive(&s.tempty[ab]);
     }
+    if (lane == 0) bulk_wait_group<0>();   // outputs written before the CTA retires
   }
 
   tc_fence_before();

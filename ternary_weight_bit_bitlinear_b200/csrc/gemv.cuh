@@ -133,7 +133,8 @@ gemv_tile_kernel(const __grid_constant__ GemvParams p) {
   const uint32_t sw = static_cast<uint32_t>(lane & 7);
 
   for (int u = blockIdx.x * kGemvWarps + warp; u < p.total_units; u += total_warps) {
-    const GemvProblem& pr = p.prob[gemv_locate(p, u)];
+    // by value: registers, not re-read from parameter space after each store
+    const GemvProblem pr = p.prob[gemv_locate(p, u)];
     const int row0 = (u - pr.unit_begin) * kGemvTileRows;
     const int nchunks = (pr.K + kGemvChunkK - 1) / kGemvChunkK;
     const GemvCopyPlan cp = gemv_plan(pr, row0, lane);
