@@ -5,7 +5,10 @@
 
 #include <climits>
 #include <cstdint>
+#include <algorithm>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "bitlinear.h"
 #include "gemm.cuh"
@@ -21,6 +24,23 @@ constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Launch with programmatic stream serialisation (see pdl_wait_prior_grid).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 bitlinear_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
@@ -107,7 +127,8 @@ bitlinear_status launch_gemv_tile(const bl::GemvParams& p, DeviceInfo* dev, cuda
   const int64_t upw = (p.total_units + cap - 1) / cap;
   const int64_t warps = (p.total_units + upw - 1) / upw;
   const int grid = static_cast<int>((warps + bl::kGemvWarps - 1) / bl::kGemvWarps);
-  kernel<<<grid, bl::kGemvThreads, smem, s>>>(p);
+  if (launch_pdl(kernel, grid, bl::kGemvThreads, smem, s, p) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
   return launch_status();
 }
 
@@ -188,7 +209,8 @@ bitlinear_status launch_gemm(const bl::GemmParams& p, DeviceInfo* dev, int slot,
     dev->gemm_attr_set[slot] = true;
   }
   const int grid = p.total_tiles < dev->sms ? p.total_tiles : dev->sms;
-  kernel<<<grid, bl::kGemmThreads, smem, s>>>(p);
+  if (launch_pdl(kernel, grid, bl::kGemmThreads, smem, s, p) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
   return launch_status();
 }
 
@@ -209,6 +231,43 @@ bitlinear_status check_matmul_args(const uint32_t* packed, const float* alpha, i
 
 bitlinear_status check_problem(const bitlinear_problem& q, int64_t N) {
   return check_matmul_args(q.packed, q.alpha, q.M, q.K, q.xq, q.amax, q.xsum, N, q.y, q.acc);
+}
+
+// Longest-processing-time-first schedule: tiles (already ordered by K,
+// descending) go one by one to the CTA with the least work so far (cost = K,
+// the tile's main-loop length).  Skipped when the grid or the tile count does
+// not fit the parameter tables; the kernel then takes tiles round-robin.
+void build_gemm_schedule(bl::GemmParams& p, int sms) {
+  const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+  p.use_sched = 0;
+  if (grid > bl::kGemmMaxGrid || p.total_tiles > bl::kGemmMaxSched || p.num_problems < 2) return;
+  std::vector<std::pair<int64_t, int>> heap;   // (load, cta), min-heap
+  heap.reserve(grid);
+  for (int c = 0; c < grid; ++c) heap.push_back({0, c});
+  std::vector<int> owner(p.total_tiles);
+  std::vector<int> count(grid, 0);
+  auto cmp = [](const std::pair<int64_t, int>& a, const std::pair<int64_t, int>& b) {
+    return a.first != b.first ? a.first > b.first : a.second > b.second;
+  };
+  std::make_heap(heap.begin(), heap.end(), cmp);
+  for (int pi = 0; pi < p.num_problems; ++pi) {
+    const bl::GemmProblem& g = p.prob[pi];
+    const int end = pi + 1 < p.num_problems ? p.prob[pi + 1].tile_begin : p.total_tiles;
+    for (int t = g.tile_begin; t < end; ++t) {
+      std::pop_heap(heap.begin(), heap.end(), cmp);
+      auto& least = heap.back();
+      owner[t] = least.second;
+      count[least.second] += 1;
+      least.first += g.K;
+      std::push_heap(heap.begin(), heap.end(), cmp);
+    }
+  }
+  p.sched_begin[0] = 0;
+  for (int c = 0; c < grid; ++c)
+    p.sched_begin[c + 1] = static_cast<uint16_t>(p.sched_begin[c] + count[c]);
+  std::vector<int> fill(p.sched_begin, p.sched_begin + grid);
+  for (int t = 0; t < p.total_tiles; ++t) p.sched[fill[owner[t]]++] = static_cast<uint16_t>(t);
+  p.use_sched = 1;
 }
 
 // Tensor-core GEMM over problems that share N (all validated, M % 128 == 0):
@@ -263,6 +322,7 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     if (tiles > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     p.num_problems = n;
     p.total_tiles = static_cast<int>(tiles);
+    build_gemm_schedule(p, dev->sms);
     st = wide ? launch_gemm<256, 3>(p, dev, 1, s) : launch_gemm<128, 5>(p, dev, 0, s);
     if (st != BITLINEAR_OK) return st;
   }
@@ -348,10 +408,11 @@ bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* acts, int64_t 
   int64_t rows = 0;
   auto flush = [&]() -> bitlinear_status {
     if (p.count == 0) return BITLINEAR_OK;
-    bl::quant_rows_kernel<<<static_cast<int>(rows), bl::kQuantThreads, 0, s>>>(p);
+    const cudaError_t e =
+        launch_pdl(bl::quant_rows_kernel, static_cast<int>(rows), bl::kQuantThreads, 0, s, p);
     memset(&p, 0, sizeof p);
     rows = 0;
-    return launch_status();
+    return e == cudaSuccess ? launch_status() : BITLINEAR_ERR_CUDA;
   };
   for (int64_t i = 0; i < count; ++i) {
     const bitlinear_act& a = acts[i];

@@ -31,6 +31,8 @@ constexpr int kGemmBK = 128;                       // int8 elements per k-block
 constexpr int kGemmPackedRowBytes = kGemmBK / 4;   // 32 bytes of 2-bit fields
 constexpr int kGemmThreads = 320;                  // 10 warps
 constexpr int kGemmMaxProblems = 8;
+constexpr int kGemmMaxGrid = 160;      // CTAs a host-built schedule can describe
+constexpr int kGemmMaxSched = 4096;    // tiles a host-built schedule can describe
 
 struct GemmProblem {
   const float* alpha;
@@ -50,7 +52,25 @@ struct GemmParams {
   GemmProblem prob[kGemmMaxProblems];
   int num_problems;
   int total_tiles;
+  // Tile schedule: with use_sched, CTA b runs sched[sched_begin[b] ..
+  // sched_begin[b+1]) in that order (built on the host, longest tiles first,
+  // each to the least-loaded CTA); otherwise tiles b, b + grid, b + 2 grid...
+  int use_sched;
+  uint16_t sched_begin[kGemmMaxGrid + 1];
+  uint16_t sched[kGemmMaxSched];
 };
+
+__device__ __forceinline__ int gemm_my_count(const GemmParams& p) {
+  if (p.use_sched) return p.sched_begin[blockIdx.x + 1] - p.sched_begin[blockIdx.x];
+  return static_cast<int>(blockIdx.x) < p.total_tiles
+             ? (p.total_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+             : 0;
+}
+
+__device__ __forceinline__ int gemm_my_tile(const GemmParams& p, int i) {
+  if (p.use_sched) return p.sched[p.sched_begin[blockIdx.x] + i];
+  return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+}
 
 template <int BN, int STAGES>
 struct GemmSmem {
@@ -87,6 +107,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Smem = GemmSmem<BN, STAGES>;
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
   const uint32_t base = smem_u32(smem_raw);
   Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
 
@@ -127,7 +149,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
-      for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+      for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti) {
+        const int tile = gemm_my_tile(p, ti);
         int pi, m_blk, n_blk;
         gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
         const int kblocks = p.prob[pi].K / kGemmBK;
@@ -148,7 +171,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
       uint32_t stage = 0, phase = 0;
       int it = 0;
-      for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++it) {
+      for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti, ++it) {
+        const int tile = gemm_my_tile(p, ti);
         int pi, m_blk, n_blk;
         gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
         const int kblocks = p.prob[pi].K / kGemmBK;
@@ -192,7 +216,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     const int u = threadIdx.x - 64;   // weight row within the tile
     const uint32_t sw = static_cast<uint32_t>(u & 7);
     uint32_t stage = 0, phase = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+    for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti) {
+        const int tile = gemm_my_tile(p, ti);
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
       const int kblocks = p.prob[pi].K / kGemmBK;
@@ -224,7 +249,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     const int r_in_tile = static_cast<int>(quarter) * 32 + lane;
     int it = 0;
     int ep_buf = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++it) {
+    for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti, ++it) {
+        const int tile = gemm_my_tile(p, ti);
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
       // by value: registers, not re-read from parameter space after each store

@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(kGemvThreads)
 gemv_tile_kernel(const __grid_constant__ GemvParams p) {
   using C = GemvCfg<NT>;
   extern __shared__ __align__(128) uint8_t smem[];
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* ring = smem + warp * C::kWarpBytes;
   const int total_warps = gridDim.x * kGemvWarps;

@@ -28,6 +28,21 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ PDL
+// Programmatic dependent launch.  Kernels launched with the programmatic
+// stream-serialisation attribute may start while the previous kernel of the
+// stream is finishing; griddepcontrol.wait blocks until that kernel has
+// completed and its memory is visible.  Every library kernel waits before its
+// first global access, so nothing is ever read early; what overlaps is the
+// launch and the CTA set-up.
+__device__ __forceinline__ void pdl_wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_allow_next_grid() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -55,10 +55,12 @@ __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_kernel(const __grid_constant__ QuantParams p) {
   __shared__ float red_f[kQuantThreads / 32];
   __shared__ int red_i[kQuantThreads / 32];
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
   const int g = blockIdx.x;
   int mi = 0;
   while (mi + 1 < p.count && g >= p.m[mi + 1].row_begin) ++mi;
-  const QuantMatrix& A = p.m[mi];
+  const QuantMatrix A = p.m[mi];   // by value: registers, not parameter-space reloads
   const int n = g - A.row_begin;
   const int K4 = A.K / 4;
   const float4* row = reinterpret_cast<const float4*>(A.x + static_cast<int64_t>(n) * A.K);

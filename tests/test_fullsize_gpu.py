@@ -1,0 +1,167 @@
+"""Parity at the full sizes of the benchmark configurations, in the launch
+configuration the benchmark times (grouped quantisation, one grouped GEMV
+launch per 256 layers, one grouped GEMM launch per 8 layers), checked on
+sampled outputs the oracle computes one by one.
+
+For a sampled layer the oracle gets the whole latent weight tensor on the
+host (alpha is a whole-tensor statistic), ternarises only the sampled rows and
+quantises the sampled tokens.  Packed words of the sampled rows, alpha, the
+int8 activations and the fp32 outputs must match exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ternary_weight_bit_bitlinear_b200 import api, build, _lib, inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    _lib.load()
+    yield
+    torch.cuda.empty_cache()
+    assert _lib.bitlinear_device_error(clear=True) == _lib.OK
+
+
+def _input_proj(p):
+    return 0 if p < 3 else 3 if p == 3 else 4 if p < 6 else 6
+
+
+class Model:
+    """All layers of one model shape, packed on the device; inputs per layer."""
+
+    def __init__(self, cfg, layers, N, outlier_frac=0.0):
+        wl = inputs.WORKLOADS[cfg]
+        self.cfg, self.shape, self.layers, self.N = cfg, wl.model, layers, N
+        self.w = {}
+        for l in range(layers):
+            for p, (_, M, K) in enumerate(self.shape.projections()):
+                W = inputs.latent_weights(M, K, inputs.weight_seed(cfg, l, p), device="cuda")
+                self.w[(l, p)] = api.pack_weights(W)
+                del W
+        self.x = {}
+        for l in range(layers):
+            for p in (0, 3, 4, 6):
+                K = self.shape.ffn if p == 6 else self.shape.hidden
+                self.x[(l, p)] = inputs.activations(N, K, inputs.act_seed(cfg, l, p),
+                                                    device="cuda", outlier_frac=outlier_frac)
+        keys = sorted(self.x)
+        outs = api.quant_act_grouped([self.x[k] for k in keys])
+        self.q = dict(zip(keys, outs))
+
+    def layer_list(self):
+        return [(l, p) for l in range(self.layers) for p in range(7)]
+
+    def run_gemv(self):
+        lst = self.layer_list()
+        qs = [self.q[(l, _input_proj(p))] for l, p in lst]
+        ys = api.gemv_grouped([self.w[k] for k in lst], [q[0] for q in qs], [q[1] for q in qs],
+                              [q[2] for q in qs])
+        return dict(zip(lst, ys))
+
+    def run_gemm(self, layer):
+        lst = [(layer, p) for p in range(7)]
+        qs = [self.q[(l, _input_proj(p))] for l, p in lst]
+        ys = api.gemm_grouped([self.w[k] for k in lst], [q[0] for q in qs], [q[1] for q in qs],
+                              [q[2] for q in qs])
+        return dict(zip(lst, ys))
+
+    def check(self, l, p, y, rows, tokens):
+        _, M, K = self.shape.projections()[p]
+        W = inputs.latent_weights(M, K, inputs.weight_seed(self.cfg, l, p),
+                                  device="cuda").cpu().numpy()
+        alpha = oracle.absmean(W)
+        packed, a_dev = self.w[(l, p)]
+        assert a_dev.item() == alpha
+        Wr = W[rows]
+        del W
+        codes = oracle.ternarize(Wr, alpha)
+        assert np.array_equal(packed[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+                              .view(np.uint32), oracle.pack(codes))
+        x = self.x[(l, _input_proj(p))][torch.as_tensor(tokens, device="cuda")].cpu().numpy()
+        q, amax, qsum = oracle.quant_act(x)
+        xq_dev = self.q[(l, _input_proj(p))][0][torch.as_tensor(tokens, device="cuda")]
+        assert np.array_equal(xq_dev.cpu().numpy(), q)
+        acc = oracle.matmul_i32(codes, q)
+        y_ref = oracle.rescale(acc, alpha, amax)
+        y_dev = y[torch.as_tensor(tokens, device="cuda")][:, torch.as_tensor(rows, device="cuda")]
+        assert np.array_equal(y_dev.cpu().numpy(), y_ref)
+
+
+def _rows(M, n, seed):
+    r = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, M - 1], r.integers(0, M, n)]))
+    return rows
+
+
+def test_config1_single_1024_gemv():
+    wl = inputs.WORKLOADS[1]
+    M, K = wl.single
+    W = inputs.latent_weights(M, K, inputs.weight_seed(1, 0, 0), device="cuda")
+    x = inputs.activations(1, K, inputs.act_seed(1, 0, 0), device="cuda",
+                           outlier_count=wl.outlier_count)
+    ref = oracle.bitlinear(W.cpu().numpy(), x.cpu().numpy())
+    packed, alpha = api.pack_weights(W)
+    xq, amax, xsum = api.quant_act(x)
+    y, acc = api.gemv(packed, alpha, xq, amax, xsum, with_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
+def test_config2_2b_decode_stream_30_layers():
+    m = Model(2, 30, 1)
+    ys = m.run_gemv()
+    for (l, p) in [(0, 0), (7, 1), (15, 4), (29, 6), (29, 3)]:
+        M = m.shape.projections()[p][1]
+        m.check(l, p, ys[(l, p)], _rows(M, 40, 10 * l + p), [0])
+
+
+def test_config3_7b_prefill_512_grouped():
+    m = Model(3, 1, 512)
+    ys = m.run_gemm(0)
+    for p in range(7):
+        M = m.shape.projections()[p][1]
+        m.check(0, p, ys[(0, p)], _rows(M, 24, p), np.arange(512))
+
+
+@pytest.mark.parametrize("N", [1, 2, 4, 8, 16, 32, 64, 128])
+def test_config4_8b_batch_sweep(N):
+    m = Model(4, 2, N, outlier_frac=0.01)
+    # the dispatcher used at each N: GEMV up to 16 tokens, tensor cores above
+    for l in range(2):
+        for p in (0, 1, 4, 6):
+            packed, alpha = m.w[(l, p)]
+            xq, amax, xsum = m.q[(l, _input_proj(p))]
+            y = api.matmul(packed, alpha, xq, amax, xsum)
+            M = m.shape.projections()[p][1]
+            m.check(l, p, y, _rows(M, 12, N + p), np.arange(N))
+
+
+def test_config5_70b_weight_stream_and_prefill():
+    m = Model(5, 80, 1)
+    # 80 layers x 855,638,016 weights at 2 bits: 17,112,760,320 bytes
+    assert sum(pk.numel() * 4 for pk, _ in m.w.values()) == 80 * m.shape.weights_per_layer() // 4 \
+        == 17_112_760_320
+    ys = m.run_gemv()
+    for (l, p) in [(0, 0), (40, 1), (79, 5), (79, 6)]:
+        M = m.shape.projections()[p][1]
+        m.check(l, p, ys[(l, p)], _rows(M, 16, l + p), [0])
+    del ys
+    # prefill N = 2048 on one layer of the same weights
+    N = 2048
+    x = {p: inputs.activations(N, m.shape.ffn if p == 6 else m.shape.hidden,
+                               inputs.act_seed(5, 0, p) + 7, device="cuda") for p in (0, 3, 4, 6)}
+    m.x.update({(0, p): v for p, v in x.items()})
+    outs = api.quant_act_grouped([x[p] for p in (0, 3, 4, 6)])
+    m.q.update({(0, p): o for p, o in zip((0, 3, 4, 6), outs)})
+    ys = m.run_gemm(0)
+    tokens = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(5).integers(0, N, 30)]))
+    for p in (0, 1, 4, 6):
+        M = m.shape.projections()[p][1]
+        m.check(0, p, ys[(0, p)], _rows(M, 8, 100 + p), tokens)
