@@ -8,6 +8,7 @@
 // Work unit: 32 consecutive rows of one layer, one row per lane, all of its K
 // (layers of one launch may differ in K).
 // Each warp runs its own pipeline of k-chunks (512 weights = 128 bytes per row,
+// continuing from one unit into the next without draining,
 // plus the matching 512 int8 activations of every token), brought in with
 // 16-byte cp.async copies into a STAGES-deep ring in shared memory.  A row's
 // 16-byte chunks are stored XOR-swizzled by row (chunk c of row r at c ^ r%8),
@@ -131,15 +132,48 @@ gemv_tile_kernel(const __grid_constant__ GemvParams p) {
   pdl_allow_next_grid();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* ring = smem + warp * C::kWarpBytes;
-  const int total_warps = gridDim.x * kGemvWarps;
+  const int stride = gridDim.x * kGemvWarps;
   const uint32_t sw = static_cast<uint32_t>(lane & 7);
 
-  for (int u = blockIdx.x * kGemvWarps + warp; u < p.total_units; u += total_warps) {
+  // The copy side runs ahead of the compute side through this warp's whole
+  // sequence of (unit, k-chunk) pairs, across unit boundaries, so the ring
+  // stays full from the first unit to the last.
+  int iu = blockIdx.x * kGemvWarps + warp;   // unit and chunk to issue next
+  int ic = 0;
+  GemvProblem ipr;
+  GemvCopyPlan icp;
+  int inchunks = 0;
+  if (iu < p.total_units) {
+    ipr = p.prob[gemv_locate(p, iu)];
+    icp = gemv_plan(ipr, (iu - ipr.unit_begin) * kGemvTileRows, lane);
+    inchunks = (ipr.K + kGemvChunkK - 1) / kGemvChunkK;
+  }
+  int slot = 0;
+  auto issue_next = [&]() {
+    if (iu < p.total_units) {
+      gemv_issue<NT>(ipr, icp, ic, ring + slot * C::kStageBytes, lane);
+      if (++ic == inchunks) {
+        ic = 0;
+        iu += stride;
+        if (iu < p.total_units) {
+          ipr = p.prob[gemv_locate(p, iu)];
+          icp = gemv_plan(ipr, (iu - ipr.unit_begin) * kGemvTileRows, lane);
+          inchunks = (ipr.K + kGemvChunkK - 1) / kGemvChunkK;
+        }
+      }
+    }
+    cp_async_commit();   // one group per stage, empty once the sequence is done
+    slot = (slot + 1) & (C::kStages - 1);
+  };
+#pragma unroll 1
+  for (int s = 0; s < C::kStages - 1; ++s) issue_next();
+
+  int cslot = 0;
+  for (int cu = blockIdx.x * kGemvWarps + warp; cu < p.total_units; cu += stride) {
     // by value: registers, not re-read from parameter space after each store
-    const GemvProblem pr = p.prob[gemv_locate(p, u)];
-    const int row0 = (u - pr.unit_begin) * kGemvTileRows;
+    const GemvProblem pr = p.prob[gemv_locate(p, cu)];
+    const int row0 = (cu - pr.unit_begin) * kGemvTileRows;
     const int nchunks = (pr.K + kGemvChunkK - 1) / kGemvChunkK;
-    const GemvCopyPlan cp = gemv_plan(pr, row0, lane);
 
     int acc[NT][4];
 #pragma unroll
@@ -147,19 +181,12 @@ gemv_tile_kernel(const __grid_constant__ GemvParams p) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[t][j] = 0;
 
-#pragma unroll
-    for (int s = 0; s < C::kStages - 1; ++s) {
-      if (s < nchunks) gemv_issue<NT>(pr, cp, s, ring + s * C::kStageBytes, lane);
-      cp_async_commit();
-    }
     for (int kc = 0; kc < nchunks; ++kc) {
-      const int nxt = kc + C::kStages - 1;
-      if (nxt < nchunks)
-        gemv_issue<NT>(pr, cp, nxt, ring + (nxt % C::kStages) * C::kStageBytes, lane);
-      cp_async_commit();
+      issue_next();
       cp_async_wait<C::kStages - 1>();
       __syncwarp();
-      const uint8_t* st = ring + (kc % C::kStages) * C::kStageBytes;
+      const uint8_t* st = ring + cslot * C::kStageBytes;
+      cslot = (cslot + 1) & (C::kStages - 1);
       const uint8_t* wrow = st + lane * kGemvChunkBytes;
       const uint8_t* xs = st + C::kWeightBytes;
 #pragma unroll
