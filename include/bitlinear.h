@@ -112,6 +112,24 @@ BITLINEAR_API bitlinear_status bitlinear_quant_act(const float* x, int64_t N, in
                                      int8_t* xq, float* amax, int32_t* xsum,
                                      bitlinear_stream_t stream);
 
+/*
+ * Per-tensor variant of bitlinear_quant_act: one absmax over the whole x
+ * [N,K], as in the reading notes' I2_S setting (section 2.3 "technical
+ * details", section 4.1: per-tensor int8 activations).  Every amax[n] receives
+ * that one maximum and every element uses s = 127/amax; the results feed
+ * bitlinear_gemv / bitlinear_gemm unchanged.  At N = 1 it equals the
+ * per-token call.
+ *   workspace: device scratch of bitlinear_quant_act_per_tensor_workspace_bytes()
+ *   bytes (16-byte aligned, contents need not be initialised; it is cleared on
+ *   the stream).  Two launches.
+ */
+BITLINEAR_API size_t bitlinear_quant_act_per_tensor_workspace_bytes(void);
+BITLINEAR_API bitlinear_status bitlinear_quant_act_per_tensor(const float* x, int64_t N, int64_t K,
+                                                              int8_t* xq, float* amax,
+                                                              int32_t* xsum, void* workspace,
+                                                              size_t workspace_bytes,
+                                                              bitlinear_stream_t stream);
+
 /* One activation matrix of a grouped quantisation call (same conventions and
  * results as bitlinear_quant_act, per matrix). */
 typedef struct {

@@ -39,6 +39,8 @@ def lib():
         L.oracle_unpack.restype = ctypes.c_int
         L.oracle_quant_act.argtypes = [p, i64, i64, p, p, p]
         L.oracle_quant_act.restype = None
+        L.oracle_quant_act_per_tensor.argtypes = [p, i64, i64, p, p, p]
+        L.oracle_quant_act_per_tensor.restype = None
         L.oracle_matmul_i32.argtypes = [p, i64, i64, p, i64, p]
         L.oracle_matmul_i32.restype = None
         L.oracle_matmul_addsub.argtypes = [p, i64, i64, p, i64, p]
@@ -110,6 +112,18 @@ def quant_act(x):
     amax = np.empty(N, dtype=np.float32)
     qsum = np.empty(N, dtype=np.int32)
     lib().oracle_quant_act(px, N, K, q.ctypes.data, amax.ctypes.data, qsum.ctypes.data)
+    return q, amax, qsum
+
+
+def quant_act_per_tensor(x):
+    """x fp32 [N,K] -> (q, amax [N] all equal to max|x|, qsum [N])."""
+    x, px = _c(x, np.float32)
+    N, K = x.shape
+    q = np.empty((N, K), dtype=np.int8)
+    amax = np.empty(N, dtype=np.float32)
+    qsum = np.empty(N, dtype=np.int32)
+    lib().oracle_quant_act_per_tensor(px, N, K, q.ctypes.data, amax.ctypes.data,
+                                      qsum.ctypes.data)
     return q, amax, qsum
 
 

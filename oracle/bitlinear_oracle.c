@@ -246,6 +246,37 @@ void oracle_quant_act(const float* x, int64_t N, int64_t K,
     }
 }
 
+/* The reading notes' I2_S setting, section 2.3 "technical details" and
+ * section 4.1 "lossless inference conditions": per-tensor int8 activations.
+ * The same rule as above with the maximum taken over the whole tensor. */
+void oracle_quant_act_per_tensor(const float* x, int64_t N, int64_t K,
+                                 int8_t* q, float* amax, int32_t* qsum)
+{
+    float a = 0.0f;
+    for (int64_t i = 0; i < N * K; ++i) {
+        float v = fabsf(x[i]);
+        if (v > a) a = v;
+    }
+    for (int64_t n = 0; n < N; ++n) {
+        amax[n] = a;
+        int32_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            int v = 0;
+            if (a != 0.0f) {
+                float s = 127.0f / a;
+                float t = rintf(x[n * K + k] * s);
+                if (isnan(t)) v = 0;
+                else if (t > 127.0f) v = 127;
+                else if (t < -128.0f) v = -128;
+                else v = (int)t;
+            }
+            q[n * K + k] = (int8_t)v;
+            sum += v;
+        }
+        if (qsum) qsum[n] = sum;
+    }
+}
+
 /* ------------------------------------------------------------------------- */
 /* The mpGEMM: int32 accumulation of ternary x int8 products (reading notes   */
 /* section 4.1: MAD-based int8 multiply-add).                                */

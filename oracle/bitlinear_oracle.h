@@ -64,6 +64,11 @@ int oracle_unpack(const uint32_t* packed, int64_t M, int64_t K, int8_t* codes);
 void oracle_quant_act(const float* x, int64_t N, int64_t K,
                       int8_t* q, float* amax, int32_t* qsum);
 
+/* Per-tensor variant: one absmax over the whole x [N,K]; every amax[n] gets
+ * that value and every element uses s = 127/amax. */
+void oracle_quant_act_per_tensor(const float* x, int64_t N, int64_t K,
+                                 int8_t* q, float* amax, int32_t* qsum);
+
 /* Triple-loop int32 matmul acc[n*M+m] = sum_k codes[m*K+k] * q[n*K+k]. */
 void oracle_matmul_i32(const int8_t* codes, int64_t M, int64_t K,
                        const int8_t* q, int64_t N, int32_t* acc);

@@ -63,6 +63,10 @@ def load(path: str = LIB_PATH):
     L.bitlinear_pack_weights.restype = st
     L.bitlinear_pack_weights_noalloc.argtypes = [p, i64, i64, p, p, p]
     L.bitlinear_pack_weights_noalloc.restype = st
+    L.bitlinear_quant_act_per_tensor_workspace_bytes.argtypes = []
+    L.bitlinear_quant_act_per_tensor_workspace_bytes.restype = sz
+    L.bitlinear_quant_act_per_tensor.argtypes = [p, i64, i64, p, p, p, p, sz, p]
+    L.bitlinear_quant_act_per_tensor.restype = st
     L.bitlinear_quant_act_grouped.argtypes = [ctypes.POINTER(Act), i64, p]
     L.bitlinear_quant_act_grouped.restype = st
     L.bitlinear_quant_act.argtypes = [p, i64, i64, p, p, p, p]
@@ -123,6 +127,13 @@ def bitlinear_pack_weights_noalloc(W, M, K, packed, alpha, stream=None):
 
 def bitlinear_quant_act(x, N, K, xq, amax, xsum, stream=None):
     return load().bitlinear_quant_act(_p(x), N, K, _p(xq), _p(amax), _p(xsum), _stream(stream))
+
+
+def bitlinear_quant_act_per_tensor(x, N, K, xq, amax, xsum, workspace, workspace_bytes,
+                                   stream=None):
+    return load().bitlinear_quant_act_per_tensor(_p(x), N, K, _p(xq), _p(amax), _p(xsum),
+                                                 _p(workspace), workspace_bytes,
+                                                 _stream(stream))
 
 
 def make_acts(entries):

@@ -49,6 +49,20 @@ def quant_act(x, stream=None, with_sum=True):
     return xq, amax, xsum
 
 
+def quant_act_per_tensor(x, stream=None):
+    """Per-tensor variant: one absmax over all of x; amax[n] holds it for every n."""
+    _need(x, torch.float32, "x")
+    N, K = x.shape
+    xq = torch.empty((N, K), dtype=torch.int8, device=x.device)
+    amax = torch.empty(N, dtype=torch.float32, device=x.device)
+    xsum = torch.empty(N, dtype=torch.int32, device=x.device)
+    nbytes = _lib.load().bitlinear_quant_act_per_tensor_workspace_bytes()
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    _lib.check(_lib.bitlinear_quant_act_per_tensor(x, N, K, xq, amax, xsum, ws, nbytes, stream),
+               "bitlinear_quant_act_per_tensor")
+    return xq, amax, xsum
+
+
 def quant_act_grouped(xs, stream=None):
     """Quantise several fp32 activation matrices in one launch; returns a list
     of (xq, amax, xsum)."""

@@ -433,6 +433,48 @@ bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* acts, int64_t 
   return flush();
 }
 
+size_t bitlinear_quant_act_per_tensor_workspace_bytes(void) { return 16; }
+
+bitlinear_status bitlinear_quant_act_per_tensor(const float* x, int64_t N, int64_t K, int8_t* xq,
+                                                float* amax, int32_t* xsum, void* workspace,
+                                                size_t workspace_bytes,
+                                                bitlinear_stream_t stream) {
+  if (N < 0 || K < 0) return BITLINEAR_ERR_INVALID_ARG;
+  if (K == 0 || K % 128 != 0 || K > kMaxK || N > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0) return BITLINEAR_OK;
+  if (!x || !xq || !amax) return BITLINEAR_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < 16) return BITLINEAR_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(xq) || !aligned4(amax) || (xsum && !aligned4(xsum)) ||
+      !aligned16(workspace))
+    return BITLINEAR_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  bitlinear_status st = device_info(&dev);
+  if (st != BITLINEAR_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto* word = static_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(word, 0, 4, s) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  const int64_t n4 = N * K / 4;
+  int64_t g = (n4 + bl::kQuantThreads - 1) / bl::kQuantThreads;
+  if (g > dev->sms * 8) g = dev->sms * 8;
+  if (launch_pdl(bl::tensor_absmax_kernel, static_cast<int>(g), bl::kQuantThreads, 0, s,
+                 reinterpret_cast<const float4*>(x), n4, word) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  bl::QuantParams p;
+  memset(&p, 0, sizeof p);
+  p.count = 1;
+  p.m[0].x = x;
+  p.m[0].xq = xq;
+  p.m[0].amax = amax;
+  p.m[0].xsum = xsum;
+  p.m[0].tensor_amax = word;
+  p.m[0].K = static_cast<int>(K);
+  p.m[0].row_begin = 0;
+  if (launch_pdl(bl::quant_rows_kernel, static_cast<int>(N), bl::kQuantThreads, 0, s, p) !=
+      cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  return launch_status();
+}
+
 bitlinear_status bitlinear_gemv(const uint32_t* packed, const float* alpha, int64_t M, int64_t K,
                                 const int8_t* xq, const float* amax, const int32_t* xsum,
                                 int64_t N, float* y, int32_t* acc, bitlinear_stream_t stream) {

@@ -10,6 +10,11 @@
 // is reduced with warp shuffles and one shared-memory exchange, the row is
 // quantised from registers, stored four int8 per 32-bit word, and the row sum
 // reduced the same way.
+//
+// Per-tensor mode (the reading notes' own I2_S setting, section 2.3 and
+// section 4.1: one int8 scale for the whole activation tensor): a first
+// kernel folds max|x| over the matrix into one word, and the row kernel takes
+// that maximum instead of the row's.
 #pragma once
 
 #include "ptx.cuh"
@@ -25,6 +30,7 @@ struct QuantMatrix {
   int8_t* xq;
   float* amax;
   int32_t* xsum;   // may be null
+  const unsigned int* tensor_amax;   // per-tensor mode: bits of max|x| over the matrix
   int K;
   int row_begin;   // first global row of this matrix
 };
@@ -74,15 +80,19 @@ quant_rows_kernel(const __grid_constant__ QuantParams p) {
     v[j] = i < K4 ? __ldg(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
     m = fmaxf(m, absmax4(v[j]));
   }
-  for (int i = threadIdx.x + kQuantRegF4 * kQuantThreads; i < K4; i += kQuantThreads)
-    m = fmaxf(m, absmax4(__ldg(row + i)));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  if (lane == 0) red_f[warp] = m;
-  __syncthreads();
   float amax = 0.0f;
+  if (A.tensor_amax) {
+    amax = __uint_as_float(*A.tensor_amax);
+  } else {
+    for (int i = threadIdx.x + kQuantRegF4 * kQuantThreads; i < K4; i += kQuantThreads)
+      m = fmaxf(m, absmax4(__ldg(row + i)));
 #pragma unroll
-  for (int w = 0; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, red_f[w]);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) red_f[warp] = m;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, red_f[w]);
+  }
 
   uint32_t* out = reinterpret_cast<uint32_t*>(A.xq + static_cast<int64_t>(n) * A.K);
   int sum = 0;
@@ -110,6 +120,30 @@ quant_rows_kernel(const __grid_constant__ QuantParams p) {
       for (int w = 0; w < kQuantThreads / 32; ++w) t += red_i[w];
       A.xsum[n] = t;
     }
+  }
+}
+
+// Per-tensor maximum of |x| over n4 float4s, folded into *out (the bits of a
+// non-negative float order like unsigned integers, so atomicMax on them is
+// the float maximum).  *out must start at 0.
+__global__ void __launch_bounds__(kQuantThreads)
+tensor_absmax_kernel(const float4* __restrict__ x, int64_t n4, unsigned int* __restrict__ out) {
+  __shared__ float red[kQuantThreads / 32];
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+  float m = 0.0f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride)
+    m = fmaxf(m, absmax4(__ldg(x + i)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kQuantThreads / 32; ++w) b = fmaxf(b, red[w]);
+    atomicMax(out, __float_as_uint(b));
   }
 }
 

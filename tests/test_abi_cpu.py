@@ -167,3 +167,19 @@ def test_quant_act_grouped_argument_errors(L):
         _lib.ERR_MISALIGNED
     assert f((A * 2)(good, A(FAKE, 4, 256, FAKE, FAKE + 1, FAKE)), 2, None) == \
         _lib.ERR_MISALIGNED
+
+
+def test_quant_act_per_tensor_argument_errors(L):
+    f = L.bitlinear_quant_act_per_tensor
+    ws = L.bitlinear_quant_act_per_tensor_workspace_bytes()
+    assert ws >= 4
+    p = _p
+    assert f(p(FAKE), 2, 100, p(FAKE), p(FAKE), None, p(FAKE), ws, None) == \
+        _lib.ERR_UNSUPPORTED_SHAPE
+    assert f(p(FAKE), -2, 128, p(FAKE), p(FAKE), None, p(FAKE), ws, None) == _lib.ERR_INVALID_ARG
+    assert f(p(0), 2, 128, p(FAKE), p(FAKE), None, p(FAKE), ws, None) == _lib.ERR_INVALID_ARG
+    assert f(p(FAKE), 2, 128, p(FAKE), p(FAKE), None, p(0), ws, None) == _lib.ERR_WORKSPACE
+    assert f(p(FAKE), 2, 128, p(FAKE), p(FAKE), None, p(FAKE), 2, None) == _lib.ERR_WORKSPACE
+    assert f(p(FAKE), 2, 128, p(FAKE), p(FAKE), None, p(MISALIGNED), ws, None) == \
+        _lib.ERR_MISALIGNED
+    assert f(p(FAKE), 0, 128, p(FAKE), p(FAKE), None, p(FAKE), ws, None) == _lib.OK

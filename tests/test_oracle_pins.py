@@ -257,6 +257,28 @@ def test_quant_act_rounding_within_half_step():
     assert (err <= step * (0.5 + 1e-4)).all()   # s and x*s each round once
 
 
+def test_per_tensor_quant_pins():
+    x = inputs.activations(5, 256, seed=44, outlier_count=3).numpy()
+    q, amax, qsum = oracle.quant_act_per_tensor(x)
+    # one scale: every amax entry is max|x| over the tensor
+    assert (amax == np.abs(x).max()).all()
+    # a single token is the per-token rule
+    for n in range(5):
+        q1, a1, s1 = oracle.quant_act(x[n:n + 1])
+        qt, at, st = oracle.quant_act_per_tensor(x[n:n + 1])
+        assert np.array_equal(q1, qt) and a1[0] == at[0] and s1[0] == st[0]
+    # the token holding the tensor maximum quantises as it would per token
+    top = np.argmax(np.abs(x).max(axis=1))
+    assert np.array_equal(q[top], oracle.quant_act(x[top:top + 1])[0][0])
+    # hand values: amax = 127 gives s = 1, so q = rint(x) with ties to even
+    y = np.array([[0.5, 2.5, -1.5, 3.0], [127.0, -0.5, 1.5, 0.0]], np.float32)
+    qy, ay, sy = oracle.quant_act_per_tensor(y)
+    assert qy.tolist() == [[0, 2, -2, 3], [127, 0, 2, 0]] and sy.tolist() == [3, 129]
+    # all zero
+    qz, az, sz = oracle.quant_act_per_tensor(np.zeros((3, 128), np.float32))
+    assert not qz.any() and not az.any() and not sz.any()
+
+
 # ----------------------------------------------------------------------------- matmul
 
 @pytest.mark.parametrize("M,K,N", [(1, 16, 1), (5, 16, 3), (16, 16, 2), (7, 32, 3)])

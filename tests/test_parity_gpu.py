@@ -127,6 +127,45 @@ def test_quant_act_grouped_parity():
         assert np.array_equal(xsum.cpu().numpy(), s_ref)
 
 
+@pytest.mark.parametrize("N,K", [(1, 2560), (7, 1024), (64, 4096), (300, 6912), (2, 131072)])
+def test_quant_act_per_tensor_parity(N, K):
+    x = inputs.activations(N, K, seed=N * 5 + K, outlier_frac=0.01)
+    xq, amax, xsum = api.quant_act_per_tensor(x.cuda())
+    q_ref, a_ref, s_ref = oracle.quant_act_per_tensor(x.numpy())
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(amax.cpu().numpy(), a_ref)
+    assert np.array_equal(xsum.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("N", [3, 200])
+def test_per_tensor_activations_through_matmul(N):
+    M, K = 384, 2048
+    W = inputs.latent_weights(M, K, seed=61)
+    x = inputs.activations(N, K, seed=62, outlier_frac=0.01)
+    a = oracle.absmean(W.numpy())
+    codes = oracle.ternarize(W.numpy(), a)
+    q, amax, _ = oracle.quant_act_per_tensor(x.numpy())
+    acc = oracle.matmul_i32(codes, q)
+    y_ref = oracle.rescale(acc, a, amax)
+    packed, alpha = api.pack_weights(W.cuda())
+    xq, am, xs = api.quant_act_per_tensor(x.cuda())
+    y, acc_d = api.matmul(packed, alpha, xq, am, xs, with_acc=True)
+    assert np.array_equal(acc_d.cpu().numpy(), acc)
+    assert np.array_equal(y.cpu().numpy(), y_ref)
+
+
+def test_quant_act_per_tensor_edge_cases():
+    x = np.zeros((3, 256), np.float32)
+    xq, amax, xsum = api.quant_act_per_tensor(dev_t(x))
+    assert not xq.cpu().numpy().any() and not amax.cpu().numpy().any()
+    x[1, 7] = -127.0
+    x[2, :4] = [0.5, 1.5, 2.5, -2.5]
+    xq, amax, xsum = api.quant_act_per_tensor(dev_t(x))
+    q_ref, a_ref, s_ref = oracle.quant_act_per_tensor(x)
+    assert np.array_equal(xq.cpu().numpy(), q_ref) and (amax.cpu().numpy() == 127).all()
+    assert xq[2, :4].tolist() == [0, 2, 2, -2]
+
+
 # ----------------------------------------------------------------------------- matmul
 
 def _layer(M, K, N, seed, outlier_frac=0.0):
