@@ -46,6 +46,27 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "source": "fallback"}
 INT8_PER_BF16 = 2.0          # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
 
+# DRAM bytes (read + write) per launch from one ncu capture of each workload's
+# dominant kernel (summaries in profiles/).  They describe the kernel source
+# they were taken on, identified by a sha256 prefix: once that file changes
+# the figure no longer applies and the bench reports null.
+NCU_TRAFFIC = {
+    "gemv": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemv.cuh",
+             "sha256": "f891fc3c908a67f0", "bytes": 522_180_608 + 5_733_888,
+             "profile": "profiles/gemv_tile_2b_decode_stream.md"},
+}
+
+
+def ncu_traffic(kernel):
+    import hashlib
+    ent = NCU_TRAFFIC.get(kernel)
+    if not ent:
+        return None
+    with open(os.path.join(ROOT, ent["file"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != ent["sha256"]:
+            return None
+    return ent["bytes"]
+
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -311,7 +332,8 @@ def measure_prefill(dev, s, peaks, K):
                      "unit": "TOPS", "frac": round(tops / int8_peak, 4),
                      "peak_note": "int8 peak = measured bf16 burst x nominal int8:bf16 ratio 2 (%s)"
                                   % peaks["source"],
-                     "frac_of_nominal_4500": round(tops / 4500.0, 4), "traffic": None},
+                     "frac_of_nominal_4500": round(tops / 4500.0, 4),
+                     "traffic": ncu_traffic("gemm")},
         "l2": "256 MB buffer written between timed steps (flush)",
     }
     del flush
@@ -491,7 +513,8 @@ def run_ours(args, rank, world, local_rank):
                 "bytes_per_launch": dec.alg_bytes,
                 "avg_launch_ms": round(per["gemv"], 5),
                 "timing": "events around each launch, second pass of %d steps" % K2,
-                "traffic": None,
+                "traffic": ncu_traffic("gemv"),
+                "traffic_source": NCU_TRAFFIC["gemv"]["profile"],
             },
             "kernel_ms": {k: round(v, 5) for k, v in per.items()},
             "decode_chain": {

@@ -323,7 +323,7 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     p.num_problems = n;
     p.total_tiles = static_cast<int>(tiles);
     build_gemm_schedule(p, dev->sms);
-    st = wide ? launch_gemm<256, 3>(p, dev, 1, s) : launch_gemm<128, 5>(p, dev, 0, s);
+    st = wide ? launch_gemm<256, 4>(p, dev, 1, s) : launch_gemm<128, 7>(p, dev, 0, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;

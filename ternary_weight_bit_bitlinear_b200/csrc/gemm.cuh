@@ -10,7 +10,9 @@
 //               swizzle) into a STAGES-deep shared-memory ring;
 //   warps 2-5   unpackers: one weight row per thread, 2-bit fields -> int8
 //               codes+1 written in the 128-byte-swizzled K-major layout the
-//               MMA reads, then a proxy fence and an mbarrier arrive;
+//               MMA reads (a double buffer of its own, so the TMA ring only
+//               holds what is in flight from memory), then a proxy fence and an
+//               mbarrier arrive;
 //   warp 1      MMA issuer: 4 x tcgen05.mma kind::i8 (K = 32 each) per stage,
 //               tcgen05.commit frees the stage; accumulators double-buffered
 //               in tensor memory so the epilogue of tile i overlaps tile i+1;
@@ -31,6 +33,7 @@ constexpr int kGemmBK = 128;                       // int8 elements per k-block
 constexpr int kGemmPackedRowBytes = kGemmBK / 4;   // 32 bytes of 2-bit fields
 constexpr int kGemmThreads = 320;                  // 10 warps
 constexpr int kGemmMaxProblems = 8;
+constexpr int kGemmUnpackBufs = 2;    // unpacked A tiles live only from unpack to MMA
 constexpr int kGemmMaxGrid = 160;      // CTAs a host-built schedule can describe
 constexpr int kGemmMaxSched = 4096;    // tiles a host-built schedule can describe
 
@@ -76,13 +79,14 @@ template <int BN, int STAGES>
 struct GemmSmem {
   // every array below up to ep_out is a multiple of 1024 bytes, so all of
   // them start 1024-byte aligned
-  uint8_t b[STAGES][BN * kGemmBK];
-  uint8_t a[STAGES][kGemmBM * kGemmBK];                     // unpacked codes+1
-  uint8_t apk[STAGES][kGemmBM * kGemmPackedRowBytes];       // packed tile
+  uint8_t b[STAGES][BN * kGemmBK];                          // TMA ring: activations
+  uint8_t apk[STAGES][kGemmBM * kGemmPackedRowBytes];       // TMA ring: packed weights
+  uint8_t a[kGemmUnpackBufs][kGemmBM * kGemmBK];            // unpacked codes+1
   float ep_out[4][2][32 * 32];   // per epilogue warp: two 32 (n) x 32 (m) fp32 blocks
   uint64_t full[STAGES];
-  uint64_t unpacked[STAGES];
   uint64_t empty[STAGES];
+  uint64_t ufull[kGemmUnpackBufs];    // unpacked tile ready (128 arrivals)
+  uint64_t uempty[kGemmUnpackBufs];   // unpacked tile consumed by the MMAs (commit)
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -121,8 +125,11 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.unpacked[i], 128);
       mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < kGemmUnpackBufs; ++i) {
+      mbar_init(&s.ufull[i], 128);
+      mbar_init(&s.uempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
@@ -169,7 +176,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
-      uint32_t stage = 0, phase = 0;
+      uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
       int it = 0;
       for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti, ++it) {
         const int tile = gemm_my_tile(p, ti);
@@ -183,12 +190,12 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&s.full[stage], phase, abort) ||
-              !mbar_wait(&s.unpacked[stage], phase, abort)) {
+              !mbar_wait(&s.ufull[ub], uphase, abort)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(s.a[stage]);
+          const uint32_t a_addr = smem_u32(s.a[ub]);
           const uint32_t b_addr = smem_u32(s.b[stage]);
 #pragma unroll
           for (int kk = 0; kk < kGemmBK / 32; ++kk) {
@@ -196,7 +203,9 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
                       smem_desc_k_sw128(b_addr + 32 * kk), idesc, (kb | kk) != 0);
           }
           mma_commit(&s.empty[stage]);
+          mma_commit(&s.uempty[ub]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++ub == kGemmUnpackBufs) { ub = 0; uphase ^= 1u; }
         }
         if (!ok) break;
         mma_commit(&s.tfull[ab]);
@@ -215,18 +224,22 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     // ------------------------------------------------------------ unpackers
     const int u = threadIdx.x - 64;   // weight row within the tile
     const uint32_t sw = static_cast<uint32_t>(u & 7);
-    uint32_t stage = 0, phase = 0;
+    const int half = (u >> 2) & 1;   // read order of the two 16-byte halves: no bank conflict
+    uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
     for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti) {
         const int tile = gemm_my_tile(p, ti);
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
       const int kblocks = p.prob[pi].K / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(&s.full[stage], phase, abort)) goto unpack_done;
+        if (!mbar_wait(&s.full[stage], phase, abort) ||
+            !mbar_wait(&s.uempty[ub], uphase ^ 1u, abort))
+          goto unpack_done;
         const uint4* src = reinterpret_cast<const uint4*>(s.apk[stage] + u * kGemmPackedRowBytes);
-        const uint4 p0 = src[0], p1 = src[1];
+        const uint4 h0 = src[half], h1 = src[half ^ 1];
+        const uint4 p0 = half ? h1 : h0, p1 = half ? h0 : h1;
         const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        uint8_t* row = s.a[stage] + (u >> 3) * 1024 + (u & 7) * 128;
+        uint8_t* row = s.a[ub] + (u >> 3) * 1024 + (u & 7) * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t w = words[j];
@@ -238,8 +251,9 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
           *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(j) ^ sw) << 4)) = v;
         }
         fence_proxy_async_smem();
-        mbar_arrive(&s.unpacked[stage]);
+        mbar_arrive(&s.ufull[ub]);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++ub == kGemmUnpackBufs) { ub = 0; uphase ^= 1u; }
       }
     }
   unpack_done:;
