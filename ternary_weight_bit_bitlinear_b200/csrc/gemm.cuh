@@ -16,7 +16,8 @@
 //   warp 1      MMA issuer: 4 x tcgen05.mma kind::i8 (K = 32 each) per stage,
 //               tcgen05.commit frees the stage; accumulators double-buffered
 //               in tensor memory so the epilogue of tile i overlaps tile i+1;
-//   warps 6-9   epilogue: tcgen05.ld, acc - xsum (removes the +1 code offset),
+//   warps 6-13  epilogue, two warps per TMEM lane quarter, alternate 32-column
+//               chunks: tcgen05.ld, acc - xsum (removes the +1 code offset),
 //               rescale by alpha * amax/127, staged in shared memory per 32 x 32
 //               block and written by bulk tensor stores.
 //
@@ -31,7 +32,8 @@ namespace bl {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;                       // int8 elements per k-block
 constexpr int kGemmPackedRowBytes = kGemmBK / 4;   // 32 bytes of 2-bit fields
-constexpr int kGemmThreads = 320;                  // 10 warps
+constexpr int kGemmEpiWarps = 8;                   // two per TMEM lane quarter
+constexpr int kGemmThreads = (6 + kGemmEpiWarps) * 32;   // 14 warps
 constexpr int kGemmMaxProblems = 8;
 constexpr int kGemmUnpackBufs = 2;    // unpacked A tiles live only from unpack to MMA
 constexpr int kGemmMaxGrid = 160;      // CTAs a host-built schedule can describe
@@ -82,7 +84,7 @@ struct GemmSmem {
   uint8_t b[STAGES][BN * kGemmBK];                          // TMA ring: activations
   uint8_t apk[STAGES][kGemmBM * kGemmPackedRowBytes];       // TMA ring: packed weights
   uint8_t a[kGemmUnpackBufs][kGemmBM * kGemmBK];            // unpacked codes+1
-  float ep_out[4][2][32 * 32];   // per epilogue warp: two 32 (n) x 32 (m) fp32 blocks
+  float ep_out[kGemmEpiWarps][32 * 32];   // per epilogue warp: one 32 (n) x 32 (m) block
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t ufull[kGemmUnpackBufs];    // unpacked tile ready (128 arrivals)
@@ -90,8 +92,8 @@ struct GemmSmem {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
-  float ep_scale[4][BN];   // per epilogue warp: alpha * amax/127 of the tile's tokens
-  int ep_xsum[4][BN];      // per epilogue warp: activation sums of the tile's tokens
+  float ep_scale[kGemmEpiWarps][BN / 2];   // per epilogue warp: alpha * amax/127 of its tokens
+  int ep_xsum[kGemmEpiWarps][BN / 2];      // per epilogue warp: activation sums of its tokens
   uint32_t tmem_slot;
   int abort;
 };
@@ -133,7 +135,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], 128);
+      mbar_init(&s.tempty[i], kGemmEpiWarps * 32);
     }
     mbar_init(&s.drain, 1);
     s.abort = 0;
@@ -261,8 +263,9 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     // ------------------------------------------------------------ epilogue
     const uint32_t quarter = static_cast<uint32_t>(warp & 3);   // TMEM lanes 32q .. 32q+31
     const int r_in_tile = static_cast<int>(quarter) * 32 + lane;
+    const int e = warp - 6;                 // epilogue warp 0..7
+    const int half = e >> 2;                // this warp stores column chunks cc = half, half+2, ...
     int it = 0;
-    int ep_buf = 0;
     for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti, ++it) {
         const int tile = gemm_my_tile(p, ti);
       int pi, m_blk, n_blk;
@@ -274,44 +277,44 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       tc_fence_after();
       const int m = m_blk * kGemmBM + r_in_tile;
       // this warp's copy of the tile's per-token scale and sum
-      float* sc = s.ep_scale[quarter];
-      int* xs = s.ep_xsum[quarter];
+      float* sc = s.ep_scale[e];
+      int* xs = s.ep_xsum[e];
       {
         // all loads in flight at once, then the divisions
         const float alpha = __ldg(pr.alpha);
-        float am[BN / 32];
-        int xv[BN / 32];
+        float am[BN / 64];
+        int xv[BN / 64];
 #pragma unroll
-        for (int k = 0; k < BN / 32; ++k) {
-          const int n = n_blk * BN + k * 32 + lane;
+        for (int k = 0; k < BN / 64; ++k) {
+          const int n = n_blk * BN + (2 * k + half) * 32 + lane;
           am[k] = n < pr.N ? __ldg(pr.amax + n) : 0.0f;
           xv[k] = n < pr.N ? __ldg(pr.xsum + n) : 0;
         }
         __syncwarp();
 #pragma unroll
-        for (int k = 0; k < BN / 32; ++k) {
+        for (int k = 0; k < BN / 64; ++k) {
           sc[k * 32 + lane] = __fmul_rn(alpha, __fdiv_rn(am[k], 127.0f));
           xs[k * 32 + lane] = xv[k];
         }
         __syncwarp();
       }
       // Each 32 (token) x 32 (row) block is staged in shared memory, [n][m],
-      // and written with one bulk tensor store; two staging buffers per warp.
+      // and written with one bulk tensor store (one staging buffer per warp).
 #pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
+      for (int cc = half; cc < BN / 32; cc += 2) {
         uint32_t r[32];
         __syncwarp();
         tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + ab * BN + cc * 32, r);
         tmem_ld_wait();
         const int n0 = n_blk * BN + cc * 32;
         if (n0 >= pr.N) continue;          // tokens past N: nothing to store
-        float* blk = s.ep_out[quarter][ep_buf];
-        if (lane == 0) bulk_wait_group_read<1>();   // this buffer's previous store has read it
+        float* blk = s.ep_out[e];
+        if (lane == 0) bulk_wait_group_read<0>();   // the previous store has read the block
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const int a = static_cast<int>(r[j]) - xs[cc * 32 + j];
-          blk[j * 32 + lane] = __fmul_rn(__int2float_rn(a), sc[cc * 32 + j]);
+          const int a = static_cast<int>(r[j]) - xs[(cc >> 1) * 32 + j];
+          blk[j * 32 + lane] = __fmul_rn(__int2float_rn(a), sc[(cc >> 1) * 32 + j]);
           if (pr.acc && n0 + j < pr.N)
             pr.acc[static_cast<int64_t>(n0 + j) * pr.M + m] = a;
         }
@@ -321,7 +324,6 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
           tma_store_2d(&p.tmY[pi], blk, m_blk * kGemmBM + static_cast<int>(quarter) * 32, n0);
           bulk_commit_group();
         }
-        ep_buf ^= 1;
       }
       tc_fence_before();
       mbar_arrive(&s.tempty[ab]);
