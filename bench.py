@@ -54,6 +54,9 @@ NCU_TRAFFIC = {
     "gemv": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemv.cuh",
              "sha256": "f891fc3c908a67f0", "bytes": 522_180_608 + 5_733_888,
              "profile": "profiles/gemv_tile_2b_decode_stream.md"},
+    "gemm": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
+             "sha256": "7a558782e6ea35ab", "bytes": 62_585_600 + 31_000_064,
+             "profile": "profiles/gemm_i8_tcgen05_7b_prefill.md"},
 }
 
 
@@ -333,7 +336,8 @@ def measure_prefill(dev, s, peaks, K):
                      "peak_note": "int8 peak = measured bf16 burst x nominal int8:bf16 ratio 2 (%s)"
                                   % peaks["source"],
                      "frac_of_nominal_4500": round(tops / 4500.0, 4),
-                     "traffic": ncu_traffic("gemm")},
+                     "traffic": ncu_traffic("gemm"),
+                     "traffic_source": NCU_TRAFFIC["gemm"]["profile"]},
         "l2": "256 MB buffer written between timed steps (flush)",
     }
     del flush
