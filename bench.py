@@ -54,6 +54,9 @@ NCU_TRAFFIC = {
     "gemv": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemv.cuh",
              "sha256": "f891fc3c908a67f0", "bytes": 522_180_608 + 5_733_888,
              "profile": "profiles/gemv_tile_2b_decode_stream.md"},
+    "gemv_quant": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemv_quant.cuh",
+                   "sha256": "", "bytes": None,
+                   "profile": "profiles/gemv_quant_2b_decode_stream.md"},
     "gemm": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
              "sha256": "7a558782e6ea35ab", "bytes": 62_585_600 + 31_000_064,
              "profile": "profiles/gemm_i8_tcgen05_7b_prefill.md"},
@@ -184,12 +187,28 @@ class DecodeWorkload:
             self.ys.append(ys_l)
         self.prob = _lib.make_problems(entries)
         self.n_prob = len(entries)
+        # the same 210 linears on fp32 inputs for the fused quantise+GEMV kernel;
+        # projections that share an input get the same row view, side by side
+        fents = [(packed, alpha, M, K, self._x(l, p), self.ys[l][p], None)
+                 for l in range(L) for p, (packed, alpha, M, K) in enumerate(self.weights[l])]
+        self.fprob = _lib.make_fused_problems(fents)
         self.acts = _lib.make_acts([(self.Xh, self.XQh, self.AMh, self.XSh),
                                     (self.Xf, self.XQf, self.AMf, self.XSf)])
         self.packed_bytes = sum(M * K // 4 for row in self.weights for _, _, M, K in row)
         # algorithmic bytes of the grouped GEMV launch: packed weights, the int8
         # activations and alpha/amax/xsum each layer reads, and its fp32 outputs
         self.alg_bytes = sum(M * K // 4 + K + 12 + 4 * M for (_, _, M, K, *_r) in entries)
+        # ... and of the fused launch: packed weights, alpha and fp32 outputs per
+        # layer, plus every distinct fp32 input once
+        self.alg_bytes_fused = (sum(M * K // 4 + 4 + 4 * M for (_, _, M, K, *_r) in entries)
+                                + 4 * (self.Xh.numel() + self.Xf.numel()))
+
+    def _x(self, l, p):
+        """fp32 row view of the input projection p of layer l reads."""
+        if p == 6:
+            return self.Xf[l:l + 1]
+        r = 3 * l + (0 if p < 3 else 1 if p == 3 else 2)
+        return self.Xh[r:r + 1]
 
     def _act(self, l, p):
         """(xq, amax, xsum) row views of the input projection p of layer l reads."""
@@ -205,9 +224,27 @@ class DecodeWorkload:
     def gemv(self, s):
         _lib.check(_lib.bitlinear_gemv_grouped(self.prob, self.n_prob, 1, s), "gemv_grouped")
 
-    def step(self, s):
+    def two_step(self, s):
+        """Quantiser launch, then the GEMV launch."""
         self.quant(s)
         self.gemv(s)
+
+    def step(self, s):
+        """The decode path: one fused quantise+GEMV launch over all 210 linears."""
+        _lib.check(_lib.bitlinear_gemv_quant_grouped(self.fprob, self.n_prob, 1, s),
+                   "gemv_quant_grouped")
+
+    def chain_step_fused(self, s):
+        """The dependent per-layer order with the fused kernel: four launches
+        per layer (q/k/v, o, gate/up, down)."""
+        for l in range(self.layers):
+            w = self.weights[l]
+            for projs in ((0, 1, 2), (3,), (4, 5), (6,)):
+                ents = [(w[p][0], w[p][1], w[p][2], w[p][3], self._x(l, p), self.ys[l][p], None)
+                        for p in projs]
+                arr = _lib.make_fused_problems(ents)
+                _lib.check(_lib.bitlinear_gemv_quant_grouped(arr, len(ents), 1, s),
+                           "gemv_quant_grouped")
 
     def chain_step(self, s):
         """The order a real decoder imposes: per layer, quantise an input, then
@@ -376,13 +413,14 @@ def run_ours(args, rank, world, local_rank):
     dec = DecodeWorkload(dev)
     for _ in range(args.warmup):
         dec.step(s)
+        dec.two_step(s)
     torch.cuda.synchronize()
 
-    # ---- headline: K timed decode steps.  Only the ends carry events: an event
-    # between two launches would serialise the programmatic dependent launch
-    # that lets the GEMV start while the quantiser finishes.
+    # ---- headline: K timed decode steps, each one fused quantise+GEMV launch
+    # over the 210 linears.  Only the ends carry events: an event between two
+    # launches would serialise the programmatic dependent launch that lets one
+    # step's CTAs start while the previous step's last CTAs finish.
     K = args.steps
-    names = ("quant", "gemv")
     clocks = ClockSampler(local_rank)
     clocks.start()
     barrier()
@@ -397,60 +435,83 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     total_ms = max_over_ranks(t0.elapsed_time(t1))
 
-    # ---- kernel breakdown: a second pass over the same steps with events
-    # around every launch (these launches therefore do not overlap)
+    # ---- the two-step path (quantiser launch, then GEMV launch), same steps
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = events(2)
+    t0.record(s)
+    for i in range(K):
+        dec.two_step(s)
+    t1.record(s)
+    torch.cuda.synchronize()
+    barrier()
+    two_ms = max_over_ranks(t0.elapsed_time(t1)) / K
+
+    # ---- per-launch breakdown: a second pass with events around every launch
+    # (these launches therefore do not overlap)
     K2 = min(K, 4000)
-    ev = events(3 * K2)
+    ev = events(5 * K2)
     for e in ev:              # create every event before the timed pass
         e.record(s)
     torch.cuda.synchronize()
     for i in range(K2):
-        e = ev[3 * i:3 * i + 3]
+        e = ev[5 * i:5 * i + 5]
         e[0].record(s)
-        dec.quant(s)
+        dec.step(s)
         e[1].record(s)
-        dec.gemv(s)
         e[2].record(s)
+        dec.quant(s)
+        e[3].record(s)
+        dec.gemv(s)
+        e[4].record(s)
     torch.cuda.synchronize()
-    per = {k: 0.0 for k in names}
+    per = {"gemv_quant": 0.0, "quant": 0.0, "gemv": 0.0}
     for i in range(K2):
-        e = ev[3 * i:3 * i + 3]
-        for j, k in enumerate(names):
-            per[k] += e[j].elapsed_time(e[j + 1])
+        e = ev[5 * i:5 * i + 5]
+        per["gemv_quant"] += e[0].elapsed_time(e[1])
+        per["quant"] += e[2].elapsed_time(e[3])
+        per["gemv"] += e[3].elapsed_time(e[4])
     per = {k: v / K2 for k, v in per.items()}
     ms_per_step = total_ms / K
     gbs = world * dec.packed_bytes / (ms_per_step * 1e-3) / 1e9
+    fused_gbs = dec.alg_bytes_fused / (per["gemv_quant"] * 1e-3) / 1e9
     gemv_gbs = dec.alg_bytes / (per["gemv"] * 1e-3) / 1e9
     hbm_peak = peaks["hbm_gbs"]
     if args.only == "decode":
         print(json.dumps({"partial_run": "decode", "value": round(gbs, 1), "unit": "GB/s",
-                          "kernel_ms": per, "gemv_gbs": round(gemv_gbs, 1), "clocks": clk}))
+                          "two_step_gbs": round(dec.packed_bytes / (two_ms * 1e-3) / 1e9, 1),
+                          "kernel_ms": per, "gemv_quant_gbs": round(fused_gbs, 1),
+                          "gemv_gbs": round(gemv_gbs, 1), "clocks": clk}))
         return
 
-    # ---- dependent per-layer chain, CUDA graph
-    chain_ms = None
-    try:
-        gs = torch.cuda.Stream()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(gs):
-            dec.chain_step(gs)          # warm
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=gs):
-            dec.chain_step(gs)
-        for _ in range(3):
-            g.replay()
-        torch.cuda.synchronize()
-        reps = max(20, K // 50)
-        a, b = events(2)
-        a.record(s)
-        for _ in range(reps):
-            g.replay()
-        b.record(s)
-        torch.cuda.synchronize()
-        chain_ms = a.elapsed_time(b) / reps
-        del g
-    except Exception as exc:  # noqa: BLE001
-        chain_ms = "failed: %s" % exc
+    # ---- dependent per-layer chains, each in one CUDA graph
+    def time_graph(fn):
+        try:
+            gs = torch.cuda.Stream()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(gs):
+                fn(gs)          # warm
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=gs):
+                fn(gs)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            reps = max(20, K // 50)
+            a, b = events(2)
+            a.record(s)
+            for _ in range(reps):
+                g.replay()
+            b.record(s)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / reps
+            del g
+            return ms
+        except Exception as exc:  # noqa: BLE001
+            return "failed: %s" % exc
+
+    chain_ms = time_graph(dec.chain_step_fused)
+    chain2_ms = time_graph(dec.chain_step)
 
     # ---- end to end through host buffers: H2D of every input, D2H of every output
     hXh = torch.empty(dec.Xh.shape, pin_memory=True)
@@ -504,37 +565,53 @@ def run_ours(args, rank, world, local_rank):
                 "workload": "BitNet-b1.58-2B-shaped decode: 30 layers x 7 projections, N=1",
                 "layers": dec.layers, "tokens": 1,
                 "packed_bytes_per_step": dec.packed_bytes,
-                "launches_per_step": 2,
+                "launches_per_step": 1,
                 "l2": "no flush: 521 MB of packed weights per step > 126 MB L2",
                 "parallelism": "replicas" if world > 1 else "single GPU",
             },
             "pct_of_measured_hbm": round(100 * gbs / world / hbm_peak, 2),
             "roofline": {
-                "bound": "hbm", "kernel": "gemv_tile (grouped, 210 layers, K=2560 and 6912)",
-                "achieved": round(gemv_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(gemv_gbs / hbm_peak, 4),
+                "bound": "hbm",
+                "kernel": "gemv_quant (fused quantise + GEMV, grouped, 210 layers, K=2560 and 6912)",
+                "achieved": round(fused_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(fused_gbs / hbm_peak, 4),
                 "peak_note": "hbm_gbs %s (burst copy)" % peaks["source"],
-                "bytes_per_launch": dec.alg_bytes,
-                "avg_launch_ms": round(per["gemv"], 5),
+                "bytes_per_launch": dec.alg_bytes_fused,
+                "avg_launch_ms": round(per["gemv_quant"], 5),
                 "timing": "events around each launch, second pass of %d steps" % K2,
-                "traffic": ncu_traffic("gemv"),
-                "traffic_source": NCU_TRAFFIC["gemv"]["profile"],
+                "traffic": ncu_traffic("gemv_quant"),
+                "traffic_source": NCU_TRAFFIC["gemv_quant"]["profile"],
             },
             "kernel_ms": {k: round(v, 5) for k, v in per.items()},
+            "two_step": {
+                "what": "the same step as two launches: grouped quantiser, then grouped GEMV",
+                "ms_per_step": round(two_ms, 5),
+                "gbs": round(world * dec.packed_bytes / (two_ms * 1e-3) / 1e9, 1),
+                "gemv_roofline": {
+                    "achieved": round(gemv_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                    "frac": round(gemv_gbs / hbm_peak, 4), "bytes_per_launch": dec.alg_bytes,
+                    "avg_launch_ms": round(per["gemv"], 5),
+                    "traffic": ncu_traffic("gemv"),
+                    "traffic_source": NCU_TRAFFIC["gemv"]["profile"]},
+            },
             "decode_chain": {
-                "what": "same 210 linears, per-layer dependent launches (quant -> qkv, quant -> o,"
-                        " quant -> gate/up, quant -> down), one CUDA graph",
+                "what": "same 210 linears, per-layer dependent launches, one CUDA graph: fused "
+                        "(qkv, o, gate/up, down: 4 launches per layer) and two-step (a quantiser "
+                        "launch before each: 8 per layer)",
                 "ms_per_step": chain_ms if isinstance(chain_ms, str) else round(chain_ms, 4),
                 "gbs": None if isinstance(chain_ms, str) else
                 round(dec.packed_bytes / (chain_ms * 1e-3) / 1e9, 1),
-                "launches_per_step": 8 * dec.layers,
+                "launches_per_step": 4 * dec.layers,
+                "two_step_ms_per_step": chain2_ms if isinstance(chain2_ms, str)
+                else round(chain2_ms, 4),
+                "two_step_launches_per_step": 8 * dec.layers,
             },
             "prefill": prefill,
             "e2e": {"value": round(world * dec.packed_bytes / (e2e_ms * 1e-3) / 1e9, 1),
                     "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 2 * K,
-            "gpu_launches_breakdown_pass": 2 * K2,
+            "gpu_launches": K,
+            "gpu_launches_other_passes": {"two_step": 2 * K, "breakdown": 3 * K2},
             "clocks": clk,
             "cpu_baseline": cpu,
         }

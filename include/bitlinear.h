@@ -223,6 +223,53 @@ BITLINEAR_API bitlinear_status bitlinear_gemm_grouped(const bitlinear_problem* p
                                                       int64_t count, int64_t N,
                                                       bitlinear_stream_t stream);
 
+/* -------------------------------------------- decode with fused quantiser */
+
+/*
+ * Decode GEMV that takes fp32 activations and quantises them itself, in the
+ * same launch: per token amax = max|x|, q = clamp(rint(x * (127/amax)),
+ * -128, 127) exactly as bitlinear_quant_act, then the product and rescale of
+ * bitlinear_gemv.  The int8 activations never reach global memory.  This is
+ * the fused form of the I2_S path (reading notes section 2.3 and section 4.1;
+ * FairyFuse "fused kernel design": quantisation, unpacking and accumulation in
+ * one kernel with no intermediate writes).
+ *   x    fp32 [N,K] activations, 16-byte aligned, row stride K
+ *   y    fp32 [N,M] output, bit-identical to quant_act followed by gemv
+ *   acc  int32 [N,M] raw accumulators, or NULL
+ * 1 <= N <= 16, and N * 512 * ceil(K/512) <= 65536 (the int8 copy each warp
+ * keeps in shared memory): N = 1 takes K up to 65536, N = 16 up to 4096.
+ * Larger cases return BITLINEAR_ERR_UNSUPPORTED_SHAPE; quantise with
+ * bitlinear_quant_act and call bitlinear_gemv for them.
+ */
+BITLINEAR_API bitlinear_status bitlinear_gemv_quant(const uint32_t* packed, const float* alpha,
+                                                    int64_t M, int64_t K, const float* x,
+                                                    int64_t N, float* y, int32_t* acc,
+                                                    bitlinear_stream_t stream);
+
+/* One layer of a fused grouped call: the layer and its fp32 input. */
+typedef struct {
+    const uint32_t* packed;   /* [M, K/16] words */
+    const float* alpha;       /* [1] */
+    int64_t M;
+    int64_t K;
+    const float* x;           /* [N, K] fp32 */
+    float* y;                 /* [N, M] output */
+    int32_t* acc;             /* [N, M] output, or NULL */
+} bitlinear_fused_problem;
+
+/*
+ * bitlinear_gemv_quant over a list of layers, one launch per 256 layers.
+ * Each warp quantises an input once for the run of rows it owns, so layers
+ * that read the same activations (q, k and v; gate and up) should carry the
+ * same x pointer and sit next to each other in the list.  `problems` is a HOST
+ * array read during the call only.  The shared-memory limit above applies to
+ * the largest K of each launch.  All layers are checked before anything is
+ * launched.
+ */
+BITLINEAR_API bitlinear_status bitlinear_gemv_quant_grouped(
+    const bitlinear_fused_problem* problems, int64_t count, int64_t N,
+    bitlinear_stream_t stream);
+
 /* ------------------------------------------------- weights, no allocation */
 
 /*

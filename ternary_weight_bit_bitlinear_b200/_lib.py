@@ -34,6 +34,13 @@ class Act(ctypes.Structure):
                 ("xq", ctypes.c_void_p), ("amax", ctypes.c_void_p), ("xsum", ctypes.c_void_p)]
 
 
+class FusedProblem(ctypes.Structure):
+    """Mirror of bitlinear_fused_problem (include/bitlinear.h)."""
+    _fields_ = [("packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("M", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("acc", ctypes.c_void_p)]
+
+
 class BitLinearError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -79,6 +86,10 @@ def load(path: str = LIB_PATH):
         f = getattr(L, name)
         f.argtypes = [ctypes.POINTER(Problem), i64, i64, p]
         f.restype = st
+    L.bitlinear_gemv_quant.argtypes = [p, p, i64, i64, p, i64, p, p, p]
+    L.bitlinear_gemv_quant.restype = st
+    L.bitlinear_gemv_quant_grouped.argtypes = [ctypes.POINTER(FusedProblem), i64, i64, p]
+    L.bitlinear_gemv_quant_grouped.restype = st
     L.bitlinear_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
     L.bitlinear_device_error.restype = st
     _lib = L
@@ -183,6 +194,28 @@ def bitlinear_gemv_grouped(problems, count, N, stream=None):
 def bitlinear_gemm_grouped(problems, count, N, stream=None):
     """problems: a ctypes array from make_problems()."""
     return load().bitlinear_gemm_grouped(problems, count, N, _stream(stream))
+
+
+def bitlinear_gemv_quant(packed, alpha, M, K, x, N, y, acc=None, stream=None):
+    return load().bitlinear_gemv_quant(_p(packed), _p(alpha), M, K, _p(x), N, _p(y), _p(acc),
+                                       _stream(stream))
+
+
+def make_fused_problems(entries):
+    """entries: iterable of (packed, alpha, M, K, x, y, acc-or-None); tensors for
+    the pointers.  Returns a ctypes array of FusedProblem (keep it alive while
+    the call runs)."""
+    entries = list(entries)
+    arr = (FusedProblem * max(1, len(entries)))()
+    for i, (packed, alpha, M, K, x, y, acc) in enumerate(entries):
+        arr[i] = FusedProblem(packed.data_ptr(), alpha.data_ptr(), M, K, x.data_ptr(),
+                              y.data_ptr(), 0 if acc is None else acc.data_ptr())
+    return arr
+
+
+def bitlinear_gemv_quant_grouped(problems, count, N, stream=None):
+    """problems: a ctypes array from make_fused_problems()."""
+    return load().bitlinear_gemv_quant_grouped(problems, count, N, _stream(stream))
 
 
 def bitlinear_pack_workspace_bytes(M, K):

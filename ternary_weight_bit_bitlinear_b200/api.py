@@ -160,9 +160,66 @@ def matmul(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, o
     return gemm(packed, alpha, xq, amax, xsum, M, with_acc, stream, out)
 
 
+# Shared-memory bound of the fused decode kernel: tokens x K rounded up to 512.
+GEMV_QUANT_MAX_BYTES = 65536
+
+
+def gemv_quant_fits(N, K):
+    """Whether the fused quantise+GEMV kernel takes N tokens of width K."""
+    return 1 <= N <= GEMV_MAX_TOKENS and N * (-(-K // 512) * 512) <= GEMV_QUANT_MAX_BYTES
+
+
+def gemv_quant(packed, alpha, x, M=None, with_acc=False, stream=None, out=None):
+    """Decode GEMV straight from fp32 activations x[N,K] (N <= 16): the kernel
+    quantises x per token itself.  Same y (and acc) as quant_act + gemv."""
+    _need(packed, torch.int32, "packed")
+    _need(alpha, torch.float32, "alpha")
+    _need(x, torch.float32, "x")
+    M = packed.shape[0] if M is None else M
+    N, K = x.shape
+    if packed.shape != (M, K // 16):
+        raise ValueError("packed must be [M, K/16] = [%d, %d], got %s" % (M, K // 16,
+                                                                         tuple(packed.shape)))
+    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=x.device)
+    acc = torch.empty((N, M), dtype=torch.int32, device=x.device) if with_acc else None
+    _lib.check(_lib.bitlinear_gemv_quant(packed, alpha, M, K, x, N, y, acc, stream),
+               "bitlinear_gemv_quant")
+    return (y, acc) if with_acc else y
+
+
+def gemv_quant_grouped(layers, x, with_acc=False, stream=None, outs=None):
+    """Fused decode over several layers in one launch.  layers: list of
+    (packed, alpha); x: one fp32 tensor [N,K] for all layers or a list with
+    one per layer.  Layers that share an input should pass the same tensor and
+    be adjacent (each warp then quantises it once).  Returns a list of y (and
+    of acc)."""
+    n = len(layers)
+    xs = x if isinstance(x, (list, tuple)) else [x] * n
+    N = xs[0].shape[0]
+    ys, accs, entries = [], [], []
+    for i, (packed, alpha) in enumerate(layers):
+        _need(packed, torch.int32, "packed")
+        _need(alpha, torch.float32, "alpha")
+        _need(xs[i], torch.float32, "x")
+        M, K = packed.shape[0], xs[i].shape[1]
+        if xs[i].shape[0] != N or packed.shape[1] != K // 16:
+            raise ValueError("layer %d: packed [M, K/16] must match x [N, K]; N shared" % i)
+        y = outs[i] if outs is not None else torch.empty((N, M), dtype=torch.float32,
+                                                           device=packed.device)
+        acc = torch.empty((N, M), dtype=torch.int32, device=packed.device) if with_acc else None
+        ys.append(y)
+        accs.append(acc)
+        entries.append((packed, alpha, M, K, xs[i], y, acc))
+    arr = _lib.make_fused_problems(entries)
+    _lib.check(_lib.bitlinear_gemv_quant_grouped(arr, n, N, stream),
+               "bitlinear_gemv_quant_grouped")
+    return (ys, accs) if with_acc else ys
+
+
 class TernaryLinear:
     """A BitLinear layer: packed 2-bit ternary weights + alpha, applied to fp32
-    activations as quant_act -> GEMV/GEMM with the fused rescale."""
+    activations: the fused quantise+GEMV kernel for a few tokens, else
+    quant_act -> GEMV/GEMM with the fused rescale."""
 
     def __init__(self, packed, alpha, in_features, out_features):
         self.packed, self.alpha = packed, alpha
@@ -174,5 +231,7 @@ class TernaryLinear:
         return cls(packed, alpha, W.shape[1], W.shape[0])
 
     def __call__(self, x, stream=None):
+        if gemv_quant_fits(x.shape[0], x.shape[1]):
+            return gemv_quant(self.packed, self.alpha, x, self.out_features, stream=stream)
         xq, amax, xsum = quant_act(x, stream)
         return matmul(self.packed, self.alpha, xq, amax, xsum, self.out_features, stream=stream)

@@ -13,6 +13,7 @@
 #include "bitlinear.h"
 #include "gemm.cuh"
 #include "gemv.cuh"
+#include "gemv_quant.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
 
@@ -58,6 +59,9 @@ struct DeviceInfo {
   int sms = 0;
   bool gemm_attr_set[2] = {false, false};
   int gemv_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};   // 0: not set up yet
+  bool gq_attr_set[bl::kGemvMaxTokens + 1] = {};
+  int gq_smem[bl::kGemvMaxTokens + 1] = {};               // last shared-memory size seen
+  int gq_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};      // and its occupancy
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -329,6 +333,184 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
   return BITLINEAR_OK;
 }
 
+// ---- decode GEMV with the quantiser fused in
+
+bitlinear_status check_fused_problem(const bitlinear_fused_problem& q, int64_t N) {
+  bitlinear_status st = check_mk(q.M, q.K);
+  if (st != BITLINEAR_OK) return st;
+  if (!q.packed || !q.alpha || !q.x || !q.y) return BITLINEAR_ERR_INVALID_ARG;
+  if (!aligned16(q.packed) || !aligned16(q.x) || !aligned16(q.y) || (q.acc && !aligned16(q.acc)))
+    return BITLINEAR_ERR_MISALIGNED;
+  if (!aligned4(q.alpha)) return BITLINEAR_ERR_MISALIGNED;
+  const int64_t kpad = (q.K + bl::kGemvChunkK - 1) / bl::kGemvChunkK * bl::kGemvChunkK;
+  if (N * kpad > bl::kGqMaxXBytes) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  return BITLINEAR_OK;
+}
+
+// Largest shared-memory area for which a token row is staged in place (one
+// copy round trip): above it the row goes through the ring's space in
+// pieces, which keeps the area, and so the warps per SM, unchanged.
+constexpr int kGqInPlaceMaxArea = 28 * 1024;
+
+template <int NT>
+bitlinear_status gemv_quant_blocks_per_sm(int area, DeviceInfo* dev, int* out) {
+  auto kernel = bl::gemv_quant_kernel<NT>;
+  if (!dev->gq_attr_set[NT]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bl::kGqMaxXBytes + bl::kGqRingBytes) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    dev->gq_attr_set[NT] = true;
+  }
+  if (dev->gq_smem[NT] != area) {
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, 32, area) != cudaSuccess ||
+        nb < 1)
+      return BITLINEAR_ERR_CUDA;
+    dev->gq_smem[NT] = area;
+    dev->gq_blocks_per_sm[NT] = nb;
+  }
+  *out = dev->gq_blocks_per_sm[NT];
+  return BITLINEAR_OK;
+}
+
+bitlinear_status gemv_quant_occupancy(int N, int area, DeviceInfo* dev, int* out) {
+  switch (N) {
+#define BL_GQ_CASE(n) \
+  case n: return gemv_quant_blocks_per_sm<n>(area, dev, out);
+    BL_GQ_CASE(1) BL_GQ_CASE(2) BL_GQ_CASE(3) BL_GQ_CASE(4)
+    BL_GQ_CASE(5) BL_GQ_CASE(6) BL_GQ_CASE(7) BL_GQ_CASE(8)
+    BL_GQ_CASE(9) BL_GQ_CASE(10) BL_GQ_CASE(11) BL_GQ_CASE(12)
+    BL_GQ_CASE(13) BL_GQ_CASE(14) BL_GQ_CASE(15) BL_GQ_CASE(16)
+#undef BL_GQ_CASE
+    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
+bitlinear_status gemv_quant_launch(int N, int grid, const bl::GqParams& p, cudaStream_t s) {
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (N) {
+#define BL_GQ_CASE(n) \
+  case n: e = launch_pdl(bl::gemv_quant_kernel<n>, grid, 32, static_cast<size_t>(p.area), s, p); \
+    break;
+    BL_GQ_CASE(1) BL_GQ_CASE(2) BL_GQ_CASE(3) BL_GQ_CASE(4)
+    BL_GQ_CASE(5) BL_GQ_CASE(6) BL_GQ_CASE(7) BL_GQ_CASE(8)
+    BL_GQ_CASE(9) BL_GQ_CASE(10) BL_GQ_CASE(11) BL_GQ_CASE(12)
+    BL_GQ_CASE(13) BL_GQ_CASE(14) BL_GQ_CASE(15) BL_GQ_CASE(16)
+#undef BL_GQ_CASE
+    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
+  return launch_status();
+}
+
+// Warps per segment: one each, then the rest one at a time to the segment
+// whose warps have the most work (never more warps than units).  A warp's
+// work is its share of k-chunks plus one unit's worth for quantising the
+// input first, whose copy time grows with K like a unit's.  This minimises
+// the largest per-warp estimate.
+void gemv_quant_assign(bl::GqParams& p, int warps_total) {
+  const int n = p.num_segments;
+  std::vector<int> w(n, 1);
+  int used = n;
+  auto load = [&](int g) {
+    return (static_cast<double>(p.seg[g].units) / w[g] + 1.0) * p.seg[g].chunks;
+  };
+  auto cmp = [&](int a, int b) { return load(a) < load(b); };
+  std::vector<int> heap;
+  for (int g = 0; g < n; ++g)
+    if (p.seg[g].units > 1) heap.push_back(g);
+  std::make_heap(heap.begin(), heap.end(), cmp);
+  while (used < warps_total && !heap.empty()) {
+    std::pop_heap(heap.begin(), heap.end(), cmp);
+    const int g = heap.back();
+    heap.pop_back();
+    ++w[g];
+    ++used;
+    if (w[g] < p.seg[g].units) {
+      heap.push_back(g);
+      std::push_heap(heap.begin(), heap.end(), cmp);
+    }
+  }
+  int begin = 0;
+  for (int g = 0; g < n; ++g) {
+    p.seg[g].warp_begin = begin;
+    p.seg[g].warps = w[g];
+    begin += w[g];
+  }
+}
+
+// Fused decode over validated problems sharing N: one launch per at most
+// kGqMaxProblems problems and at most as many input segments as the grid has
+// warps; every warp owns one segment's share of units.
+bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t count,
+                                  int64_t N, cudaStream_t s) {
+  DeviceInfo* dev = nullptr;
+  bitlinear_status st = device_info(&dev);
+  if (st != BITLINEAR_OK) return st;
+  const int nt = static_cast<int>(N);
+  int64_t base = 0;
+  while (base < count) {
+    // Shared-memory area from the largest K of this launch's first problems.
+    // Start from as many problems as the table holds; shrink to the number of
+    // segments the grid can give one warp each.
+    int n = static_cast<int>(std::min<int64_t>(count - base, bl::kGqMaxProblems));
+    bl::GqParams p;
+    int grid = 0;
+    for (;;) {
+      memset(&p, 0, sizeof p);
+      int64_t units = 0, kmax = 0;
+      int segs = 0;
+      for (int i = 0; i < n; ++i) {
+        const bitlinear_fused_problem& q = probs[base + i];
+        bl::GqProblem& g = p.prob[i];
+        g.packed = q.packed;
+        g.alpha = q.alpha;
+        g.y = q.y;
+        g.acc = q.acc;
+        g.M = static_cast<int>(q.M);
+        g.W = static_cast<int>(q.K / 16);
+        g.unit_begin = static_cast<int>(units);
+        const int64_t u = (q.M + bl::kGemvTileRows - 1) / bl::kGemvTileRows;
+        const bool same = segs > 0 && p.seg[segs - 1].x == q.x && p.seg[segs - 1].K == q.K;
+        if (!same) {
+          bl::GqSegment& sg = p.seg[segs++];
+          sg.x = q.x;
+          sg.K = static_cast<int>(q.K);
+          sg.chunks = static_cast<int>((q.K + bl::kGemvChunkK - 1) / bl::kGemvChunkK);
+          sg.unit_begin = static_cast<int>(units);
+          sg.prob_begin = i;
+        }
+        p.seg[segs - 1].units += static_cast<int>(u);
+        units += u;
+        kmax = std::max<int64_t>(kmax, q.K);
+        if (units > INT_MAX / 2) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+      }
+      p.num_problems = n;
+      p.num_segments = segs;
+      const int64_t chunks = (kmax + bl::kGemvChunkK - 1) / bl::kGemvChunkK;
+      p.xstride = static_cast<int>(chunks * bl::kGemvChunkK);
+      const int plain = nt * p.xstride + bl::kGqRingBytes;
+      const int in_place = (nt - 1) * p.xstride + 4 * static_cast<int>(kmax);
+      p.area = in_place > plain && in_place <= kGqInPlaceMaxArea ? in_place : plain;
+      int per_sm = 0;
+      st = gemv_quant_occupancy(nt, p.area, dev, &per_sm);
+      if (st != BITLINEAR_OK) return st;
+      const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm;
+      if (segs <= cap) {
+        grid = static_cast<int>(std::min<int64_t>(cap, units));
+        break;
+      }
+      n = std::max(1, n / 2);   // more inputs than warps: fewer problems per launch
+    }
+    gemv_quant_assign(p, grid);
+    grid = p.seg[p.num_segments - 1].warp_begin + p.seg[p.num_segments - 1].warps;
+    st = gemv_quant_launch(nt, grid, p, s);
+    if (st != BITLINEAR_OK) return st;
+    base += n;
+  }
+  return BITLINEAR_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -517,6 +699,31 @@ bitlinear_status bitlinear_gemm_grouped(const bitlinear_problem* problems, int64
     if (problems[i].M % 128 != 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   }
   return gemm_group(problems, count, N, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitlinear_status bitlinear_gemv_quant(const uint32_t* packed, const float* alpha, int64_t M,
+                                      int64_t K, const float* x, int64_t N, float* y,
+                                      int32_t* acc, bitlinear_stream_t stream) {
+  if (N < 0) return BITLINEAR_ERR_INVALID_ARG;
+  if (N > bl::kGemvMaxTokens) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  const bitlinear_fused_problem q = {packed, alpha, M, K, x, y, acc};
+  if (N == 0) return check_mk(M, K);
+  bitlinear_status st = check_fused_problem(q, N);
+  if (st != BITLINEAR_OK) return st;
+  return gemv_quant_group(&q, 1, N, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitlinear_status bitlinear_gemv_quant_grouped(const bitlinear_fused_problem* problems,
+                                              int64_t count, int64_t N,
+                                              bitlinear_stream_t stream) {
+  if (count < 0 || N < 0 || (count > 0 && !problems)) return BITLINEAR_ERR_INVALID_ARG;
+  if (count == 0 || N == 0) return BITLINEAR_OK;
+  if (N > bl::kGemvMaxTokens) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  for (int64_t i = 0; i < count; ++i) {
+    bitlinear_status st = check_fused_problem(problems[i], N);
+    if (st != BITLINEAR_OK) return st;
+  }
+  return gemv_quant_group(problems, count, N, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bitlinear_status bitlinear_device_error(int* status_out, int clear) {

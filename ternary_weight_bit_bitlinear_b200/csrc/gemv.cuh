@@ -84,7 +84,8 @@ struct GemvCopyPlan {
   int wword;               // word index of this lane's chunk within a k-chunk
 };
 
-__device__ __forceinline__ GemvCopyPlan gemv_plan(const GemvProblem& pr, int row0, int lane) {
+template <class Problem>   // any problem type with packed, M and W
+__device__ __forceinline__ GemvCopyPlan gemv_plan(const Problem& pr, int row0, int lane) {
   GemvCopyPlan cp;
   const int rr = lane >> 3, c = lane & 7;
   cp.wsrc = reinterpret_cast<const uint8_t*>(pr.packed) +
@@ -97,13 +98,13 @@ __device__ __forceinline__ GemvCopyPlan gemv_plan(const GemvProblem& pr, int row
   return cp;
 }
 
-// Issue the copies of k-chunk `kc` into stage buffer `st`.  Weight chunks
-// outside the layer are skipped (rows past M are never stored; past the last
-// word, the activations are zero, so stale bytes multiply zeros).
-template <int NT>
-__device__ __forceinline__ void gemv_issue(const GemvProblem& pr, const GemvCopyPlan& cp, int kc,
-                                           uint8_t* st, int lane) {
-  if (kc * (kGemvChunkBytes / 4) + cp.wword < pr.W) {
+// Issue the weight copies of k-chunk `kc` (W words per row) into stage buffer
+// `st`.  Weight chunks outside the layer are skipped (rows past M are never
+// stored; past the last word, the activations are zero, so stale bytes
+// multiply zeros).
+__device__ __forceinline__ void gemv_issue_weights(int W, const GemvCopyPlan& cp, int kc,
+                                                   uint8_t* st) {
+  if (kc * (kGemvChunkBytes / 4) + cp.wword < W) {
     const uint8_t* src = cp.wsrc + kc * kGemvChunkBytes;
 #pragma unroll
     for (int i = 0; i < kGemvTileRows / 4; ++i) {
@@ -112,6 +113,13 @@ __device__ __forceinline__ void gemv_issue(const GemvProblem& pr, const GemvCopy
       src += cp.wstep;
     }
   }
+}
+
+// Weights and int8 activations of k-chunk `kc` into stage buffer `st`.
+template <int NT>
+__device__ __forceinline__ void gemv_issue(const GemvProblem& pr, const GemvCopyPlan& cp, int kc,
+                                           uint8_t* st, int lane) {
+  gemv_issue_weights(pr.W, cp, kc, st);
   // activations: 512 bytes per token, 16 per lane, zero-filled past K
   const int k0 = kc * kGemvChunkK + lane * 16;
   const bool xval = k0 < pr.K;
@@ -120,6 +128,31 @@ __device__ __forceinline__ void gemv_issue(const GemvProblem& pr, const GemvCopy
     const int8_t* src = xval ? pr.xq + static_cast<int64_t>(t) * pr.K + k0 : pr.xq;
     cp_async16(st + GemvCfg<NT>::kWeightBytes + t * kGemvChunkK + lane * 16, src,
                xval ? 16u : 0u);
+  }
+}
+
+// One k-chunk of this lane's row against every token: `wrow` is the row's
+// 128 swizzled bytes in a stage, `xs` the chunk's 512 int8 activations of
+// token 0 (token t at xs + t * xstride), read as broadcasts.
+template <int NT>
+__device__ __forceinline__ void gemv_chunk_dot(const uint8_t* wrow, uint32_t sw, const uint8_t* xs,
+                                               int xstride, int (&acc)[NT][4]) {
+#pragma unroll
+  for (int c = 0; c < kGemvChunkBytes / 16; ++c) {
+    const uint4 w = *reinterpret_cast<const uint4*>(wrow + ((static_cast<uint32_t>(c) ^ sw) << 4));
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const uint4* xp = reinterpret_cast<const uint4*>(xs + t * xstride + c * 64);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 xa = xp[i];
+        acc[t][0] = dp4a_us(ws[i] & 0x03030303u, xa.x, acc[t][0]);
+        acc[t][1] = dp4a_us(ws[i] & 0x0C0C0C0Cu, xa.y, acc[t][1]);
+        acc[t][2] = dp4a_us(ws[i] & 0x30303030u, xa.z, acc[t][2]);
+        acc[t][3] = dp4a_us(ws[i] & 0xC0C0C0C0u, xa.w, acc[t][3]);
+      }
+    }
   }
 }
 
@@ -187,25 +220,7 @@ gemv_tile_kernel(const __grid_constant__ GemvParams p) {
       __syncwarp();
       const uint8_t* st = ring + cslot * C::kStageBytes;
       cslot = (cslot + 1) & (C::kStages - 1);
-      const uint8_t* wrow = st + lane * kGemvChunkBytes;
-      const uint8_t* xs = st + C::kWeightBytes;
-#pragma unroll
-      for (int c = 0; c < kGemvChunkBytes / 16; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4*>(wrow + ((static_cast<uint32_t>(c) ^ sw) << 4));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const uint4* xp = reinterpret_cast<const uint4*>(xs + t * kGemvChunkK + c * 64);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 xa = xp[i];
-            acc[t][0] = dp4a_us(ws[i] & 0x03030303u, xa.x, acc[t][0]);
-            acc[t][1] = dp4a_us(ws[i] & 0x0C0C0C0Cu, xa.y, acc[t][1]);
-            acc[t][2] = dp4a_us(ws[i] & 0x30303030u, xa.z, acc[t][2]);
-            acc[t][3] = dp4a_us(ws[i] & 0xC0C0C0C0u, xa.w, acc[t][3]);
-          }
-        }
-      }
+      gemv_chunk_dot<NT>(st + lane * kGemvChunkBytes, sw, st + C::kWeightBytes, kGemvChunkK, acc);
       __syncwarp();   // every lane is done with this stage before it is refilled
     }
 

@@ -1,0 +1,279 @@
+// gemv_quant.cuh -- decode GEMV with the per-token activation quantiser fused
+// into its prologue: fp32 activations in, fp32 outputs out, no int8 round trip
+// through global memory and no second launch.
+//
+// The fusion follows the FairyFuse "fused kernel design" (activation handling,
+// unpacking and accumulation in one kernel, no intermediate writes) and keeps
+// the I2_S arithmetic of the "Bitnet.cpp" reading notes (section 2.3, section
+// 4.1): per-token absmax int8 activations, ternary weights, int32 sums, one
+// fp32 rescale.  The quantised values are the ones quant.cuh produces:
+//   amax = max_k |x[k]|,  s = 127 / amax,  q = clamp(rint(x * s), -128, 127).
+//
+// Work split: one warp per CTA.  A launch's problems form segments: runs of
+// consecutive problems that read the same input (pointer and K; q, k and v,
+// or gate and up, when given side by side).  The host gives every segment a
+// number of warps in proportion to its k-chunk count (at least one, at most
+// its unit count), and each warp takes an equal share of its segment's units
+// (32 rows x all of K, as in gemv.cuh).  A warp therefore quantises exactly
+// one input, once, before it streams any weights:
+//   1. the first weight stages are prefetched into L2 (their addresses do not
+//      depend on the input), and when the staging below leaves the ring's
+//      space alone, the ring's first stages are already copied in;
+//   2. each token's fp32 row is copied into the warp's shared memory with
+//      16-byte cp.async copies, all in flight at once;
+//   3. amax is reduced from shared memory and the row is quantised, four int8
+//      per 32-bit word;
+//   4. the weight ring of gemv.cuh (weights only, 4 stages of 4 KB) streams
+//      the warp's units, with activations read as broadcasts from the int8
+//      copy.
+// Shared memory of a CTA: the int8 copy [NT][xstride] at the start, the ring
+// at the end.  When a token's fp32 row fits between its own int8 row and the
+// end of the area it is staged there and quantised in place; otherwise it
+// passes through the ring's space in pieces, once for the maximum and once to
+// quantise.
+#pragma once
+
+#include "gemv.cuh"
+#include "quant.cuh"
+
+namespace bl {
+
+constexpr int kGqStages = 4;                                          // power of two
+constexpr int kGqStageBytes = kGemvTileRows * kGemvChunkBytes;        // 4 KB of weights
+constexpr int kGqRingBytes = kGqStages * kGqStageBytes;
+constexpr int kGqMaxProblems = 256;
+constexpr int kGqMaxXBytes = 65536;   // tokens x K (rounded up to 512) held per warp
+
+struct GqProblem {
+  const uint32_t* packed;
+  const float* alpha;
+  float* y;                // fp32 [NT][M]
+  int32_t* acc;            // int32 [NT][M] or null
+  int M, W;                // W = K / 16 words per row
+  int unit_begin;          // first unit of this problem
+};
+
+// A run of problems that read one input.  Its units all have the same K.
+struct GqSegment {
+  const float* x;          // fp32 [NT][K]
+  int K;
+  int chunks;              // k-chunks per unit: ceil(K / 512)
+  int unit_begin, units;   // the segment's units, numbered across the launch
+  int warp_begin, warps;   // the warps (CTAs) that share them
+  int prob_begin;          // first problem of the segment
+};
+
+struct GqParams {
+  GqProblem prob[kGqMaxProblems];
+  GqSegment seg[kGqMaxProblems];
+  int num_problems;
+  int num_segments;
+  int xstride;             // bytes per token of the int8 copy: 512 x the launch's largest chunks
+  int area;                // dynamic shared memory bytes: >= NT * xstride + kGqRingBytes;
+                           // the ring takes the last kGqRingBytes
+};
+
+// Quantise x [NT][K] (fp32, 16-byte aligned rows) into xs [NT][xstride] int8,
+// zero from K up to kpad; amax and the sum of q of token t go to s_amax[t] and
+// s_xsum[t].  Run by the whole warp.
+//
+// In place: token t's row is staged at xs + t * xstride; in round r each lane
+// reads float4 32r + lane and then writes the word of the same index, i.e.
+// bytes below 128r + 128, which only reach float4s that an earlier round (or
+// this round, before the __syncwarp) has read.
+// In pieces: the window [win, win + win_bytes) takes up to win_bytes / 4
+// floats at a time, once for the maximum, once for the quantisation.
+template <int NT>
+__device__ __forceinline__ void gq_quantise(const float* __restrict__ x, int K, int kpad,
+                                            int xstride, uint8_t* xs, uint8_t* win,
+                                            int win_bytes, int area, float* s_amax,
+                                            int* s_xsum, int lane) {
+  const int K4 = K / 4;
+#pragma unroll 1
+  for (int t = 0; t < NT; ++t) {
+    uint8_t* row8 = xs + t * xstride;
+    uint32_t* out = reinterpret_cast<uint32_t*>(row8);
+    const float* row = x + static_cast<int64_t>(t) * K;
+    float m = 0.0f;
+    int sum = 0;
+    if (t * xstride + 4 * K <= area) {
+      for (int i = lane; i < K4; i += 32) cp_async16(row8 + 16 * i, row + 4 * i, 16u);
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncwarp();
+      const float4* v4 = reinterpret_cast<const float4*>(row8);
+      for (int i = lane; i < K4; i += 32) m = fmaxf(m, absmax4(v4[i]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      const float s = m == 0.0f ? 0.0f : __fdiv_rn(127.0f, m);
+      for (int base = 0; base < K4; base += 32) {   // uniform trip count: __syncwarp inside
+        const int i = base + lane;
+        const float4 v = i < K4 ? v4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();
+        if (i < K4) out[i] = m == 0.0f ? 0u : quant_pack4(v, s, sum);
+      }
+      __syncwarp();
+    } else {
+      const int P4 = win_bytes / 16;   // float4s per piece
+      const float4* w4 = reinterpret_cast<const float4*>(win);
+#pragma unroll 1
+      for (int b = 0; b < K4; b += P4) {
+        const int n = min(P4, K4 - b);
+        for (int i = lane; i < n; i += 32) cp_async16(win + 16 * i, row + 4 * (b + i), 16u);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) m = fmaxf(m, absmax4(w4[i]));
+        __syncwarp();   // the window is read before the next piece lands
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      const float s = m == 0.0f ? 0.0f : __fdiv_rn(127.0f, m);
+#pragma unroll 1
+      for (int b = 0; b < K4; b += P4) {
+        const int n = min(P4, K4 - b);
+        if (m != 0.0f) {
+          for (int i = lane; i < n; i += 32) cp_async16(win + 16 * i, row + 4 * (b + i), 16u);
+          cp_async_commit();
+          cp_async_wait<0>();
+          __syncwarp();
+        }
+        for (int i = lane; i < n; i += 32) out[b + i] = m == 0.0f ? 0u : quant_pack4(w4[i], s, sum);
+        __syncwarp();
+      }
+    }
+    for (int i = K4 + lane; i < kpad / 4; i += 32) out[i] = 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if (lane == 0) {
+      s_amax[t] = m;
+      s_xsum[t] = sum;
+    }
+    __syncwarp();
+  }
+}
+
+// Segment that warp b belongs to (the last one whose warp_begin <= b).
+__device__ __forceinline__ int gq_segment_of(const GqParams& p, int b) {
+  int lo = 0, hi = p.num_segments - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.seg[mid].warp_begin <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(32)
+gemv_quant_kernel(const __grid_constant__ GqParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float s_amax[NT];
+  __shared__ int s_xsum[NT];
+  const int lane = threadIdx.x;
+  const uint32_t sw = static_cast<uint32_t>(lane & 7);
+  uint8_t* xs = smem;
+  uint8_t* ring = smem + p.area - kGqRingBytes;
+
+  // This warp's units: an equal share of its segment's.
+  const GqSegment sg = p.seg[gq_segment_of(p, blockIdx.x)];
+  const int wi = blockIdx.x - sg.warp_begin;
+  const int u_begin =
+      sg.unit_begin + static_cast<int>(static_cast<int64_t>(sg.units) * wi / sg.warps);
+  const int u_end =
+      sg.unit_begin + static_cast<int>(static_cast<int64_t>(sg.units) * (wi + 1) / sg.warps);
+  int pi = sg.prob_begin;
+  while (pi + 1 < p.num_problems && p.prob[pi + 1].unit_begin <= u_begin) ++pi;
+
+  // Copy plan of the first unit.  Its first stages are prefetched into L2
+  // before the wait on the preceding kernel: that kernel may write the input,
+  // and a prefetch is only a cache hint, so nothing is read too early.
+  GqProblem ipr = p.prob[pi];
+  GemvCopyPlan icp = gemv_plan(ipr, (u_begin - ipr.unit_begin) * kGemvTileRows, lane);
+  if (u_begin < u_end) {
+#pragma unroll 1
+    for (int kc = 0; kc < kGqStages - 1 && kc < sg.chunks; ++kc) {
+      if (kc * (kGemvChunkBytes / 4) + icp.wword < ipr.W) {
+        const uint8_t* src = icp.wsrc + kc * kGemvChunkBytes;
+#pragma unroll 1
+        for (int i = 0; i < icp.vrows; ++i)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(src + i * icp.wstep) : "memory");
+      }
+    }
+  }
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+  if (u_begin >= u_end) return;
+
+  // Copy side: weights of (unit, k-chunk) pairs, running ahead across units.
+  int iu = u_begin, ic = 0, ipi = pi;
+  int slot = 0;
+  auto issue_next = [&]() {
+    if (iu < u_end) {
+      gemv_issue_weights(ipr.W, icp, ic, ring + slot * kGqStageBytes);
+      if (++ic == sg.chunks) {
+        ic = 0;
+        if (++iu < u_end) {
+          while (ipi + 1 < p.num_problems && p.prob[ipi + 1].unit_begin <= iu) ++ipi;
+          ipr = p.prob[ipi];
+          icp = gemv_plan(ipr, (iu - ipr.unit_begin) * kGemvTileRows, lane);
+        }
+      }
+    }
+    cp_async_commit();   // one group per stage, empty once the run is done
+    slot = (slot + 1) & (kGqStages - 1);
+  };
+  // The ring's first stages go in before the quantisation when every token's
+  // staged row ends below the ring (the wait for the staging copies then
+  // covers them too, one round trip for both).
+  const bool early_ring = (NT - 1) * p.xstride + 4 * sg.K <= p.area - kGqRingBytes;
+  if (early_ring) {
+#pragma unroll 1
+    for (int s = 0; s < kGqStages - 1; ++s) issue_next();
+  }
+  gq_quantise<NT>(sg.x, sg.K, sg.chunks * kGemvChunkK, p.xstride, xs, smem + NT * p.xstride,
+                  p.area - NT * p.xstride, p.area, s_amax, s_xsum, lane);
+  if (!early_ring) {
+#pragma unroll 1
+    for (int s = 0; s < kGqStages - 1; ++s) issue_next();
+  }
+
+  int cslot = 0;
+  for (int cu = u_begin; cu < u_end; ++cu) {
+    while (pi + 1 < p.num_problems && p.prob[pi + 1].unit_begin <= cu) ++pi;
+    const GqProblem pr = p.prob[pi];   // by value: registers, not parameter-space reloads
+    const int row0 = (cu - pr.unit_begin) * kGemvTileRows;
+
+    int acc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[t][j] = 0;
+
+    for (int kc = 0; kc < sg.chunks; ++kc) {
+      issue_next();
+      cp_async_wait<kGqStages - 1>();
+      __syncwarp();
+      const uint8_t* st = ring + cslot * kGqStageBytes;
+      cslot = (cslot + 1) & (kGqStages - 1);
+      gemv_chunk_dot<NT>(st + lane * kGemvChunkBytes, sw, xs + kc * kGemvChunkK, p.xstride, acc);
+      __syncwarp();   // every lane is done with this stage before it is refilled
+    }
+
+    const int row = row0 + lane;
+    if (row < pr.M) {
+      const float alpha = *pr.alpha;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const int a = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) -
+                      s_xsum[t];
+        const float scale = __fmul_rn(alpha, __fdiv_rn(s_amax[t], 127.0f));
+        const int64_t o = static_cast<int64_t>(t) * pr.M + row;
+        pr.y[o] = __fmul_rn(__int2float_rn(a), scale);
+        if (pr.acc) pr.acc[o] = a;
+      }
+    }
+  }
+  cp_async_wait<0>();
+}
+
+}  // namespace bl

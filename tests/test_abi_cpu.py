@@ -183,3 +183,55 @@ def test_quant_act_per_tensor_argument_errors(L):
     assert f(p(FAKE), 2, 128, p(FAKE), p(FAKE), None, p(MISALIGNED), ws, None) == \
         _lib.ERR_MISALIGNED
     assert f(p(FAKE), 0, 128, p(FAKE), p(FAKE), None, p(FAKE), ws, None) == _lib.OK
+
+
+def test_gemv_quant_argument_errors(L):
+    f = L.bitlinear_gemv_quant
+    ok = dict(packed=FAKE, alpha=FAKE, M=128, K=256, x=FAKE, N=1, y=FAKE, acc=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(_p(a["packed"]), _p(a["alpha"]), a["M"], a["K"], _p(a["x"]), a["N"],
+                 _p(a["y"]), _p(a["acc"]), None)
+
+    assert call(N=0) == _lib.OK
+    assert call(N=0, K=200) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(N=-1) == _lib.ERR_INVALID_ARG
+    assert call(N=17) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(packed=0) == _lib.ERR_INVALID_ARG
+    assert call(x=0) == _lib.ERR_INVALID_ARG
+    assert call(y=0) == _lib.ERR_INVALID_ARG
+    assert call(K=200) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(M=0) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(x=MISALIGNED) == _lib.ERR_MISALIGNED
+    assert call(y=MISALIGNED) == _lib.ERR_MISALIGNED
+    assert call(acc=MISALIGNED) == _lib.ERR_MISALIGNED
+    assert call(alpha=FAKE + 2) == _lib.ERR_MISALIGNED
+    # the int8 copy of x each warp keeps: N * K rounded up to 512 <= 65536 bytes
+    assert call(N=1, K=65536 + 128) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(N=16, K=4096 + 128) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(N=2, K=32768 + 128) == _lib.ERR_UNSUPPORTED_SHAPE
+
+
+def test_gemv_quant_grouped_argument_errors(L):
+    f = L.bitlinear_gemv_quant_grouped
+    P = _lib.FusedProblem
+
+    def prob(**kw):
+        a = dict(packed=FAKE, alpha=FAKE, M=128, K=256, x=FAKE, y=FAKE, acc=0)
+        a.update(kw)
+        return P(a["packed"], a["alpha"], a["M"], a["K"], a["x"], a["y"], a["acc"])
+
+    good = prob()
+    arr = (P * 2)(good, good)
+    assert f(arr, -1, 1, None) == _lib.ERR_INVALID_ARG
+    assert f(None, 2, 1, None) == _lib.ERR_INVALID_ARG
+    assert f(arr, 0, 1, None) == _lib.OK
+    assert f(arr, 2, 0, None) == _lib.OK
+    assert f(arr, 2, -3, None) == _lib.ERR_INVALID_ARG
+    assert f(arr, 2, 17, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert f((P * 2)(good, prob(K=200)), 2, 1, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert f((P * 2)(good, prob(K=40960)), 2, 2, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert f((P * 2)(good, prob(x=MISALIGNED)), 2, 1, None) == _lib.ERR_MISALIGNED
+    assert f((P * 2)(good, prob(x=0)), 2, 1, None) == _lib.ERR_INVALID_ARG
+    assert f((P * 2)(good, prob(alpha=FAKE + 2)), 2, 1, None) == _lib.ERR_MISALIGNED

@@ -65,6 +65,13 @@ class Model:
                               [q[2] for q in qs])
         return dict(zip(lst, ys))
 
+    def run_gemv_quant(self):
+        """The same stream through the fused quantise+GEMV kernel (fp32 inputs)."""
+        lst = self.layer_list()
+        ys = api.gemv_quant_grouped([self.w[k] for k in lst],
+                                    [self.x[(l, _input_proj(p))] for l, p in lst])
+        return dict(zip(lst, ys))
+
     def run_gemm(self, layer):
         lst = [(layer, p) for p in range(7)]
         qs = [self.q[(l, _input_proj(p))] for l, p in lst]
@@ -122,6 +129,18 @@ def test_config2_2b_decode_stream_30_layers():
         m.check(l, p, ys[(l, p)], _rows(M, 40, 10 * l + p), [0])
 
 
+def test_config2_2b_decode_stream_fused_quant():
+    m = Model(2, 30, 1)
+    ys = m.run_gemv_quant()
+    for (l, p) in [(0, 0), (3, 2), (11, 5), (29, 6), (29, 3)]:
+        M = m.shape.projections()[p][1]
+        m.check(l, p, ys[(l, p)], _rows(M, 40, 10 * l + p + 1), [0])
+    # and the whole stream equals the two-step path bit for bit
+    ref = m.run_gemv()
+    for k in ys:
+        assert torch.equal(ys[k], ref[k]), k
+
+
 def test_config3_7b_prefill_512_grouped():
     m = Model(3, 1, 512)
     ys = m.run_gemm(0)
@@ -152,7 +171,14 @@ def test_config5_70b_weight_stream_and_prefill():
     for (l, p) in [(0, 0), (40, 1), (79, 5), (79, 6)]:
         M = m.shape.projections()[p][1]
         m.check(l, p, ys[(l, p)], _rows(M, 16, l + p), [0])
-    del ys
+    # the fused quantise+GEMV kernel on the same 80-layer stream (K up to 28672)
+    yf = m.run_gemv_quant()
+    for (l, p) in [(1, 0), (79, 6)]:
+        M = m.shape.projections()[p][1]
+        m.check(l, p, yf[(l, p)], _rows(M, 16, l + p + 3), [0])
+    for k in ys:
+        assert torch.equal(yf[k], ys[k]), k
+    del ys, yf
     # prefill N = 2048 on one layer of the same weights
     N = 2048
     x = {p: inputs.activations(N, m.shape.ffn if p == 6 else m.shape.hidden,
