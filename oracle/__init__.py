@@ -33,6 +33,8 @@ def lib():
         L.oracle_absmean.restype = ctypes.c_float
         L.oracle_ternarize.argtypes = [p, i64, ctypes.c_float, p]
         L.oracle_ternarize.restype = None
+        L.oracle_packed_row_words.argtypes = [i64]
+        L.oracle_packed_row_words.restype = i64
         L.oracle_pack.argtypes = [p, i64, i64, p]
         L.oracle_pack.restype = ctypes.c_int
         L.oracle_unpack.argtypes = [p, i64, i64, p]
@@ -86,11 +88,16 @@ def ternarize(w, alpha):
     return codes
 
 
+def packed_row_words(K):
+    """Words per packed row: 4*ceil(K/64) (K/16 when K is a multiple of 64)."""
+    return int(lib().oracle_packed_row_words(int(K)))
+
+
 def pack(codes):
-    """codes int8 [M,K] -> uint32 [M, K/16]."""
+    """codes int8 [M,K] -> uint32 [M, packed_row_words(K)]."""
     codes, pc = _c(codes, np.int8)
     M, K = codes.shape
-    out = np.empty((M, K // 16), dtype=np.uint32)
+    out = np.empty((M, packed_row_words(K)), dtype=np.uint32)
     if lib().oracle_pack(pc, M, K, out.ctypes.data) != 0:
         raise ValueError("bad code or K % 16 != 0")
     return out

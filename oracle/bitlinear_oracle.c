@@ -174,17 +174,24 @@ static int field_bit(int64_t k)
     return (int)(8 * (k % 4) + 2 * ((k % 16) / 4));
 }
 
+int64_t oracle_packed_row_words(int64_t K)
+{
+    return 4 * ((K + 63) / 64);
+}
+
 int oracle_pack(const int8_t* codes, int64_t M, int64_t K, uint32_t* packed)
 {
     if (K % 16 != 0 || M < 0) return -1;
-    int64_t wpr = K / 16;
-    for (int64_t i = 0; i < M * wpr; ++i) packed[i] = 0;
+    int64_t wpr = oracle_packed_row_words(K);
+    /* every field starts as 01 (code 0), so the padding past K stays code 0 */
+    for (int64_t i = 0; i < M * wpr; ++i) packed[i] = 0x55555555u;
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t k = 0; k < K; ++k) {
             int c = codes[m * K + k];
             if (c < -1 || c > 1) return -1;
             uint32_t field = (uint32_t)(c + 1);
-            packed[m * wpr + k / 16] |= field << field_bit(k);
+            uint32_t* w = &packed[m * wpr + k / 16];
+            *w = (*w & ~(3u << field_bit(k))) | (field << field_bit(k));
         }
     }
     return 0;
@@ -193,13 +200,16 @@ int oracle_pack(const int8_t* codes, int64_t M, int64_t K, uint32_t* packed)
 int oracle_unpack(const uint32_t* packed, int64_t M, int64_t K, int8_t* codes)
 {
     if (K % 16 != 0 || M < 0) return -1;
-    int64_t wpr = K / 16;
+    int64_t wpr = oracle_packed_row_words(K);
     int bad = 0;
     for (int64_t m = 0; m < M; ++m) {
-        for (int64_t k = 0; k < K; ++k) {
+        for (int64_t k = 0; k < 16 * wpr; ++k) {
             uint32_t field = (packed[m * wpr + k / 16] >> field_bit(k)) & 3u;
             if (field == 3u) bad = 1;
-            codes[m * K + k] = (int8_t)((int)field - 1);
+            if (k < K)
+                codes[m * K + k] = (int8_t)((int)field - 1);
+            else if (field != 1u)
+                bad = 1;       /* padding must hold code 0 */
         }
     }
     return bad ? -1 : 0;

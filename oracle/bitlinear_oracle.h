@@ -22,9 +22,11 @@
  * accumulation over bit-packed codes).
  *
  * Packed layout (defined by this project; the pages fix only 2.0 bpw):
- *   row m of W occupies K/16 little-endian uint32 words;
- *   weight k sits in word k/16 at bit 8*(k%4) + 2*((k%16)/4);
- *   the 2-bit field holds the offset-binary code c+1 in {0,1,2}; 3 never occurs.
+ *   row m of W occupies 4*ceil(K/64) little-endian uint32 words (K/16 when K
+ *   is a multiple of 64; otherwise the row is padded to a 16-byte boundary);
+ *   weight k sits in word k/16 of its row at bit 8*(k%4) + 2*((k%16)/4);
+ *   the 2-bit field holds the offset-binary code c+1 in {0,1,2}; 3 never
+ *   occurs; padding fields past K hold 01, i.e. code 0, weight nothing.
  *
  * Error convention: functions returning int give 0 on success, a negative
  * value on a rejected input (documented per function).
@@ -53,11 +55,15 @@ float oracle_absmean(const float* w, int64_t n, int* status);
 /* codes[i] = clamp(rint(w[i]/alpha), -1, 1); all zero when alpha == 0. */
 void oracle_ternarize(const float* w, int64_t n, float alpha, int8_t* codes);
 
-/* Pack codes [M,K] (K % 16 == 0) into M*K/16 words.  Returns -1 on a code
- * outside {-1,0,1} or a bad K. */
+/* Words per packed row: 4*ceil(K/64). */
+int64_t oracle_packed_row_words(int64_t K);
+
+/* Pack codes [M,K] (K % 16 == 0) into M*oracle_packed_row_words(K) words.
+ * Returns -1 on a code outside {-1,0,1} or a bad K. */
 int oracle_pack(const int8_t* codes, int64_t M, int64_t K, uint32_t* packed);
 
-/* Inverse of oracle_pack.  Returns -1 if a field holds 3. */
+/* Inverse of oracle_pack.  Returns -1 if a field holds 3 or a padding field
+ * is not code 0. */
 int oracle_unpack(const uint32_t* packed, int64_t M, int64_t K, int8_t* codes);
 
 /* Per-token absmax int8 quantisation of x [N,K].  qsum may be NULL. */

@@ -177,12 +177,13 @@ def test_pack_layout_hand_derived_words():
     c = np.zeros((2, 32), dtype=np.int8)
     c[1, 16] = 1
     p = oracle.pack(c)
-    assert p.shape == (2, 2) and p[1, 1] == 0x55555556 and p[1, 0] == 0x55555555
+    assert p.shape == (2, 4) and p[1, 1] == 0x55555556 and p[1, 0] == 0x55555555
+    assert (p[:, 2:] == 0x55555555).all()    # row padded to 16 bytes with code 0
 
 
 def test_pack_roundtrip_size_and_byte_lanes():
     r = rng(12)
-    M, K = 24, 96
+    M, K = 24, 128
     c = r.integers(-1, 2, size=(M, K)).astype(np.int8)
     p = oracle.pack(c)
     facts = json.load(open(os.path.join(GOLDEN, "pages_facts.json")))
@@ -197,6 +198,45 @@ def test_pack_roundtrip_size_and_byte_lanes():
         lanes = ((p >> np.uint32(2 * j)) & np.uint32(0x03030303)).view(np.uint8)
         lanes = lanes.reshape(M, K // 16, 4).astype(np.int16) - 1
         assert np.array_equal(lanes, c.reshape(M, K // 16, 4, 4)[:, :, j, :])
+
+
+@pytest.mark.parametrize("K", [16, 48, 80, 96, 1008])
+def test_pack_ragged_rows_padded_with_code_zero(K):
+    # rows whose K is not a multiple of 64 are padded to a 16-byte boundary;
+    # padding fields hold 01 (code 0), so a padded row weighs exactly what the
+    # unpadded one does
+    r = rng(K)
+    M = 5
+    c = r.integers(-1, 2, size=(M, K)).astype(np.int8)
+    p = oracle.pack(c)
+    wpr = -(-K // 64) * 4
+    assert oracle.packed_row_words(K) == wpr and p.shape == (M, wpr)
+    assert p.nbytes % (16 * M) == 0
+    assert np.array_equal(oracle.unpack(p, M, K), c)
+    # the first K/16 words are the unpadded layout, word by word
+    for m in range(M):
+        for w in range(K // 16):
+            word = 0
+            for i in range(16):
+                k = 16 * w + i
+                word |= (int(c[m, k]) + 1) << (8 * (k % 4) + 2 * ((k % 16) // 4))
+            assert p[m, w] == word
+    assert (p[:, K // 16:] == 0x55555555).all()
+    # a padding field that is not code 0 is rejected
+    if K % 64:
+        bad = p.copy()
+        bad[0, -1] ^= np.uint32(1)
+        with pytest.raises(ValueError):
+            oracle.unpack(bad, M, K)
+    # the padding changes no product: acc over the padded row equals acc over K
+    q = r.integers(-128, 128, size=(3, K)).astype(np.int8)
+    assert np.array_equal(oracle.matmul_i32(oracle.unpack(p, M, K), q),
+                          oracle.matmul_addsub(c, q))
+
+
+def test_packed_rows_are_unpadded_when_k_is_a_multiple_of_64():
+    for K in (64, 128, 2560, 6912, 11008, 28672):
+        assert oracle.packed_row_words(K) == K // 16
 
 
 def test_pack_rejects_bad_input():
