@@ -19,9 +19,12 @@
  * over bit-packed codes, no intermediate writes).
  *
  * Packed weight layout ("I2_S-style", defined by this library):
- *   row m occupies K/16 little-endian uint32 words (K/4 bytes), rows contiguous;
- *   weight k lives in word k/16 at bit 8*(k%4) + 2*((k%16)/4);
- *   the 2-bit field holds c+1 (0 -> -1, 1 -> 0, 2 -> +1); 3 is never written.
+ *   row m occupies WP(K) = 4*ceil(K/64) little-endian uint32 words, rows
+ *   contiguous: K/16 words (K/4 bytes, exactly 2.0 bits per weight) when K is
+ *   a multiple of 64, otherwise padded to the next 16-byte boundary;
+ *   weight k lives in word k/16 of its row at bit 8*(k%4) + 2*((k%16)/4);
+ *   the 2-bit field holds c+1 (0 -> -1, 1 -> 0, 2 -> +1); 3 is never written;
+ *   padding fields past K hold 01 (code 0).
  *   So (word >> 2j) & 0x03030303 gives, one per byte, the fields of weights
  *   16*(k/16)+4j .. +3 in k order.
  *
@@ -31,8 +34,8 @@
  *   - Pointers are DEVICE pointers unless stated otherwise.  Array pointers
  *     (W, packed, x, xq, y, acc, workspace) must be 16-byte aligned; the
  *     scalar-per-token pointers (alpha, amax, xsum) 4-byte aligned.
- *   - Shapes: K must be a positive multiple of 128 and at most 131072; M >= 1
- *     (a multiple of 128 for bitlinear_gemm); M*K <= 2^40.  N = 0 is a no-op.
+ *   - Shapes: K must be a positive multiple of 16 and at most 131072; any
+ *     M >= 1; M*K <= 2^40.  N = 0 is a no-op.
  *   - Every call is asynchronous on `stream` (NULL = the legacy default
  *     stream).  Argument errors are returned synchronously before anything is
  *     launched; a failed launch returns BITLINEAR_ERR_CUDA.
@@ -61,7 +64,7 @@ typedef struct CUstream_st* bitlinear_stream_t;
 typedef enum {
     BITLINEAR_OK = 0,
     BITLINEAR_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size */
-    BITLINEAR_ERR_UNSUPPORTED_SHAPE = 2, /* K % 128, M % 128 (GEMM), N range, size limits */
+    BITLINEAR_ERR_UNSUPPORTED_SHAPE = 2, /* K % 16, N range, size limits */
     BITLINEAR_ERR_MISALIGNED = 3,        /* pointer not 16-byte aligned */
     BITLINEAR_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than required */
     BITLINEAR_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
@@ -84,7 +87,8 @@ BITLINEAR_API size_t bitlinear_pack_workspace_bytes(int64_t M, int64_t K);
  * Absmean-ternarise and pack one weight tensor (reading notes section 1.1 and
  * 2.3; scale rule as in BitNet b1.58, alpha = mean|W|).
  *   W        fp32 [M,K] latent weights (device, read only)
- *   packed   uint32 [M, K/16] output in the layout above (M*K/4 bytes)
+ *   packed   uint32 [M, WP(K)] output in the layout above (M*K/4 bytes when
+ *            K is a multiple of 64)
  *   alpha    fp32 [1] output: mean|W| rounded to nearest-even once, from an
  *            exact, order-independent sum; 0 when W is all zero (every code 0)
  *   workspace, workspace_bytes: scratch of bitlinear_pack_workspace_bytes()
@@ -174,7 +178,9 @@ BITLINEAR_API bitlinear_status bitlinear_gemv(const uint32_t* packed, const floa
  * accumulators in tensor memory): packed weight tiles are brought in by TMA,
  * expanded to int8 in shared memory and multiplied with TMA-loaded int8
  * activation tiles; the rescale is fused into the epilogue.  Same arguments
- * and results as bitlinear_gemv; M must be a multiple of 128.
+ * and results as bitlinear_gemv, any M.  Ragged tiles read zeros past M, K
+ * and N through the tensor maps; when 4*M is not a multiple of 16 the
+ * outputs are written with plain stores instead of tensor stores.
  * The reading notes (section 4.4) name prefill, where the work turns
  * compute-bound, as the stage their CPU kernels leave unoptimised.
  */
@@ -186,11 +192,11 @@ BITLINEAR_API bitlinear_status bitlinear_gemm(const uint32_t* packed, const floa
 
 /*
  * One linear layer of a grouped call.  Every pointer follows the conventions
- * above; M and K are this layer's shape (K a multiple of 128; for the GEMM, M a
- * multiple of 128).  All layers of one call share the token count N.
+ * above; M and K are this layer's shape.  All layers of one call share the
+ * token count N.
  */
 typedef struct {
-    const uint32_t* packed;   /* [M, K/16] words */
+    const uint32_t* packed;   /* [M, WP(K)] words */
     const float* alpha;       /* [1] */
     int64_t M;
     int64_t K;
@@ -248,7 +254,7 @@ BITLINEAR_API bitlinear_status bitlinear_gemv_quant(const uint32_t* packed, cons
 
 /* One layer of a fused grouped call: the layer and its fp32 input. */
 typedef struct {
-    const uint32_t* packed;   /* [M, K/16] words */
+    const uint32_t* packed;   /* [M, WP(K)] words */
     const float* alpha;       /* [1] */
     int64_t M;
     int64_t K;

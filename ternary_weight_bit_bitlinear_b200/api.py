@@ -25,11 +25,18 @@ def _need(t, dtype, name):
         raise ValueError("%s must be contiguous" % name)
 
 
+def packed_row_words(K):
+    """Words per packed row: K/16 rounded up to a multiple of 4 (rows end on a
+    16-byte boundary; the padding fields hold code 0)."""
+    return 4 * ((K + 63) // 64)
+
+
 def pack_weights(W, stream=None):
-    """fp32 W[M,K] -> (packed int32 [M, K/16] holding the uint32 words, alpha fp32 [1])."""
+    """fp32 W[M,K] -> (packed int32 [M, packed_row_words(K)] holding the uint32
+    words, alpha fp32 [1])."""
     _need(W, torch.float32, "W")
     M, K = W.shape
-    packed = torch.empty((M, K // 16), dtype=torch.int32, device=W.device)
+    packed = torch.empty((M, packed_row_words(K)), dtype=torch.int32, device=W.device)
     alpha = torch.empty(1, dtype=torch.float32, device=W.device)
     nbytes = _lib.bitlinear_pack_workspace_bytes(M, K)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
@@ -88,9 +95,9 @@ def _matmul(fn, name, packed, alpha, xq, amax, xsum, M, with_acc, stream, out=No
     _need(amax, torch.float32, "amax")
     _need(xsum, torch.int32, "xsum")
     N, K = xq.shape
-    if packed.shape != (M, K // 16):
-        raise ValueError("packed must be [M, K/16] = [%d, %d], got %s" % (M, K // 16,
-                                                                         tuple(packed.shape)))
+    if packed.shape != (M, packed_row_words(K)):
+        raise ValueError("packed must be [M, packed_row_words(K)] = [%d, %d], got %s"
+                         % (M, packed_row_words(K), tuple(packed.shape)))
     y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=xq.device)
     acc = torch.empty((N, M), dtype=torch.int32, device=xq.device) if with_acc else None
     _lib.check(fn(packed, alpha, M, K, xq, amax, xsum, N, y, acc, stream), name)
@@ -116,8 +123,9 @@ def _grouped(fn, name, layers, xq, amax, xsum, with_acc, stream, outs):
         _need(alpha, torch.float32, "alpha")
         _need(xqs[i], torch.int8, "xq")
         M, K = packed.shape[0], xqs[i].shape[1]
-        if xqs[i].shape[0] != N or packed.shape[1] != K // 16:
-            raise ValueError("layer %d: packed [M, K/16] must match xq [N, K]; N shared" % i)
+        if xqs[i].shape[0] != N or packed.shape[1] != packed_row_words(K):
+            raise ValueError("layer %d: packed [M, packed_row_words(K)] must match xq [N, K];"
+                             " N shared" % i)
         y = outs[i] if outs is not None else torch.empty((N, M), dtype=torch.float32,
                                                            device=packed.device)
         acc = torch.empty((N, M), dtype=torch.int32, device=packed.device) if with_acc else None
@@ -139,23 +147,23 @@ def gemv_grouped(layers, xq, amax, xsum, with_acc=False, stream=None, outs=None)
 
 
 def gemm_grouped(layers, xq, amax, xsum, with_acc=False, stream=None, outs=None):
-    """Tensor-core GEMM over several layers in one persistent launch (M % 128
-    == 0 for each); same arguments as gemv_grouped."""
+    """Tensor-core GEMM over several layers in one persistent launch; same
+    arguments as gemv_grouped."""
     return _grouped(_lib.bitlinear_gemm_grouped, "bitlinear_gemm_grouped", layers, xq, amax,
                     xsum, with_acc, stream, outs)
 
 
 def gemm(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out=None):
-    """Tensor-core GEMM (any N, M % 128 == 0): y[N,M] fp32 (and int32 acc)."""
+    """Tensor-core GEMM (any N and M): y[N,M] fp32 (and int32 acc)."""
     M = packed.shape[0] if M is None else M
     return _matmul(_lib.bitlinear_gemm, "bitlinear_gemm", packed, alpha, xq, amax, xsum, M,
                    with_acc, stream, out)
 
 
 def matmul(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out=None):
-    """GEMV for N <= GEMV_MAX_TOKENS (or when M is not a multiple of 128), else GEMM."""
+    """GEMV for N <= GEMV_MAX_TOKENS, else the tensor-core GEMM."""
     M = packed.shape[0] if M is None else M
-    if xq.shape[0] <= GEMV_MAX_TOKENS or M % 128 != 0:
+    if xq.shape[0] <= GEMV_MAX_TOKENS:
         return gemv(packed, alpha, xq, amax, xsum, M, with_acc, stream, out)
     return gemm(packed, alpha, xq, amax, xsum, M, with_acc, stream, out)
 
@@ -177,9 +185,9 @@ def gemv_quant(packed, alpha, x, M=None, with_acc=False, stream=None, out=None):
     _need(x, torch.float32, "x")
     M = packed.shape[0] if M is None else M
     N, K = x.shape
-    if packed.shape != (M, K // 16):
-        raise ValueError("packed must be [M, K/16] = [%d, %d], got %s" % (M, K // 16,
-                                                                         tuple(packed.shape)))
+    if packed.shape != (M, packed_row_words(K)):
+        raise ValueError("packed must be [M, packed_row_words(K)] = [%d, %d], got %s"
+                         % (M, packed_row_words(K), tuple(packed.shape)))
     y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=x.device)
     acc = torch.empty((N, M), dtype=torch.int32, device=x.device) if with_acc else None
     _lib.check(_lib.bitlinear_gemv_quant(packed, alpha, M, K, x, N, y, acc, stream),
@@ -202,8 +210,9 @@ def gemv_quant_grouped(layers, x, with_acc=False, stream=None, outs=None):
         _need(alpha, torch.float32, "alpha")
         _need(xs[i], torch.float32, "x")
         M, K = packed.shape[0], xs[i].shape[1]
-        if xs[i].shape[0] != N or packed.shape[1] != K // 16:
-            raise ValueError("layer %d: packed [M, K/16] must match x [N, K]; N shared" % i)
+        if xs[i].shape[0] != N or packed.shape[1] != packed_row_words(K):
+            raise ValueError("layer %d: packed [M, packed_row_words(K)] must match x [N, K];"
+                             " N shared" % i)
         y = outs[i] if outs is not None else torch.empty((N, M), dtype=torch.float32,
                                                            device=packed.device)
         acc = torch.empty((N, M), dtype=torch.int32, device=packed.device) if with_acc else None

@@ -47,9 +47,12 @@ bitlinear_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
 }
 
+// Words per packed row: K/16 rounded up to a multiple of 4 (16 bytes).
+int64_t packed_row_words(int64_t K) { return 4 * ((K + 63) / 64); }
+
 bitlinear_status check_mk(int64_t M, int64_t K) {
   if (M < 0 || K < 0) return BITLINEAR_ERR_INVALID_ARG;
-  if (M == 0 || K == 0 || K % 128 != 0 || K > kMaxK) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || K == 0 || K % 16 != 0 || K > kMaxK) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   if (M > INT_MAX / 2 || M * K > kMaxElems) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   return BITLINEAR_OK;
 }
@@ -174,7 +177,7 @@ bitlinear_status gemv_group(const bitlinear_problem* probs, int64_t count, int64
       g.acc = q.acc;
       g.M = static_cast<int>(q.M);
       g.K = static_cast<int>(q.K);
-      g.W = static_cast<int>(q.K / 16);
+      g.W = static_cast<int>(packed_row_words(q.K));
       g.unit_begin = static_cast<int>(units);
       units += (q.M + bl::kGemvTileRows - 1) / bl::kGemvTileRows;
     }
@@ -274,10 +277,12 @@ void build_gemm_schedule(bl::GemmParams& p, int sms) {
   p.use_sched = 1;
 }
 
-// Tensor-core GEMM over problems that share N (all validated, M % 128 == 0):
-// one persistent launch per kGemmMaxProblems problems, tiles numbered across
+// Tensor-core GEMM over problems that share N (all validated): one
+// persistent launch per kGemmMaxProblems problems, tiles numbered across
 // problems with the largest K first so the longest tiles start in the first
-// wave.
+// wave.  Ragged edges come from the tensor maps: loads past M, K or N read
+// zeros, and stores past M or N are dropped.  A y whose row pitch (4M bytes)
+// is not a multiple of 16 cannot be a TMA tensor; its epilogue stores directly.
 bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64_t N,
                             cudaStream_t s) {
   DeviceInfo* dev = nullptr;
@@ -302,13 +307,14 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     int64_t tiles = 0;
     for (int i = 0; i < n; ++i) {
       const bitlinear_problem& q = probs[base + order[i]];
-      if (!encode_u8_2d(&p.tmA[i], q.packed, static_cast<uint64_t>(q.K / 4),
+      const bool direct = q.M % 4 != 0;
+      if (!encode_u8_2d(&p.tmA[i], q.packed, static_cast<uint64_t>(packed_row_words(q.K) * 4),
                         static_cast<uint64_t>(q.M), bl::kGemmPackedRowBytes, bl::kGemmBM,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
           !encode_u8_2d(&p.tmB[i], q.xq, static_cast<uint64_t>(q.K), static_cast<uint64_t>(N),
                         bl::kGemmBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !encode_f32_2d(&p.tmY[i], q.y, static_cast<uint64_t>(q.M), static_cast<uint64_t>(N),
-                         32, 32))
+          (!direct && !encode_f32_2d(&p.tmY[i], q.y, static_cast<uint64_t>(q.M),
+                                     static_cast<uint64_t>(N), 32, 32)))
         return BITLINEAR_ERR_CUDA;
       bl::GemmProblem& g = p.prob[i];
       g.alpha = q.alpha;
@@ -321,7 +327,8 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
       g.N = static_cast<int>(N);
       g.n_tiles = static_cast<int>(n_tiles);
       g.tile_begin = static_cast<int>(tiles);
-      tiles += (q.M / bl::kGemmBM) * n_tiles;
+      g.direct_store = direct ? 1 : 0;
+      tiles += (q.M + bl::kGemmBM - 1) / bl::kGemmBM * n_tiles;
     }
     if (tiles > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     p.num_problems = n;
@@ -468,7 +475,7 @@ bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t 
         g.y = q.y;
         g.acc = q.acc;
         g.M = static_cast<int>(q.M);
-        g.W = static_cast<int>(q.K / 16);
+        g.W = static_cast<int>(packed_row_words(q.K));
         g.unit_begin = static_cast<int>(units);
         const int64_t u = (q.M + bl::kGemvTileRows - 1) / bl::kGemvTileRows;
         const bool same = segs > 0 && p.seg[segs - 1].x == q.x && p.seg[segs - 1].K == q.K;
@@ -557,11 +564,13 @@ bitlinear_status bitlinear_pack_weights(const float* W, int64_t M, int64_t K, ui
   bl::abs_bins_kernel<<<grid, bl::kBinsThreads, 0, s>>>(reinterpret_cast<const float4*>(W), n4,
                                                          bins, flag);
   bl::alpha_finalize_kernel<<<1, 32, 0, s>>>(bins, flag, static_cast<uint64_t>(M * K), alpha);
-  const int64_t words = M * K / 16;
+  const int64_t wp = packed_row_words(K);
+  const int64_t words = M * wp;
   int64_t g = (words + 255) / 256;
   if (g > dev->sms * 16) g = dev->sms * 16;
   bl::ternarize_pack_kernel<<<static_cast<int>(g), 256, 0, s>>>(
-      reinterpret_cast<const float4*>(W), words, alpha, packed);
+      reinterpret_cast<const float4*>(W), M, static_cast<int>(K / 16), static_cast<int>(wp),
+      alpha, packed);
   return launch_status();
 }
 
@@ -577,7 +586,7 @@ bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* acts, int64_t 
   for (int64_t i = 0; i < count; ++i) {
     const bitlinear_act& a = acts[i];
     if (a.N < 0 || a.K < 0) return BITLINEAR_ERR_INVALID_ARG;
-    if (a.K == 0 || a.K % 128 != 0 || a.K > kMaxK || a.N > INT_MAX)
+    if (a.K == 0 || a.K % 16 != 0 || a.K > kMaxK || a.N > INT_MAX)
       return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     if (a.N == 0) continue;
     if (!a.x || !a.xq || !a.amax) return BITLINEAR_ERR_INVALID_ARG;
@@ -622,7 +631,7 @@ bitlinear_status bitlinear_quant_act_per_tensor(const float* x, int64_t N, int64
                                                 size_t workspace_bytes,
                                                 bitlinear_stream_t stream) {
   if (N < 0 || K < 0) return BITLINEAR_ERR_INVALID_ARG;
-  if (K == 0 || K % 128 != 0 || K > kMaxK || N > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  if (K == 0 || K % 16 != 0 || K > kMaxK || N > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   if (N == 0) return BITLINEAR_OK;
   if (!x || !xq || !amax) return BITLINEAR_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < 16) return BITLINEAR_ERR_WORKSPACE;
@@ -684,7 +693,6 @@ bitlinear_status bitlinear_gemm(const uint32_t* packed, const float* alpha, int6
                                 int64_t N, float* y, int32_t* acc, bitlinear_stream_t stream) {
   bitlinear_status st = check_matmul_args(packed, alpha, M, K, xq, amax, xsum, N, y, acc);
   if (st != BITLINEAR_OK || N == 0) return st;
-  if (M % 128 != 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   const bitlinear_problem q = {packed, alpha, M, K, xq, amax, xsum, y, acc};
   return gemm_group(&q, 1, N, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -696,7 +704,6 @@ bitlinear_status bitlinear_gemm_grouped(const bitlinear_problem* problems, int64
   for (int64_t i = 0; i < count; ++i) {
     bitlinear_status st = check_problem(problems[i], N);
     if (st != BITLINEAR_OK) return st;
-    if (problems[i].M % 128 != 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   }
   return gemm_group(problems, count, N, reinterpret_cast<cudaStream_t>(stream));
 }

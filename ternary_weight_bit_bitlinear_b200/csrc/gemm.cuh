@@ -48,10 +48,11 @@ struct GemmProblem {
   int M, K, N;
   int n_tiles;      // ceil(N / BN)
   int tile_begin;   // first global tile of this problem
+  int direct_store; // 1: y is written with plain stores (its row pitch is not a TMA stride)
 };
 
 struct GemmParams {
-  CUtensorMap tmA[kGemmMaxProblems];   // packed weights as uint8 [M][K/4], box 32 x 128
+  CUtensorMap tmA[kGemmMaxProblems];   // packed weights as uint8 [M][row bytes], box 32 x 128
   CUtensorMap tmB[kGemmMaxProblems];   // xq as uint8 [N][K], box 128 x BN, 128B swizzle
   CUtensorMap tmY[kGemmMaxProblems];   // y as fp32 [N][M], box 32 x 32
   GemmProblem prob[kGemmMaxProblems];
@@ -162,7 +163,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         const int tile = gemm_my_tile(p, ti);
         int pi, m_blk, n_blk;
         gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
-        const int kblocks = p.prob[pi].K / kGemmBK;
+        const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort)) goto producer_done;
           mbar_arrive_expect_tx(&s.full[stage], kStageTx);
@@ -184,7 +185,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         const int tile = gemm_my_tile(p, ti);
         int pi, m_blk, n_blk;
         gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
-        const int kblocks = p.prob[pi].K / kGemmBK;
+        const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
         const uint32_t ab = it & 1, ap = (it >> 1) & 1;
         if (!mbar_wait(&s.tempty[ab], ap ^ 1u, abort)) break;
         tc_fence_after();
@@ -232,7 +233,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         const int tile = gemm_my_tile(p, ti);
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
-      const int kblocks = p.prob[pi].K / kGemmBK;
+      const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait(&s.full[stage], phase, abort) ||
             !mbar_wait(&s.uempty[ub], uphase ^ 1u, abort))
@@ -308,6 +309,19 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         tmem_ld_wait();
         const int n0 = n_blk * BN + cc * 32;
         if (n0 >= pr.N) continue;          // tokens past N: nothing to store
+        if (pr.direct_store) {   // rows past M and tokens past N are not stored
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int a = static_cast<int>(r[j]) - xs[(cc >> 1) * 32 + j];
+            if (m < pr.M && n0 + j < pr.N) {
+              const int64_t o = static_cast<int64_t>(n0 + j) * pr.M + m;
+              pr.y[o] = __fmul_rn(__int2float_rn(a), sc[(cc >> 1) * 32 + j]);
+              if (pr.acc) pr.acc[o] = a;
+            }
+          }
+          continue;
+        }
+        if (m_blk * kGemmBM + static_cast<int>(quarter) * 32 >= pr.M) continue;   // rows past M
         float* blk = s.ep_out[e];
         if (lane == 0) bulk_wait_group_read<0>();   // the previous store has read the block
         __syncwarp();
@@ -315,7 +329,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         for (int j = 0; j < 32; ++j) {
           const int a = static_cast<int>(r[j]) - xs[(cc >> 1) * 32 + j];
           blk[j * 32 + lane] = __fmul_rn(__int2float_rn(a), sc[(cc >> 1) * 32 + j]);
-          if (pr.acc && n0 + j < pr.N)
+          if (pr.acc && n0 + j < pr.N && m < pr.M)
             pr.acc[static_cast<int64_t>(n0 + j) * pr.M + m] = a;
         }
         fence_proxy_async_smem();

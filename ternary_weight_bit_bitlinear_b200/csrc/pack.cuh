@@ -137,18 +137,31 @@ __global__ void alpha_finalize_kernel(const unsigned long long* __restrict__ bin
   *alpha = static_cast<float>(ldexp(static_cast<double>(mant), ulp_final - 149));
 }
 
-// One thread per packed word (16 consecutive weights of one row).
+// One thread per packed word.  A row holds `wp` words: the first `kw` =
+// K/16 carry 16 consecutive weights each, the rest (when K is not a multiple
+// of 64) pad the row to a 16-byte boundary with code-0 fields (01).
 __global__ void __launch_bounds__(256)
-ternarize_pack_kernel(const float4* __restrict__ w4, int64_t words,
+ternarize_pack_kernel(const float4* __restrict__ w4, int64_t rows, int kw, int wp,
                       const float* __restrict__ alpha_ptr, uint32_t* __restrict__ packed) {
   const float alpha = *alpha_ptr;
+  const int64_t words = rows * wp;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < words;
        w += stride) {
+    int64_t src = 4 * w;                  // float4 index of the word's first weight
+    if (wp != kw) {
+      const int64_t m = w / wp;
+      const int r = static_cast<int>(w - m * wp);
+      if (r >= kw) {
+        packed[w] = 0x55555555u;
+        continue;
+      }
+      src = 4 * (m * kw + r);
+    }
     uint32_t word = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {          // weights 4j .. 4j+3 of the word
-      float4 v = __ldcs(w4 + 4 * w + j);
+      float4 v = __ldcs(w4 + src + j);
       float e4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int b = 0; b < 4; ++b) {

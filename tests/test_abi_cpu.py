@@ -109,10 +109,9 @@ def test_matmul_argument_errors(L, name):
     assert call(y=MISALIGNED) == _lib.ERR_MISALIGNED
     assert call(acc=MISALIGNED) == _lib.ERR_MISALIGNED
     assert call(xq=MISALIGNED) == _lib.ERR_MISALIGNED
+    assert call(K=40) == _lib.ERR_UNSUPPORTED_SHAPE      # K must be a multiple of 16
     if name == "bitlinear_gemv":
         assert call(N=17) == _lib.ERR_UNSUPPORTED_SHAPE
-    else:
-        assert call(M=200) == _lib.ERR_UNSUPPORTED_SHAPE
 
 
 def test_header_is_self_contained(tmp_path):
@@ -146,10 +145,9 @@ def test_grouped_argument_errors(L, name):
     assert f((P * 2)(good, prob(y=MISALIGNED)), 2, 1, None) == _lib.ERR_MISALIGNED
     assert f((P * 2)(good, prob(alpha=0)), 2, 1, None) == _lib.ERR_INVALID_ARG
     assert f((P * 2)(good, prob(alpha=FAKE + 2)), 2, 1, None) == _lib.ERR_MISALIGNED
+    assert f((P * 2)(good, prob(K=40)), 2, 1, None) == _lib.ERR_UNSUPPORTED_SHAPE
     if name == "bitlinear_gemv_grouped":
         assert f(arr, 2, 17, None) == _lib.ERR_UNSUPPORTED_SHAPE
-    else:
-        assert f((P * 2)(good, prob(M=200)), 2, 1, None) == _lib.ERR_UNSUPPORTED_SHAPE
 
 
 def test_quant_act_grouped_argument_errors(L):

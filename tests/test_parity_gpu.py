@@ -325,5 +325,5 @@ def test_rejects_bad_shapes_on_device():
     y = torch.empty(17, 256, device="cuda")
     assert _lib.bitlinear_gemv(packed, alpha, 256, 256, xq, amax, xsum, 17, y) == \
         _lib.ERR_UNSUPPORTED_SHAPE
-    assert _lib.bitlinear_gemm(packed, alpha, 200, 256, xq, amax, xsum, 17, y) == \
+    assert _lib.bitlinear_gemm(packed, alpha, 256, 200, xq, amax, xsum, 17, y) == \
         _lib.ERR_UNSUPPORTED_SHAPE

@@ -43,7 +43,7 @@ def test_noalloc_matches_workspace_entry_point_twice(L):
     for seed, (M, K) in ((7001, (640, 2560)), (7002, (2560, 6912))):
         W = inputs.latent_weights(M, K, seed=seed, device="cuda")
         ref_packed, ref_alpha = api.pack_weights(W)
-        packed = torch.empty((M, K // 16), dtype=torch.int32, device="cuda")
+        packed = torch.empty((M, api.packed_row_words(K)), dtype=torch.int32, device="cuda")
         alpha = torch.empty(1, dtype=torch.float32, device="cuda")
         _lib.check(_lib.bitlinear_pack_weights_noalloc(W, M, K, packed, alpha),
                    "bitlinear_pack_weights_noalloc")
