@@ -410,33 +410,35 @@ bitlinear_status gemv_quant_launch(int N, int grid, const bl::GqParams& p, cudaS
   return launch_status();
 }
 
-// Warps per segment: one each, then the rest one at a time to the segment
-// whose warps have the most work (never more warps than units).  A warp's
-// work is its share of k-chunks plus one unit's worth for quantising the
-// input first, whose copy time grows with K like a unit's.  This minimises
-// the largest per-warp estimate.
+// Warps per segment.  Each warp of a segment takes ceil(units / warps) units
+// at most, so a warp's work is that many units of k-chunks, plus about half a
+// unit for staging and quantising its input first (its copy time grows with K
+// like a unit's).  Starting from one warp each, the segment with the largest
+// estimate gets just enough warps for its largest share to drop by one unit,
+// until the warps run out; this minimises the largest estimate.
 void gemv_quant_assign(bl::GqParams& p, int warps_total) {
   const int n = p.num_segments;
   std::vector<int> w(n, 1);
-  int used = n;
+  int left = warps_total - n;
   auto load = [&](int g) {
-    return (static_cast<double>(p.seg[g].units) / w[g] + 1.0) * p.seg[g].chunks;
+    const int per = (p.seg[g].units + w[g] - 1) / w[g];
+    return (2 * per + 1) * p.seg[g].chunks;   // twice (per + 1/2) units of chunks
   };
-  auto cmp = [&](int a, int b) { return load(a) < load(b); };
-  std::vector<int> heap;
-  for (int g = 0; g < n; ++g)
-    if (p.seg[g].units > 1) heap.push_back(g);
-  std::make_heap(heap.begin(), heap.end(), cmp);
-  while (used < warps_total && !heap.empty()) {
-    std::pop_heap(heap.begin(), heap.end(), cmp);
-    const int g = heap.back();
+  std::vector<std::pair<int, int>> heap;   // (load, segment), max-heap
+  for (int g = 0; g < n; ++g) heap.push_back({load(g), g});
+  std::make_heap(heap.begin(), heap.end());
+  while (!heap.empty()) {
+    std::pop_heap(heap.begin(), heap.end());
+    const int g = heap.back().second;
     heap.pop_back();
-    ++w[g];
-    ++used;
-    if (w[g] < p.seg[g].units) {
-      heap.push_back(g);
-      std::push_heap(heap.begin(), heap.end(), cmp);
-    }
+    const int per = (p.seg[g].units + w[g] - 1) / w[g];
+    if (per <= 1) continue;                 // one unit per warp already: cannot drop
+    const int need = (p.seg[g].units + per - 2) / (per - 1) - w[g];
+    if (need > left) break;                 // the largest estimate cannot drop any further
+    w[g] += need;
+    left -= need;
+    heap.push_back({load(g), g});
+    std::push_heap(heap.begin(), heap.end());
   }
   int begin = 0;
   for (int g = 0; g < n; ++g) {
