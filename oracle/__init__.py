@@ -33,6 +33,12 @@ def lib():
         L.oracle_absmean.restype = ctypes.c_float
         L.oracle_ternarize.argtypes = [p, i64, ctypes.c_float, p]
         L.oracle_ternarize.restype = None
+        L.oracle_tl2_row_bytes.argtypes = [i64]
+        L.oracle_tl2_row_bytes.restype = i64
+        L.oracle_tl2_encode.argtypes = [p, i64, i64, p]
+        L.oracle_tl2_encode.restype = ctypes.c_int
+        L.oracle_tl2_decode.argtypes = [p, i64, i64, p]
+        L.oracle_tl2_decode.restype = ctypes.c_int
         L.oracle_packed_row_words.argtypes = [i64]
         L.oracle_packed_row_words.restype = i64
         L.oracle_pack.argtypes = [p, i64, i64, p]
@@ -108,6 +114,29 @@ def unpack(packed, M, K):
     out = np.empty((M, K), dtype=np.int8)
     if lib().oracle_unpack(pp, M, K, out.ctypes.data) != 0:
         raise ValueError("invalid 2-bit field (3) or bad K")
+    return out
+
+
+def tl2_row_bytes(K):
+    """Bytes of one TL2-style row (index plane, sign plane, 2-bit remainder)."""
+    return int(lib().oracle_tl2_row_bytes(int(K)))
+
+
+def tl2_encode(codes):
+    """codes int8 [M,K] -> uint8 [M, tl2_row_bytes(K)] (5 bits per 3 weights)."""
+    codes, pc = _c(codes, np.int8)
+    M, K = codes.shape
+    out = np.empty((M, tl2_row_bytes(K)), dtype=np.uint8)
+    if lib().oracle_tl2_encode(pc, M, K, out.ctypes.data) != 0:
+        raise ValueError("bad code or K % 16 != 0")
+    return out
+
+
+def tl2_decode(data, M, K):
+    data, pd = _c(data, np.uint8)
+    out = np.empty((M, K), dtype=np.int8)
+    if lib().oracle_tl2_decode(pd, M, K, out.ctypes.data) != 0:
+        raise ValueError("invalid TL2 row")
     return out
 
 

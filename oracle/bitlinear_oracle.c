@@ -216,6 +216,123 @@ int oracle_unpack(const uint32_t* packed, int64_t M, int64_t K, int8_t* codes)
 }
 
 /* ------------------------------------------------------------------------- */
+/* TL2-style storage at 5/3 bits per weight (reading notes section 2.3       */
+/* "technical details": three ternary weights stored as a 1-bit sign plus a  */
+/* 4-bit index, 5 bits in all, by folding each combination onto its mirror  */
+/* image; K split into a part stored in groups of three and a remainder).    */
+/* The index table and byte layout are this project's own (see header).     */
+/* ------------------------------------------------------------------------- */
+
+static int64_t tl2_blocks(int64_t K) { return K / 96; }
+
+int64_t oracle_tl2_row_bytes(int64_t K)
+{
+    int64_t nb = tl2_blocks(K);
+    int64_t k2 = K - 96 * nb;
+    return 16 * nb + 16 * ((nb + 3) / 4) + 16 * ((k2 + 63) / 64);
+}
+
+/* One group of three codes -> (sign, index): the base-3 number of the codes
+ * plus one, v = 9(c0+1) + 3(c1+1) + (c2+1) in [0, 26], mirrors to 26 - v when
+ * every code is negated; v = 13 is (0,0,0), its own mirror.  The index is
+ * |v - 13| in [0, 13] and the sign says which side of 13 v lies on. */
+static void tl2_encode_group(int c0, int c1, int c2, int* sign, int* index)
+{
+    int v = 9 * (c0 + 1) + 3 * (c1 + 1) + (c2 + 1);
+    if (v >= 13) { *sign = 0; *index = v - 13; }
+    else         { *sign = 1; *index = 13 - v; }
+}
+
+static void tl2_decode_group(int sign, int index, int* c)
+{
+    int v = sign ? 13 - index : 13 + index;
+    c[0] = v / 9 - 1;
+    c[1] = (v / 3) % 3 - 1;
+    c[2] = v % 3 - 1;
+}
+
+int oracle_tl2_encode(const int8_t* codes, int64_t M, int64_t K, uint8_t* out)
+{
+    if (K % 16 != 0 || M < 0) return -1;
+    int64_t nb = tl2_blocks(K), k3 = 96 * nb, k2 = K - k3;
+    int64_t rb = oracle_tl2_row_bytes(K);
+    int64_t sign_off = 16 * nb, tail_off = sign_off + 16 * ((nb + 3) / 4);
+    for (int64_t m = 0; m < M; ++m) {
+        const int8_t* c = codes + m * K;
+        uint8_t* row = out + m * rb;
+        for (int64_t i = 0; i < rb; ++i) row[i] = 0;
+        for (int64_t k = 0; k < K; ++k)
+            if (c[k] < -1 || c[k] > 1) return -1;
+        for (int64_t b = 0; b < nb; ++b) {
+            uint32_t signs = 0;
+            for (int g = 0; g < 32; ++g) {
+                int64_t k = 96 * b + 3 * g;
+                int s, idx;
+                tl2_encode_group(c[k], c[k + 1], c[k + 2], &s, &idx);
+                row[16 * b + g / 2] |= (uint8_t)(idx << (4 * (g % 2)));
+                signs |= (uint32_t)s << g;
+            }
+            for (int j = 0; j < 4; ++j)
+                row[sign_off + 4 * b + j] = (uint8_t)(signs >> (8 * j));
+        }
+        /* the remainder: the 2-bit layout of oracle_pack, padded with code 0 */
+        int64_t tail_words = 4 * ((k2 + 63) / 64);
+        for (int64_t w = 0; w < tail_words; ++w) {
+            uint32_t word = 0x55555555u;
+            for (int64_t i = 0; i < 16; ++i) {
+                int64_t j = 16 * w + i;
+                if (j >= k2) break;
+                int bit = field_bit(j);
+                word = (word & ~(3u << bit)) | ((uint32_t)(c[k3 + j] + 1) << bit);
+            }
+            for (int j = 0; j < 4; ++j)
+                row[tail_off + 4 * w + j] = (uint8_t)(word >> (8 * j));
+        }
+    }
+    return 0;
+}
+
+int oracle_tl2_decode(const uint8_t* in, int64_t M, int64_t K, int8_t* codes)
+{
+    if (K % 16 != 0 || M < 0) return -1;
+    int64_t nb = tl2_blocks(K), k3 = 96 * nb, k2 = K - k3;
+    int64_t rb = oracle_tl2_row_bytes(K);
+    int64_t sign_off = 16 * nb, tail_off = sign_off + 16 * ((nb + 3) / 4);
+    int bad = 0;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint8_t* row = in + m * rb;
+        int8_t* c = codes + m * K;
+        for (int64_t b = 0; b < nb; ++b) {
+            uint32_t signs = 0;
+            for (int j = 0; j < 4; ++j) signs |= (uint32_t)row[sign_off + 4 * b + j] << (8 * j);
+            for (int g = 0; g < 32; ++g) {
+                int idx = (row[16 * b + g / 2] >> (4 * (g % 2))) & 15;
+                int s = (signs >> g) & 1;
+                if (idx > 13 || (idx == 0 && s)) bad = 1;   /* never written */
+                int d[3];
+                tl2_decode_group(s, idx > 13 ? 0 : idx, d);
+                for (int i = 0; i < 3; ++i) c[96 * b + 3 * g + i] = (int8_t)d[i];
+            }
+        }
+        for (int64_t i = sign_off + 4 * nb; i < tail_off; ++i)
+            if (row[i] != 0) bad = 1;                        /* sign-plane padding */
+        int64_t tail_words = 4 * ((k2 + 63) / 64);
+        for (int64_t w = 0; w < tail_words; ++w) {
+            uint32_t word = 0;
+            for (int j = 0; j < 4; ++j) word |= (uint32_t)row[tail_off + 4 * w + j] << (8 * j);
+            for (int64_t i = 0; i < 16; ++i) {
+                int64_t j = 16 * w + i;
+                uint32_t f = (word >> field_bit(j)) & 3u;
+                if (f == 3u) bad = 1;
+                if (j < k2) c[k3 + j] = (int8_t)((int)f - 1);
+                else if (f != 1u) bad = 1;                   /* padding holds code 0 */
+            }
+        }
+    }
+    return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Activation quantisation: absmax to int8 (reading notes section 2.3 and    */
 /* 4.1: int8 activations).  Per token (one scale per row of x).  The scale   */
 /* s = 127/amax is one fp32 division; the product x*s is rounded half-even   */

@@ -66,6 +66,23 @@ int oracle_pack(const int8_t* codes, int64_t M, int64_t K, uint32_t* packed);
  * is not code 0. */
 int oracle_unpack(const uint32_t* packed, int64_t M, int64_t K, int8_t* codes);
 
+/* TL2-style storage, 5 bits per three weights (defined by this project; the
+ * pages fix the 1-bit sign + 4-bit index split and the 5/3 bits per weight).
+ * Per row, with nb = floor(K/96) blocks of 96 weights and K2 = K - 96*nb:
+ *   bytes [0, 16*nb)        index plane: block b's group g (weights 96b+3g ..
+ *                           96b+3g+2) has its 4-bit index in byte 16b + g/2,
+ *                           low nibble for even g;
+ *   next 16*ceil(nb/4)      sign plane: block b's 32 signs in the
+ *                           little-endian uint32 at 4b (bit g), zero padding;
+ *   next 16*ceil(K2/64)     the last K2 weights in the 2-bit layout of
+ *                           oracle_pack (a K2-wide row, padded with code 0).
+ * A group's v = 9(c0+1) + 3(c1+1) + (c2+1): index |v - 13|, sign (v < 13).
+ * Negating a group's codes flips its sign bit only.  K % 16 == 0. */
+int64_t oracle_tl2_row_bytes(int64_t K);
+int oracle_tl2_encode(const int8_t* codes, int64_t M, int64_t K, uint8_t* out);
+/* Inverse; -1 on an index above 13, a negative zero group, or bad padding. */
+int oracle_tl2_decode(const uint8_t* in, int64_t M, int64_t K, int8_t* codes);
+
 /* Per-token absmax int8 quantisation of x [N,K].  qsum may be NULL. */
 void oracle_quant_act(const float* x, int64_t N, int64_t K,
                       int8_t* q, float* amax, int32_t* qsum);

@@ -429,3 +429,76 @@ def test_seeded_regression_fixture():
     assert out["q"].ravel().tolist() == g["q"]
     assert out["acc"].ravel().tolist() == g["acc"]
     assert out["y"].ravel().tolist() == g["y"]
+
+
+# ----------------------------------------------------------------------------- TL2-style storage
+
+def _tl2_group(c0, c1, c2):
+    """(sign, index) of a group of three codes at the front of a 96-wide row."""
+    codes = np.zeros((1, 96), dtype=np.int8)
+    codes[0, :3] = (c0, c1, c2)
+    row = oracle.tl2_encode(codes)[0]
+    return int(row[16] & 1), int(row[0] & 15)      # sign plane starts after 16 index bytes
+
+
+def test_tl2_mirror_consolidation_and_sign_index_split():
+    # 27 combinations of three ternary weights fold onto 14 indices (4 bits) and
+    # a sign bit: negating every code of a group flips its sign and nothing else
+    import itertools
+    seen = {}
+    for combo in itertools.product((-1, 0, 1), repeat=3):
+        s, i = _tl2_group(*combo)
+        assert 0 <= i <= 13
+        seen[(s, i)] = combo
+        ns, ni = _tl2_group(*[-c for c in combo])
+        if any(combo):
+            assert ni == i and ns == 1 - s, combo
+        else:
+            assert (s, i) == (0, 0) and (ns, ni) == (0, 0)
+    assert len(seen) == 27                                  # one code per combination
+    assert len({i for _, i in seen}) == 14
+
+
+@pytest.mark.parametrize("K", [16, 96, 112, 384, 2560, 6912, 4096, 176])
+def test_tl2_roundtrip_size_and_remainder(K):
+    r = rng(K + 3)
+    M = 4
+    c = r.integers(-1, 2, size=(M, K)).astype(np.int8)
+    t = oracle.tl2_encode(c)
+    nb, k2 = K // 96, K % 96
+    assert t.shape == (M, 16 * nb + 16 * (-(-nb // 4)) + 16 * (-(-k2 // 64)))
+    assert t.shape[1] % 16 == 0
+    assert np.array_equal(oracle.tl2_decode(t, M, K), c)
+    # the remainder (the last K % 96 weights) is the 2-bit layout of oracle.pack
+    if k2:
+        tail = t[:, t.shape[1] - 16 * (-(-k2 // 64)):].copy().view(np.uint32)
+        assert np.array_equal(tail, oracle.pack(c[:, 96 * nb:]))
+
+
+def test_tl2_bits_per_weight_from_the_pages():
+    facts = json.load(open(os.path.join(GOLDEN, "pages_facts.json")))
+    K = 384                        # four whole blocks of 96: no remainder, no padding
+    assert oracle.tl2_row_bytes(K) * 8 / K == pytest.approx(5 / 3, abs=1e-12)
+    assert oracle.tl2_row_bytes(K) * 8 / K == pytest.approx(
+        facts["tl2_bits_per_weight"]["value"], abs=0.005)
+    # the shapes of the 2B model: 6912 = 72 blocks exactly; 2560 keeps a 64-weight remainder
+    assert oracle.tl2_row_bytes(6912) == 6912 * 5 // 3 // 8
+    assert oracle.tl2_row_bytes(2560) == 26 * 16 + 112 + 16
+
+
+def test_tl2_rejects_invalid_rows():
+    c = np.zeros((1, 96), dtype=np.int8)
+    t = oracle.tl2_encode(c)
+    assert not t.any()                           # all-zero codes: index 0, sign 0 everywhere
+    bad = t.copy()
+    bad[0, 0] = 14                               # index above 13
+    with pytest.raises(ValueError):
+        oracle.tl2_decode(bad, 1, 96)
+    bad = t.copy()
+    bad[0, 16] = 1                               # sign on the zero group (negative zero)
+    with pytest.raises(ValueError):
+        oracle.tl2_decode(bad, 1, 96)
+    bad = t.copy()
+    bad[0, 20] = 1                               # sign-plane padding
+    with pytest.raises(ValueError):
+        oracle.tl2_decode(bad, 1, 96)
