@@ -192,6 +192,14 @@ class DecodeWorkload:
         fents = [(packed, alpha, M, K, self._x(l, p), self.ys[l][p], None)
                  for l in range(L) for p, (packed, alpha, M, K) in enumerate(self.weights[l])]
         self.fprob = _lib.make_fused_problems(fents)
+        # the same weights in TL2-style storage (5 bits per three weights)
+        self.tl2 = [[api.tl2_from_packed(packed, K) for (packed, _, _, K) in row]
+                    for row in self.weights]
+        tents = [(self.tl2[l][p], alpha, M, K, self._act(l, p)[0], self._act(l, p)[1],
+                  self.ys[l][p], None)
+                 for l in range(L) for p, (_, alpha, M, K) in enumerate(self.weights[l])]
+        self.tl2prob = _lib.make_tl2_problems(tents)
+        self.tl2_bytes = sum(t.numel() for row in self.tl2 for t in row)
         self.acts = _lib.make_acts([(self.Xh, self.XQh, self.AMh, self.XSh),
                                     (self.Xf, self.XQf, self.AMf, self.XSf)])
         self.packed_bytes = sum(M * K // 4 for row in self.weights for _, _, M, K in row)
@@ -228,6 +236,11 @@ class DecodeWorkload:
         """Quantiser launch, then the GEMV launch."""
         self.quant(s)
         self.gemv(s)
+
+    def gemv_tl2(self, s):
+        """The GEMV launch over the TL2-style copy of the weights."""
+        _lib.check(_lib.bitlinear_gemv_tl2_grouped(self.tl2prob, self.n_prob, 1, s),
+                   "gemv_tl2_grouped")
 
     def step(self, s):
         """The decode path: one fused quantise+GEMV launch over all 210 linears."""
@@ -472,6 +485,21 @@ def run_ours(args, rank, world, local_rank):
         per["quant"] += e[2].elapsed_time(e[3])
         per["gemv"] += e[3].elapsed_time(e[4])
     per = {k: v / K2 for k, v in per.items()}
+    # ---- the TL2-style storage: the GEMV launch alone, events around each
+    K3 = min(K2, 2000)
+    for _ in range(3):
+        dec.gemv_tl2(s)
+    ev = events(2 * K3)
+    for e in ev:
+        e.record(s)
+    torch.cuda.synchronize()
+    for i in range(K3):
+        ev[2 * i].record(s)
+        dec.gemv_tl2(s)
+        ev[2 * i + 1].record(s)
+    torch.cuda.synchronize()
+    per["gemv_tl2"] = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K3)) / K3
+    del ev
     ms_per_step = total_ms / K
     gbs = world * dec.packed_bytes / (ms_per_step * 1e-3) / 1e9
     fused_gbs = dec.alg_bytes_fused / (per["gemv_quant"] * 1e-3) / 1e9
@@ -479,6 +507,9 @@ def run_ours(args, rank, world, local_rank):
     hbm_peak = peaks["hbm_gbs"]
     if args.only == "decode":
         print(json.dumps({"partial_run": "decode", "value": round(gbs, 1), "unit": "GB/s",
+                          "tl2_gemv_ms": round(per["gemv_tl2"], 5),
+                          "tl2_equiv_gbs": round(dec.packed_bytes / (per["gemv_tl2"] * 1e-3)
+                                                 / 1e9, 1),
                           "two_step_gbs": round(dec.packed_bytes / (two_ms * 1e-3) / 1e9, 1),
                           "kernel_ms": per, "gemv_quant_gbs": round(fused_gbs, 1),
                           "gemv_gbs": round(gemv_gbs, 1), "clocks": clk}))
@@ -594,6 +625,16 @@ def run_ours(args, rank, world, local_rank):
                     "traffic": ncu_traffic("gemv"),
                     "traffic_source": NCU_TRAFFIC["gemv"]["profile"]},
             },
+            "tl2_storage": {
+                "what": "the GEMV launch over the same 210 layers stored at 5 bits per three "
+                        "weights (TL2-style), int8 activations from the quantiser",
+                "bytes_per_launch": dec.tl2_bytes,
+                "packed_2bit_bytes": dec.packed_bytes,
+                "avg_launch_ms": round(per["gemv_tl2"], 5),
+                "tl2_bytes_gbs": round(dec.tl2_bytes / (per["gemv_tl2"] * 1e-3) / 1e9, 1),
+                "weights_per_s_as_2bit_gbs": round(dec.packed_bytes / (per["gemv_tl2"] * 1e-3)
+                                                   / 1e9, 1),
+            },
             "decode_chain": {
                 "what": "same 210 linears, per-layer dependent launches, one CUDA graph: fused "
                         "(qkv, o, gate/up, down: 4 launches per layer) and two-step (a quantiser "
@@ -611,7 +652,8 @@ def run_ours(args, rank, world, local_rank):
                     "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": K,
-            "gpu_launches_other_passes": {"two_step": 2 * K, "breakdown": 3 * K2},
+            "gpu_launches_other_passes": {"two_step": 2 * K, "breakdown": 3 * K2,
+                                          "tl2": K3 + 3},
             "clocks": clk,
             "cpu_baseline": cpu,
         }

@@ -276,6 +276,66 @@ BITLINEAR_API bitlinear_status bitlinear_gemv_quant_grouped(
     const bitlinear_fused_problem* problems, int64_t count, int64_t N,
     bitlinear_stream_t stream);
 
+/* --------------------------------------- TL2-style storage, 5/3 bits/weight */
+
+/*
+ * A second storage of the same ternary codes at 5 bits per three weights:
+ * each group of three is folded onto its mirror image and stored as a 1-bit
+ * sign and a 4-bit index, and K is split into a part stored in groups of
+ * three and a remainder (reading notes section 2.3 "technical details":
+ * signed-unsigned weight splitting, block-fitting weight splitting; 1.67
+ * bits per weight).  It moves 1/6 fewer weight bytes than the 2-bit layout.
+ * Row layout (this library's own; rows contiguous, each 16-byte aligned):
+ *   [0, 16*nb)            index plane, nb = floor(K/96) blocks of 96 weights:
+ *                         group g of block b (weights 96b+3g .. 96b+3g+2) has
+ *                         its index in byte 16b + g/2, low nibble for even g
+ *   [16*nb, +16*ceil(nb/4))  sign plane: uint32 per block, bit g; zero padding
+ *   then 16*ceil(K2/64)   the last K2 = K - 96*nb weights in the 2-bit layout
+ *                         above (a K2-wide row, padded with code 0)
+ * For codes (c0,c1,c2) let v = 9(c0+1) + 3(c1+1) + (c2+1) in [0, 26]: the
+ * index is |v - 13| and the sign is (v < 13).
+ */
+
+/* Bytes of one TL2 row for K (a multiple of 16, at most 131072), else 0. */
+BITLINEAR_API size_t bitlinear_tl2_row_bytes(int64_t K);
+
+/*
+ * Re-encode packed 2-bit weights [M, WP(K)] (from bitlinear_pack_weights) as
+ * TL2 rows: tl2 receives M * bitlinear_tl2_row_bytes(K) bytes.  alpha is
+ * unchanged and is used with either storage.
+ */
+BITLINEAR_API bitlinear_status bitlinear_tl2_from_packed(const uint32_t* packed, int64_t M,
+                                                         int64_t K, uint8_t* tl2,
+                                                         bitlinear_stream_t stream);
+
+/*
+ * Decode GEMV (1 <= N <= 16) over TL2 rows: the results of bitlinear_gemv
+ * (y, and acc when non-NULL) for the same codes and activations.  xq and
+ * amax come from a quantiser call; the activation sum is not needed.
+ */
+BITLINEAR_API bitlinear_status bitlinear_gemv_tl2(const uint8_t* tl2, const float* alpha,
+                                                  int64_t M, int64_t K, const int8_t* xq,
+                                                  const float* amax, int64_t N, float* y,
+                                                  int32_t* acc, bitlinear_stream_t stream);
+
+/* One layer of a grouped TL2 call. */
+typedef struct {
+    const uint8_t* tl2;       /* [M, bitlinear_tl2_row_bytes(K)] bytes */
+    const float* alpha;       /* [1] */
+    int64_t M;
+    int64_t K;
+    const int8_t* xq;         /* [N, K] */
+    const float* amax;        /* [N] */
+    float* y;                 /* [N, M] output */
+    int32_t* acc;             /* [N, M] output, or NULL */
+} bitlinear_tl2_problem;
+
+/* bitlinear_gemv_tl2 over a list of layers, one launch per 256 layers;
+ * `problems` is a HOST array read during the call only. */
+BITLINEAR_API bitlinear_status bitlinear_gemv_tl2_grouped(const bitlinear_tl2_problem* problems,
+                                                          int64_t count, int64_t N,
+                                                          bitlinear_stream_t stream);
+
 /* ------------------------------------------------- weights, no allocation */
 
 /*

@@ -41,6 +41,13 @@ class FusedProblem(ctypes.Structure):
                 ("acc", ctypes.c_void_p)]
 
 
+class Tl2Problem(ctypes.Structure):
+    """Mirror of bitlinear_tl2_problem (include/bitlinear.h)."""
+    _fields_ = [("tl2", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("M", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("xq", ctypes.c_void_p), ("amax", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("acc", ctypes.c_void_p)]
+
+
 class BitLinearError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -90,6 +97,14 @@ def load(path: str = LIB_PATH):
     L.bitlinear_gemv_quant.restype = st
     L.bitlinear_gemv_quant_grouped.argtypes = [ctypes.POINTER(FusedProblem), i64, i64, p]
     L.bitlinear_gemv_quant_grouped.restype = st
+    L.bitlinear_tl2_row_bytes.argtypes = [i64]
+    L.bitlinear_tl2_row_bytes.restype = sz
+    L.bitlinear_tl2_from_packed.argtypes = [p, i64, i64, p, p]
+    L.bitlinear_tl2_from_packed.restype = st
+    L.bitlinear_gemv_tl2.argtypes = [p, p, i64, i64, p, p, i64, p, p, p]
+    L.bitlinear_gemv_tl2.restype = st
+    L.bitlinear_gemv_tl2_grouped.argtypes = [ctypes.POINTER(Tl2Problem), i64, i64, p]
+    L.bitlinear_gemv_tl2_grouped.restype = st
     L.bitlinear_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
     L.bitlinear_device_error.restype = st
     _lib = L
@@ -216,6 +231,31 @@ def make_fused_problems(entries):
 def bitlinear_gemv_quant_grouped(problems, count, N, stream=None):
     """problems: a ctypes array from make_fused_problems()."""
     return load().bitlinear_gemv_quant_grouped(problems, count, N, _stream(stream))
+
+
+def bitlinear_tl2_from_packed(packed, M, K, tl2, stream=None):
+    return load().bitlinear_tl2_from_packed(_p(packed), M, K, _p(tl2), _stream(stream))
+
+
+def bitlinear_gemv_tl2(tl2, alpha, M, K, xq, amax, N, y, acc=None, stream=None):
+    return load().bitlinear_gemv_tl2(_p(tl2), _p(alpha), M, K, _p(xq), _p(amax), N, _p(y),
+                                     _p(acc), _stream(stream))
+
+
+def make_tl2_problems(entries):
+    """entries: iterable of (tl2, alpha, M, K, xq, amax, y, acc-or-None); tensors
+    for the pointers.  Returns a ctypes array of Tl2Problem."""
+    entries = list(entries)
+    arr = (Tl2Problem * max(1, len(entries)))()
+    for i, (tl2, alpha, M, K, xq, amax, y, acc) in enumerate(entries):
+        arr[i] = Tl2Problem(tl2.data_ptr(), alpha.data_ptr(), M, K, xq.data_ptr(),
+                            amax.data_ptr(), y.data_ptr(), 0 if acc is None else acc.data_ptr())
+    return arr
+
+
+def bitlinear_gemv_tl2_grouped(problems, count, N, stream=None):
+    """problems: a ctypes array from make_tl2_problems()."""
+    return load().bitlinear_gemv_tl2_grouped(problems, count, N, _stream(stream))
 
 
 def bitlinear_pack_workspace_bytes(M, K):

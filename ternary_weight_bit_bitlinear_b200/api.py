@@ -225,6 +225,44 @@ def gemv_quant_grouped(layers, x, with_acc=False, stream=None, outs=None):
     return (ys, accs) if with_acc else ys
 
 
+def tl2_row_bytes(K):
+    """Bytes of one TL2-style row (5 bits per three weights, see include/bitlinear.h)."""
+    n = _lib.load().bitlinear_tl2_row_bytes(int(K))
+    if n == 0:
+        raise ValueError("K must be a positive multiple of 16, at most 131072")
+    return n
+
+
+def tl2_from_packed(packed, K, stream=None):
+    """Re-encode 2-bit packed weights [M, packed_row_words(K)] as TL2-style
+    rows: uint8 [M, tl2_row_bytes(K)]."""
+    _need(packed, torch.int32, "packed")
+    M = packed.shape[0]
+    if packed.shape[1] != packed_row_words(K):
+        raise ValueError("packed must be [M, packed_row_words(K)]")
+    out = torch.empty((M, tl2_row_bytes(K)), dtype=torch.uint8, device=packed.device)
+    _lib.check(_lib.bitlinear_tl2_from_packed(packed, M, K, out, stream),
+               "bitlinear_tl2_from_packed")
+    return out
+
+
+def gemv_tl2(tl2, alpha, xq, amax, M=None, with_acc=False, stream=None, out=None):
+    """Decode GEMV over TL2-style rows (N <= 16): same y (and acc) as gemv."""
+    _need(tl2, torch.uint8, "tl2")
+    _need(alpha, torch.float32, "alpha")
+    _need(xq, torch.int8, "xq")
+    _need(amax, torch.float32, "amax")
+    M = tl2.shape[0] if M is None else M
+    N, K = xq.shape
+    if tl2.shape != (M, tl2_row_bytes(K)):
+        raise ValueError("tl2 must be [M, tl2_row_bytes(K)] = [%d, %d]" % (M, tl2_row_bytes(K)))
+    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=xq.device)
+    acc = torch.empty((N, M), dtype=torch.int32, device=xq.device) if with_acc else None
+    _lib.check(_lib.bitlinear_gemv_tl2(tl2, alpha, M, K, xq, amax, N, y, acc, stream),
+               "bitlinear_gemv_tl2")
+    return (y, acc) if with_acc else y
+
+
 class TernaryLinear:
     """A BitLinear layer: packed 2-bit ternary weights + alpha, applied to fp32
     activations: the fused quantise+GEMV kernel for a few tokens, else

@@ -16,6 +16,7 @@
 #include "gemv_quant.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
+#include "tl2.cuh"
 
 namespace {
 
@@ -62,6 +63,7 @@ struct DeviceInfo {
   int sms = 0;
   bool gemm_attr_set[2] = {false, false};
   int gemv_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};   // 0: not set up yet
+  int tl2_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};    // 0: not set up yet
   bool gq_attr_set[bl::kGemvMaxTokens + 1] = {};
   int gq_smem[bl::kGemvMaxTokens + 1] = {};               // last shared-memory size seen
   int gq_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};      // and its occupancy
@@ -520,6 +522,95 @@ bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t 
   return BITLINEAR_OK;
 }
 
+// ---- TL2-style storage
+
+bitlinear_status check_tl2_problem(const bitlinear_tl2_problem& q, int64_t N) {
+  bitlinear_status st = check_mk(q.M, q.K);
+  if (st != BITLINEAR_OK) return st;
+  if (!q.tl2 || !q.alpha || !q.xq || !q.amax || !q.y) return BITLINEAR_ERR_INVALID_ARG;
+  if (!aligned16(q.tl2) || !aligned16(q.xq) || !aligned16(q.y) || (q.acc && !aligned16(q.acc)))
+    return BITLINEAR_ERR_MISALIGNED;
+  if (!aligned4(q.alpha) || !aligned4(q.amax)) return BITLINEAR_ERR_MISALIGNED;
+  (void)N;
+  return BITLINEAR_OK;
+}
+
+template <int NT>
+bitlinear_status launch_gemv_tl2(const bl::Tl2Params& p, DeviceInfo* dev, cudaStream_t s) {
+  auto kernel = bl::gemv_tl2_kernel<NT>;
+  constexpr int smem = bl::Tl2Cfg<NT>::kSmemBytes;
+  int& per_sm = dev->tl2_blocks_per_sm[NT];
+  if (per_sm == 0) {
+    int nb = 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, bl::kTl2Threads, smem) !=
+            cudaSuccess ||
+        nb < 1)
+      return BITLINEAR_ERR_CUDA;
+    per_sm = nb;
+  }
+  const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm * bl::kTl2Warps;
+  const int64_t upw = (p.total_units + cap - 1) / cap;
+  const int64_t warps = (p.total_units + upw - 1) / upw;
+  const int grid = static_cast<int>((warps + bl::kTl2Warps - 1) / bl::kTl2Warps);
+  if (launch_pdl(kernel, grid, bl::kTl2Threads, smem, s, p) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  return launch_status();
+}
+
+bitlinear_status launch_gemv_tl2_n(int N, const bl::Tl2Params& p, DeviceInfo* dev,
+                                   cudaStream_t s) {
+  switch (N) {
+#define BL_TL2_CASE(n) \
+  case n: return launch_gemv_tl2<n>(p, dev, s);
+    BL_TL2_CASE(1) BL_TL2_CASE(2) BL_TL2_CASE(3) BL_TL2_CASE(4)
+    BL_TL2_CASE(5) BL_TL2_CASE(6) BL_TL2_CASE(7) BL_TL2_CASE(8)
+    BL_TL2_CASE(9) BL_TL2_CASE(10) BL_TL2_CASE(11) BL_TL2_CASE(12)
+    BL_TL2_CASE(13) BL_TL2_CASE(14) BL_TL2_CASE(15) BL_TL2_CASE(16)
+#undef BL_TL2_CASE
+    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
+bitlinear_status gemv_tl2_group(const bitlinear_tl2_problem* probs, int64_t count, int64_t N,
+                                cudaStream_t s) {
+  DeviceInfo* dev = nullptr;
+  bitlinear_status st = device_info(&dev);
+  if (st != BITLINEAR_OK) return st;
+  for (int64_t base = 0; base < count; base += bl::kTl2MaxProblems) {
+    const int n = static_cast<int>(count - base < bl::kTl2MaxProblems
+                                       ? count - base : bl::kTl2MaxProblems);
+    bl::Tl2Params p;
+    memset(&p, 0, sizeof p);
+    int64_t units = 0;
+    for (int i = 0; i < n; ++i) {
+      const bitlinear_tl2_problem& q = probs[base + i];
+      bl::Tl2Problem& g = p.prob[i];
+      g.tl2 = q.tl2;
+      g.alpha = q.alpha;
+      g.xq = q.xq;
+      g.amax = q.amax;
+      g.y = q.y;
+      g.acc = q.acc;
+      g.M = static_cast<int>(q.M);
+      g.K = static_cast<int>(q.K);
+      g.nb = static_cast<int>(bl::tl2_blocks(q.K));
+      g.row_bytes = static_cast<int>(bl::tl2_row_bytes(q.K));
+      g.sign_off = static_cast<int>(bl::tl2_sign_offset(q.K));
+      g.tail_off = static_cast<int>(bl::tl2_tail_offset(q.K));
+      g.unit_begin = static_cast<int>(units);
+      units += (q.M + bl::kGemvTileRows - 1) / bl::kGemvTileRows;
+    }
+    if (units > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+    p.num_problems = n;
+    p.total_units = static_cast<int>(units);
+    st = launch_gemv_tl2_n(static_cast<int>(N), p, dev, s);
+    if (st != BITLINEAR_OK) return st;
+  }
+  return BITLINEAR_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -733,6 +824,52 @@ bitlinear_status bitlinear_gemv_quant_grouped(const bitlinear_fused_problem* pro
     if (st != BITLINEAR_OK) return st;
   }
   return gemv_quant_group(problems, count, N, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t bitlinear_tl2_row_bytes(int64_t K) {
+  if (K <= 0 || K % 16 != 0 || K > kMaxK) return 0;
+  return static_cast<size_t>(bl::tl2_row_bytes(K));
+}
+
+bitlinear_status bitlinear_tl2_from_packed(const uint32_t* packed, int64_t M, int64_t K,
+                                           uint8_t* tl2, bitlinear_stream_t stream) {
+  bitlinear_status st = check_mk(M, K);
+  if (st != BITLINEAR_OK) return st;
+  if (!packed || !tl2) return BITLINEAR_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(tl2)) return BITLINEAR_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != BITLINEAR_OK) return st;
+  const int64_t nb = bl::tl2_blocks(K);
+  const int64_t total = M * (nb + (K - bl::kTl2Block * nb + 63) / 64);
+  int64_t g = (total + 255) / 256;
+  if (g > dev->sms * 16) g = dev->sms * 16;
+  bl::tl2_convert_kernel<<<static_cast<int>(g), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      packed, M, K, static_cast<int>(packed_row_words(K)), tl2);
+  return launch_status();
+}
+
+bitlinear_status bitlinear_gemv_tl2(const uint8_t* tl2, const float* alpha, int64_t M, int64_t K,
+                                    const int8_t* xq, const float* amax, int64_t N, float* y,
+                                    int32_t* acc, bitlinear_stream_t stream) {
+  if (N < 0) return BITLINEAR_ERR_INVALID_ARG;
+  if (N > bl::kGemvMaxTokens) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  const bitlinear_tl2_problem q = {tl2, alpha, M, K, xq, amax, y, acc};
+  if (N == 0) return check_mk(M, K);
+  bitlinear_status st = check_tl2_problem(q, N);
+  if (st != BITLINEAR_OK) return st;
+  return gemv_tl2_group(&q, 1, N, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitlinear_status bitlinear_gemv_tl2_grouped(const bitlinear_tl2_problem* problems, int64_t count,
+                                            int64_t N, bitlinear_stream_t stream) {
+  if (count < 0 || N < 0 || (count > 0 && !problems)) return BITLINEAR_ERR_INVALID_ARG;
+  if (count == 0 || N == 0) return BITLINEAR_OK;
+  if (N > bl::kGemvMaxTokens) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  for (int64_t i = 0; i < count; ++i) {
+    bitlinear_status st = check_tl2_problem(problems[i], N);
+    if (st != BITLINEAR_OK) return st;
+  }
+  return gemv_tl2_group(problems, count, N, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bitlinear_status bitlinear_device_error(int* status_out, int clear) {

@@ -233,3 +233,38 @@ def test_gemv_quant_grouped_argument_errors(L):
     assert f((P * 2)(good, prob(x=MISALIGNED)), 2, 1, None) == _lib.ERR_MISALIGNED
     assert f((P * 2)(good, prob(x=0)), 2, 1, None) == _lib.ERR_INVALID_ARG
     assert f((P * 2)(good, prob(alpha=FAKE + 2)), 2, 1, None) == _lib.ERR_MISALIGNED
+
+
+def test_tl2_argument_errors(L):
+    assert L.bitlinear_tl2_row_bytes(384) == 80
+    assert L.bitlinear_tl2_row_bytes(6912) == 1440
+    assert L.bitlinear_tl2_row_bytes(40) == 0 and L.bitlinear_tl2_row_bytes(0) == 0
+    f = L.bitlinear_tl2_from_packed
+    assert f(_p(FAKE), 4, 40, _p(FAKE), None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert f(_p(0), 4, 96, _p(FAKE), None) == _lib.ERR_INVALID_ARG
+    assert f(_p(FAKE), 4, 96, _p(MISALIGNED), None) == _lib.ERR_MISALIGNED
+    assert f(_p(FAKE), -1, 96, _p(FAKE), None) == _lib.ERR_INVALID_ARG
+    g = L.bitlinear_gemv_tl2
+    ok = dict(tl2=FAKE, alpha=FAKE, M=64, K=192, xq=FAKE, amax=FAKE, N=1, y=FAKE, acc=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(_p(a["tl2"]), _p(a["alpha"]), a["M"], a["K"], _p(a["xq"]), _p(a["amax"]),
+                 a["N"], _p(a["y"]), _p(a["acc"]), None)
+
+    assert call(N=0) == _lib.OK
+    assert call(N=17) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(N=-1) == _lib.ERR_INVALID_ARG
+    assert call(K=40) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert call(tl2=0) == _lib.ERR_INVALID_ARG
+    assert call(amax=0) == _lib.ERR_INVALID_ARG
+    assert call(tl2=MISALIGNED) == _lib.ERR_MISALIGNED
+    assert call(amax=FAKE + 2) == _lib.ERR_MISALIGNED
+    P = _lib.Tl2Problem
+    good = P(FAKE, FAKE, 64, 192, FAKE, FAKE, FAKE, 0)
+    G = L.bitlinear_gemv_tl2_grouped
+    assert G((P * 1)(good), 0, 1, None) == _lib.OK
+    assert G((P * 1)(good), 1, 17, None) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert G(None, 1, 1, None) == _lib.ERR_INVALID_ARG
+    assert G((P * 2)(good, P(FAKE, FAKE, 64, 40, FAKE, FAKE, FAKE, 0)), 2, 1, None) == \
+        _lib.ERR_UNSUPPORTED_SHAPE

@@ -141,6 +141,30 @@ def test_config2_2b_decode_stream_fused_quant():
         assert torch.equal(ys[k], ref[k]), k
 
 
+def test_config2_2b_decode_stream_tl2_storage():
+    # the same 30-layer stream re-encoded at 5/3 bits per weight: every output
+    # equals the 2-bit path's, and sampled rows equal the oracle's
+    m = Model(2, 30, 1)
+    ref = m.run_gemv()
+    lst = m.layer_list()
+    tl2 = {k: api.tl2_from_packed(m.w[k][0], m.shape.projections()[k[1]][2]) for k in lst}
+    ents, ys = [], {}
+    for l, p in lst:
+        _, M, K = m.shape.projections()[p]
+        xq, amax, _ = m.q[(l, _input_proj(p))]
+        ys[(l, p)] = torch.empty((1, M), device="cuda")
+        ents.append((tl2[(l, p)], m.w[(l, p)][1], M, K, xq, amax, ys[(l, p)], None))
+    arr = _lib.make_tl2_problems(ents)
+    assert _lib.bitlinear_gemv_tl2_grouped(arr, len(ents), 1, None) == _lib.OK
+    assert sum(t.numel() for t in tl2.values()) * 6 < sum(
+        m.w[k][0].numel() * 4 for k in lst) * 5.2     # about 1/6 fewer bytes
+    for (l, p) in [(0, 0), (9, 4), (29, 6)]:
+        M = m.shape.projections()[p][1]
+        m.check(l, p, ys[(l, p)], _rows(M, 30, 7 * l + p), [0])
+    for k in lst:
+        assert torch.equal(ys[k], ref[k]), k
+
+
 def test_config3_7b_prefill_512_grouped():
     m = Model(3, 1, 512)
     ys = m.run_gemm(0)
