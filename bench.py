@@ -52,10 +52,10 @@ INT8_PER_BF16 = 2.0          # nominal dense int8 : bf16 tensor throughput (4.5 
 # the figure no longer applies and the bench reports null.
 NCU_TRAFFIC = {
     "gemv": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemv.cuh",
-             "sha256": "f891fc3c908a67f0", "bytes": 522_180_608 + 5_733_888,
-             "profile": "profiles/gemv_tile_2b_decode_stream.md"},
+             "sha256": "d0ffe60ca94b9a32", "bytes": 522_076_623 + 2_235_136,
+             "profile": "profiles/launches_decode_2b.md"},
     "gemv_quant": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemv_quant.cuh",
-                   "sha256": "", "bytes": None,
+                   "sha256": "cad4236b5fa00ff6", "bytes": 523_105_877 + 2_638_464,
                    "profile": "profiles/gemv_quant_2b_decode_stream.md"},
     "gemm": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
              "sha256": "7a558782e6ea35ab", "bytes": 62_585_600 + 31_000_064,
