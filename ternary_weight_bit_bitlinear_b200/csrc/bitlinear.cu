@@ -12,6 +12,7 @@
 
 #include "bitlinear.h"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "gemv.cuh"
 #include "gemv_quant.cuh"
 #include "pack.cuh"
@@ -223,6 +224,24 @@ bitlinear_status launch_gemm(const bl::GemmParams& p, DeviceInfo* dev, int slot,
   return launch_status();
 }
 
+// CTA-pair GEMM for wide token blocks: two CTAs (a compile-time cluster) per
+// 256 x 256 tile, one pair per two SMs.
+template <int STAGES>
+bitlinear_status launch_gemm_pair(const bl::GemmParams& p, DeviceInfo* dev, cudaStream_t s) {
+  auto kernel = bl::gemm_i8_pair_kernel<STAGES>;
+  const int smem = static_cast<int>(sizeof(bl::GemmPairSmem<STAGES>)) + 1024;
+  if (!dev->gemm_attr_set[1]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    dev->gemm_attr_set[1] = true;
+  }
+  const int pairs = p.total_tiles < dev->sms / 2 ? p.total_tiles : dev->sms / 2;
+  if (launch_pdl(kernel, 2 * pairs, bl::kGemmThreads, smem, s, p) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  return launch_status();
+}
+
 bitlinear_status check_matmul_args(const uint32_t* packed, const float* alpha, int64_t M,
                                    int64_t K, const int8_t* xq, const float* amax,
                                    const int32_t* xsum, int64_t N, float* y, int32_t* acc) {
@@ -290,8 +309,9 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
   DeviceInfo* dev = nullptr;
   bitlinear_status st = device_info(&dev);
   if (st != BITLINEAR_OK) return st;
-  const bool wide = N > 128;
-  const int BN = wide ? 256 : 128;
+  const bool wide = N > 128;   // 256-token tiles on CTA pairs, else 128-token tiles per CTA
+  const int BN = wide ? bl::kPairBN : 128;
+  const int BMt = wide ? bl::kPairBM : bl::kGemmBM;
   const int64_t n_tiles = (N + BN - 1) / BN;
   for (int64_t base = 0; base < count; base += bl::kGemmMaxProblems) {
     const int n = static_cast<int>(count - base < bl::kGemmMaxProblems
@@ -314,7 +334,7 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
                         static_cast<uint64_t>(q.M), bl::kGemmPackedRowBytes, bl::kGemmBM,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
           !encode_u8_2d(&p.tmB[i], q.xq, static_cast<uint64_t>(q.K), static_cast<uint64_t>(N),
-                        bl::kGemmBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                        bl::kGemmBK, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||   // 128 tokens per box
           (!direct && !encode_f32_2d(&p.tmY[i], q.y, static_cast<uint64_t>(q.M),
                                      static_cast<uint64_t>(N), 32, 32)))
         return BITLINEAR_ERR_CUDA;
@@ -330,13 +350,13 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
       g.n_tiles = static_cast<int>(n_tiles);
       g.tile_begin = static_cast<int>(tiles);
       g.direct_store = direct ? 1 : 0;
-      tiles += (q.M + bl::kGemmBM - 1) / bl::kGemmBM * n_tiles;
+      tiles += (q.M + BMt - 1) / BMt * n_tiles;
     }
     if (tiles > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     p.num_problems = n;
     p.total_tiles = static_cast<int>(tiles);
-    build_gemm_schedule(p, dev->sms);
-    st = wide ? launch_gemm<256, 4>(p, dev, 1, s) : launch_gemm<128, 7>(p, dev, 0, s);
+    build_gemm_schedule(p, wide ? dev->sms / 2 : dev->sms);
+    st = wide ? launch_gemm_pair<5>(p, dev, s) : launch_gemm<128, 7>(p, dev, 0, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;

@@ -66,16 +66,23 @@ struct GemmParams {
   uint16_t sched[kGemmMaxSched];
 };
 
+// Tiles of worker `who` out of `nwho` (a CTA, or a CTA pair).
+__device__ __forceinline__ int gemm_my_count(const GemmParams& p, int who, int nwho) {
+  if (p.use_sched) return p.sched_begin[who + 1] - p.sched_begin[who];
+  return who < p.total_tiles ? (p.total_tiles - 1 - who) / nwho + 1 : 0;
+}
+
+__device__ __forceinline__ int gemm_my_tile(const GemmParams& p, int who, int nwho, int i) {
+  if (p.use_sched) return p.sched[p.sched_begin[who] + i];
+  return who + i * nwho;
+}
+
 __device__ __forceinline__ int gemm_my_count(const GemmParams& p) {
-  if (p.use_sched) return p.sched_begin[blockIdx.x + 1] - p.sched_begin[blockIdx.x];
-  return static_cast<int>(blockIdx.x) < p.total_tiles
-             ? (p.total_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
-             : 0;
+  return gemm_my_count(p, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
 }
 
 __device__ __forceinline__ int gemm_my_tile(const GemmParams& p, int i) {
-  if (p.use_sched) return p.sched[p.sched_begin[blockIdx.x] + i];
-  return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+  return gemm_my_tile(p, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), i);
 }
 
 template <int BN, int STAGES>
@@ -88,7 +95,7 @@ struct GemmSmem {
   float ep_out[kGemmEpiWarps][32 * 32];   // per epilogue warp: one 32 (n) x 32 (m) block
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t ufull[kGemmUnpackBufs];    // unpacked tile ready (128 arrivals)
+  uint64_t ufull[kGemmUnpackBufs];    // unpacked tile ready (one arrival per unpack warp)
   uint64_t uempty[kGemmUnpackBufs];   // unpacked tile consumed by the MMAs (commit)
   uint64_t tfull[2];
   uint64_t tempty[2];
@@ -131,12 +138,12 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < kGemmUnpackBufs; ++i) {
-      mbar_init(&s.ufull[i], 128);
+      mbar_init(&s.ufull[i], 4);                   // one arrival per unpack warp
       mbar_init(&s.uempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], kGemmEpiWarps * 32);
+      mbar_init(&s.tempty[i], kGemmEpiWarps);      // one arrival per epilogue warp
     }
     mbar_init(&s.drain, 1);
     s.abort = 0;
@@ -253,8 +260,9 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
           v.w = (w >> 6) & 0x03030303u;
           *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(j) ^ sw) << 4)) = v;
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&s.ufull[ub]);
+        fence_proxy_async_smem();   // each thread's stores, before the warp's one arrival
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.ufull[ub]);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         if (++ub == kGemmUnpackBufs) { ub = 0; uphase ^= 1u; }
       }
@@ -340,7 +348,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         }
       }
       tc_fence_before();
-      mbar_arrive(&s.tempty[ab]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.tempty[ab]);
     }
     if (lane == 0) bulk_wait_group<0>();   // outputs written before the CTA retires
   }
