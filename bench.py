@@ -57,9 +57,10 @@ NCU_TRAFFIC = {
     "gemv_quant": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemv_quant.cuh",
                    "sha256": "cad4236b5fa00ff6", "bytes": 523_105_877 + 2_638_464,
                    "profile": "profiles/gemv_quant_2b_decode_stream.md"},
-    "gemm": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
-             "sha256": "7a558782e6ea35ab", "bytes": 62_585_600 + 31_000_064,
-             "profile": "profiles/gemm_i8_tcgen05_7b_prefill.md"},
+    "gemm": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
+                      "ternary_weight_bit_bitlinear_b200/csrc/gemm_pair.cuh"],
+             "sha256": "b998379b52960f46", "bytes": 62_609_152 + 31_356_416,
+             "profile": "profiles/gemm_i8_pair_7b_prefill.md"},
 }
 
 
@@ -68,9 +69,13 @@ def ncu_traffic(kernel):
     ent = NCU_TRAFFIC.get(kernel)
     if not ent:
         return None
-    with open(os.path.join(ROOT, ent["file"]), "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest()[:16] != ent["sha256"]:
-            return None
+    files = ent["file"] if isinstance(ent["file"], list) else [ent["file"]]
+    h = hashlib.sha256()
+    for name in files:   # the kernel's sources, hashed in order
+        with open(os.path.join(ROOT, name), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != ent["sha256"]:
+        return None
     return ent["bytes"]
 
 
@@ -380,7 +385,7 @@ def measure_prefill(dev, s, peaks, K):
         "gemm_ms": round(gemm_ms, 4), "quant_ms": round(quant_ms, 4),
         "step_tops_incl_quant": round(pre.flops / ((gemm_ms + quant_ms) * 1e-3) / 1e12, 1),
         "per_projection_ms_separate_launches": [round(v / P, 4) for v in per_proj],
-        "roofline": {"bound": "tensor", "kernel": "gemm_i8_tcgen05 (grouped, 7 layers)",
+        "roofline": {"bound": "tensor", "kernel": "gemm_i8_pair (CTA pairs, grouped, 7 layers)",
                      "achieved": round(tops, 1), "peak": round(int8_peak, 1),
                      "unit": "TOPS", "frac": round(tops / int8_peak, 4),
                      "peak_note": "int8 peak = measured bf16 burst x nominal int8:bf16 ratio 2 (%s)"
