@@ -413,6 +413,24 @@ def measure_prefill(dev, s, peaks, K):
     return prefill
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_max(v, dist=None, device="cpu"):
+    """The maximum of v over the ranks of the process group (v without one).
+    Every rank must call it at the same point."""
+    if dist is None:
+        return v
+    t = torch.tensor([float(v)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def whole_job_gbs(world, bytes_per_rank_step, ms_per_step):
+    """Replicas: every rank streams the same bytes per step; the job's rate is
+    all ranks' bytes over the slowest rank's step time."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -432,11 +450,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return t.item()
+        return rank_max(v, dist, dev)
 
     if args.only == "prefill":
         print(json.dumps({"partial_run": "prefill", "prefill": measure_prefill(dev, s, peaks,
@@ -520,7 +534,7 @@ def run_ours(args, rank, world, local_rank):
     per["gemv_tl2"] = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(K3)) / K3
     del ev
     ms_per_step = total_ms / K
-    gbs = world * dec.packed_bytes / (ms_per_step * 1e-3) / 1e9
+    gbs = whole_job_gbs(world, dec.packed_bytes, ms_per_step)
     fused_gbs = dec.alg_bytes_fused / (per["gemv_quant"] * 1e-3) / 1e9
     gemv_gbs = dec.alg_bytes / (per["gemv"] * 1e-3) / 1e9
     hbm_peak = peaks["hbm_gbs"]
@@ -663,7 +677,7 @@ def run_ours(args, rank, world, local_rank):
             "two_step": {
                 "what": "the same step as two launches: grouped quantiser, then grouped GEMV",
                 "ms_per_step": round(two_ms, 5),
-                "gbs": round(world * dec.packed_bytes / (two_ms * 1e-3) / 1e9, 1),
+                "gbs": round(whole_job_gbs(world, dec.packed_bytes, two_ms), 1),
                 "gemv_roofline": {
                     "achieved": round(gemv_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                     "frac": round(gemv_gbs / hbm_peak, 4), "bytes_per_launch": dec.alg_bytes,
@@ -694,7 +708,7 @@ def run_ours(args, rank, world, local_rank):
                 "two_step_launches_per_step": 8 * dec.layers,
             },
             "prefill": prefill,
-            "e2e": {"value": round(world * dec.packed_bytes / (e2e_ms * 1e-3) / 1e9, 1),
+            "e2e": {"value": round(whole_job_gbs(world, dec.packed_bytes, e2e_ms), 1),
                     "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "how": "per step: pinned host -> device copy of the fp32 inputs, one fused "
