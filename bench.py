@@ -42,6 +42,7 @@ from ternary_weight_bit_bitlinear_b200 import _lib, api, inputs  # noqa: E402
 METRIC = "ternary BitLinear GB/s (% HBM peak) at N=1; int8 TOPS (% peak) at N=512"
 DECODE_CFG = 2
 PREFILL_CFG = 3
+SWEEP_CFG = 4
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "source": "fallback"}
 INT8_PER_BF16 = 2.0          # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
@@ -413,6 +414,67 @@ def measure_prefill(dev, s, peaks, K):
     return prefill
 
 
+def measure_crossover(dev, s, reps=30):
+    """The 8B-shaped batch sweep on one layer (7 projections, one grouped launch
+    per path): the CUDA-core GEMV (N <= 16) against the tensor-core GEMM, with
+    L2 flushed before every timed launch.  Locates the GEMV -> GEMM crossover."""
+    wl = inputs.WORKLOADS[SWEEP_CFG]
+    layers = []
+    for p, (name, M, K) in enumerate(wl.model.projections()):
+        W = inputs.latent_weights(M, K, inputs.weight_seed(SWEEP_CFG, 0, p), device=dev)
+        layers.append(api.pack_weights(W) + (M, K))
+        del W
+    packed_bytes = sum(M * K // 4 for (_, _, M, K) in layers)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = {"workload": "8B-shaped layer (q 4096x4096, k/v 1024x4096, o 4096x4096, gate/up "
+                       "14336x4096, down 4096x14336), 7 projections per grouped launch",
+           "N": [], "gemv_us": [], "gemm_us": [], "gemv_gbs": [], "gemm_tops": []}
+    for N in wl.tokens:
+        xs = {}
+        for p in (0, 3, 4, 6):
+            K = wl.model.ffn if p == 6 else wl.model.hidden
+            x = inputs.activations(N, K, inputs.act_seed(SWEEP_CFG, 0, p), device=dev,
+                                   outlier_frac=wl.outlier_frac)
+            xs[p] = api.quant_act(x)
+        src = [0, 0, 0, 3, 4, 4, 6]
+        ents = []
+        for p, (packed, alpha, M, K) in enumerate(layers):
+            xq, am, xsum = xs[src[p]]
+            ents.append((packed, alpha, M, K, xq, am, xsum,
+                         torch.empty((N, M), device=dev), None))
+        prob = _lib.make_problems(ents)
+        res = {}
+        for path, fn in (("gemv", _lib.bitlinear_gemv_grouped), ("gemm", _lib.bitlinear_gemm_grouped)):
+            if path == "gemv" and N > api.GEMV_MAX_TOKENS:
+                res[path] = None
+                continue
+            for _ in range(3):
+                _lib.check(fn(prob, len(ents), N, s), path)
+            tot = 0.0
+            for _ in range(reps):
+                flush_l2(flush)
+                a, b = events(2)
+                a.record(s)
+                _lib.check(fn(prob, len(ents), N, s), path)
+                b.record(s)
+                torch.cuda.synchronize()
+                tot += a.elapsed_time(b)
+            res[path] = tot / reps
+        flops = sum(2 * M * N * K for (_, _, M, K) in layers)
+        out["N"].append(N)
+        out["gemv_us"].append(None if res["gemv"] is None else round(res["gemv"] * 1e3, 2))
+        out["gemm_us"].append(round(res["gemm"] * 1e3, 2))
+        out["gemv_gbs"].append(None if res["gemv"] is None else
+                               round(packed_bytes / (res["gemv"] * 1e-3) / 1e9, 1))
+        out["gemm_tops"].append(round(flops / (res["gemm"] * 1e-3) / 1e12, 1))
+    faster = [n for n, v, m in zip(out["N"], out["gemv_us"], out["gemm_us"])
+              if v is not None and m < v]
+    out["gemm_faster_at_N"] = faster
+    out["dispatch"] = "api.matmul: GEMV below N = %d, GEMM from there" % api.GEMM_MIN_TOKENS
+    del flush
+    return out
+
+
 # ----------------------------------------------------------------------------- ranks
 
 def rank_max(v, dist=None, device="cpu"):
@@ -455,6 +517,9 @@ def run_ours(args, rank, world, local_rank):
     if args.only == "prefill":
         print(json.dumps({"partial_run": "prefill", "prefill": measure_prefill(dev, s, peaks,
                                                                               args.steps)}))
+        return
+    if args.only == "crossover":
+        print(json.dumps({"partial_run": "crossover", "crossover": measure_crossover(dev, s)}))
         return
     dec = DecodeWorkload(dev)
     for _ in range(args.warmup):
@@ -632,6 +697,7 @@ def run_ours(args, rank, world, local_rank):
     del tables
 
     prefill = measure_prefill(dev, s, peaks, K)
+    crossover = measure_crossover(dev, s)
 
     # ---- CPU oracle baseline (rank 0, N=1 only)
     cpu = None
@@ -708,6 +774,7 @@ def run_ours(args, rank, world, local_rank):
                 "two_step_launches_per_step": 8 * dec.layers,
             },
             "prefill": prefill,
+            "crossover": crossover,
             "e2e": {"value": round(whole_job_gbs(world, dec.packed_bytes, e2e_ms), 1),
                     "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -837,7 +904,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "decode", "prefill"], default="all",
+    ap.add_argument("--only", choices=["all", "decode", "prefill", "crossover"], default="all",
                     help="profiling runs: time only one part and print a partial line")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -9,9 +9,15 @@ import torch
 
 from . import _lib
 
-# Largest token count the CUDA-core GEMV handles; above it the tensor-core
-# GEMM takes over (the crossover table lives in `matmul`).
+# Largest token count the CUDA-core GEMV handles.
 GEMV_MAX_TOKENS = 16
+
+# Smallest token count for which `matmul` and `TernaryLinear` use the
+# tensor-core GEMM.  Measured on an 8B-shaped layer (7 projections, one grouped
+# launch, cold L2): GEMV 32 / 39 / 58 / 80 / 198 us and GEMM 54 / 54 / 56 /
+# 58 / 55 us at N = 1 / 2 / 4 / 8 / 16 -- the GEMV's per-token dp4a work
+# overtakes the weight stream from N = 4 on.
+GEMM_MIN_TOKENS = 4
 
 
 def _need(t, dtype, name):
@@ -161,9 +167,9 @@ def gemm(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out
 
 
 def matmul(packed, alpha, xq, amax, xsum, M=None, with_acc=False, stream=None, out=None):
-    """GEMV for N <= GEMV_MAX_TOKENS, else the tensor-core GEMM."""
+    """GEMV below GEMM_MIN_TOKENS tokens, else the tensor-core GEMM."""
     M = packed.shape[0] if M is None else M
-    if xq.shape[0] <= GEMV_MAX_TOKENS:
+    if xq.shape[0] < GEMM_MIN_TOKENS:
         return gemv(packed, alpha, xq, amax, xsum, M, with_acc, stream, out)
     return gemm(packed, alpha, xq, amax, xsum, M, with_acc, stream, out)
 
@@ -175,6 +181,11 @@ GEMV_QUANT_MAX_BYTES = 65536
 def gemv_quant_fits(N, K):
     """Whether the fused quantise+GEMV kernel takes N tokens of width K."""
     return 1 <= N <= GEMV_MAX_TOKENS and N * (-(-K // 512) * 512) <= GEMV_QUANT_MAX_BYTES
+
+
+def use_fused_decode(N, K):
+    """TernaryLinear's choice: the fused kernel below the GEMM crossover."""
+    return N < GEMM_MIN_TOKENS and gemv_quant_fits(N, K)
 
 
 def gemv_quant(packed, alpha, x, M=None, with_acc=False, stream=None, out=None):
@@ -265,8 +276,8 @@ def gemv_tl2(tl2, alpha, xq, amax, M=None, with_acc=False, stream=None, out=None
 
 class TernaryLinear:
     """A BitLinear layer: packed 2-bit ternary weights + alpha, applied to fp32
-    activations: the fused quantise+GEMV kernel for a few tokens, else
-    quant_act -> GEMV/GEMM with the fused rescale."""
+    activations: the fused quantise+GEMV kernel below GEMM_MIN_TOKENS tokens,
+    else quant_act -> tensor-core GEMM with the fused rescale."""
 
     def __init__(self, packed, alpha, in_features, out_features):
         self.packed, self.alpha = packed, alpha
@@ -278,7 +289,7 @@ class TernaryLinear:
         return cls(packed, alpha, W.shape[1], W.shape[0])
 
     def __call__(self, x, stream=None):
-        if gemv_quant_fits(x.shape[0], x.shape[1]):
+        if use_fused_decode(x.shape[0], x.shape[1]):
             return gemv_quant(self.packed, self.alpha, x, self.out_features, stream=stream)
         xq, amax, xsum = quant_act(x, stream)
         return matmul(self.packed, self.alpha, xq, amax, xsum, self.out_features, stream=stream)
