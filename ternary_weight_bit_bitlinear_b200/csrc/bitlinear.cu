@@ -62,7 +62,7 @@ bitlinear_status check_mk(int64_t M, int64_t K) {
 // Per-device facts, looked up once per device.
 struct DeviceInfo {
   int sms = 0;
-  bool gemm_attr_set[2] = {false, false};
+  bool gemm_attr_set[4] = {false, false, false, false};
   int gemv_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};   // 0: not set up yet
   int tl2_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};    // 0: not set up yet
   bool gq_attr_set[bl::kGemvMaxTokens + 1] = {};
@@ -309,8 +309,13 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
   DeviceInfo* dev = nullptr;
   bitlinear_status st = device_info(&dev);
   if (st != BITLINEAR_OK) return st;
-  const bool wide = N > 128;   // 256-token tiles on CTA pairs, else 128-token tiles per CTA
-  const int BN = wide ? bl::kPairBN : 128;
+  // Wide token blocks: 256-token tiles on CTA pairs.  Narrow ones: one CTA per
+  // 128-row tile, 32, 64 or 128 tokens wide -- the narrower the tile, the
+  // smaller its activation stage and the deeper the ring of weight stages the
+  // same shared memory holds (16, 12 or 7), which is what streams the weights
+  // when there are few tokens.
+  const bool wide = N > 128;
+  const int BN = wide ? bl::kPairBN : N <= 32 ? 32 : N <= 64 ? 64 : 128;
   const int BMt = wide ? bl::kPairBM : bl::kGemmBM;
   const int64_t n_tiles = (N + BN - 1) / BN;
   for (int64_t base = 0; base < count; base += bl::kGemmMaxProblems) {
@@ -334,7 +339,8 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
                         static_cast<uint64_t>(q.M), bl::kGemmPackedRowBytes, bl::kGemmBM,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
           !encode_u8_2d(&p.tmB[i], q.xq, static_cast<uint64_t>(q.K), static_cast<uint64_t>(N),
-                        bl::kGemmBK, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||   // 128 tokens per box
+                        bl::kGemmBK, wide ? bl::kPairHalfN : BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B) ||
           (!direct && !encode_f32_2d(&p.tmY[i], q.y, static_cast<uint64_t>(q.M),
                                      static_cast<uint64_t>(N), 32, 32)))
         return BITLINEAR_ERR_CUDA;
@@ -356,7 +362,10 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     p.num_problems = n;
     p.total_tiles = static_cast<int>(tiles);
     build_gemm_schedule(p, wide ? dev->sms / 2 : dev->sms);
-    st = wide ? launch_gemm_pair<5>(p, dev, s) : launch_gemm<128, 7>(p, dev, 0, s);
+    st = wide      ? launch_gemm_pair<5>(p, dev, s)
+         : BN == 32 ? launch_gemm<32, 16>(p, dev, 2, s)
+         : BN == 64 ? launch_gemm<64, 12>(p, dev, 3, s)
+                    : launch_gemm<128, 7>(p, dev, 0, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;

@@ -85,6 +85,10 @@ __device__ __forceinline__ int gemm_my_tile(const GemmParams& p, int i) {
   return gemm_my_tile(p, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), i);
 }
 
+// Per epilogue warp: the 32-token chunks it handles (alternate ones: half 0
+// takes chunks 0, 2, ..., half 1 takes 1, 3, ...), 32 table entries each.
+__host__ __device__ constexpr int gemm_ep_chunks(int BN) { return (BN / 32 + 1) / 2; }
+
 template <int BN, int STAGES>
 struct GemmSmem {
   // every array below up to ep_out is a multiple of 1024 bytes, so all of
@@ -100,8 +104,8 @@ struct GemmSmem {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
-  float ep_scale[kGemmEpiWarps][BN / 2];   // per epilogue warp: alpha * amax/127 of its tokens
-  int ep_xsum[kGemmEpiWarps][BN / 2];      // per epilogue warp: activation sums of its tokens
+  float ep_scale[kGemmEpiWarps][32 * gemm_ep_chunks(BN)];   // per epilogue warp: alpha * amax/127
+  int ep_xsum[kGemmEpiWarps][32 * gemm_ep_chunks(BN)];      // per epilogue warp: activation sums
   uint32_t tmem_slot;
   int abort;
 };
@@ -291,17 +295,19 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       {
         // all loads in flight at once, then the divisions
         const float alpha = __ldg(pr.alpha);
-        float am[BN / 64];
-        int xv[BN / 64];
+        constexpr int kChunks = gemm_ep_chunks(BN);
+        float am[kChunks];
+        int xv[kChunks];
 #pragma unroll
-        for (int k = 0; k < BN / 64; ++k) {
+        for (int k = 0; k < kChunks; ++k) {
           const int n = n_blk * BN + (2 * k + half) * 32 + lane;
-          am[k] = n < pr.N ? __ldg(pr.amax + n) : 0.0f;
-          xv[k] = n < pr.N ? __ldg(pr.xsum + n) : 0;
+          const bool in = 2 * k + half < BN / 32 && n < pr.N;
+          am[k] = in ? __ldg(pr.amax + n) : 0.0f;
+          xv[k] = in ? __ldg(pr.xsum + n) : 0;
         }
         __syncwarp();
 #pragma unroll
-        for (int k = 0; k < BN / 64; ++k) {
+        for (int k = 0; k < kChunks; ++k) {
           sc[k * 32 + lane] = __fmul_rn(alpha, __fdiv_rn(am[k], 127.0f));
           xs[k * 32 + lane] = xv[k];
         }
