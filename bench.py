@@ -60,7 +60,7 @@ NCU_TRAFFIC = {
                    "profile": "profiles/gemv_quant_2b_decode_stream.md"},
     "gemm": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
                       "ternary_weight_bit_bitlinear_b200/csrc/gemm_pair.cuh"],
-             "sha256": "b998379b52960f46", "bytes": 62_609_152 + 31_356_416,
+             "sha256": "0eb46b29ec660fd4", "bytes": 62_596_096 + 29_230_080,
              "profile": "profiles/gemm_i8_pair_7b_prefill.md"},
 }
 

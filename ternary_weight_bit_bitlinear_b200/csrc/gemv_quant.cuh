@@ -83,11 +83,15 @@ struct GqParams {
 // this round, before the __syncwarp) has read.
 // In pieces: the window [win, win + win_bytes) takes up to win_bytes / 4
 // floats at a time, once for the maximum, once for the quantisation.
+//
+// With first_staged, token 0's row was staged in place already (gq_stage_first)
+// as the oldest of kGqStages cp.async groups still pending; the others belong
+// to the weight ring.
 template <int NT>
 __device__ __forceinline__ void gq_quantise(const float* __restrict__ x, int K, int kpad,
                                             int xstride, uint8_t* xs, uint8_t* win,
                                             int win_bytes, int area, float* s_amax,
-                                            int* s_xsum, int lane) {
+                                            int* s_xsum, bool first_staged, int lane) {
   const int K4 = K / 4;
 #pragma unroll 1
   for (int t = 0; t < NT; ++t) {
@@ -97,9 +101,13 @@ __device__ __forceinline__ void gq_quantise(const float* __restrict__ x, int K, 
     float m = 0.0f;
     int sum = 0;
     if (t * xstride + 4 * K <= area) {
-      for (int i = lane; i < K4; i += 32) cp_async16(row8 + 16 * i, row + 4 * i, 16u);
-      cp_async_commit();
-      cp_async_wait<0>();
+      if (t == 0 && first_staged) {
+        cp_async_wait<kGqStages - 1>();
+      } else {
+        for (int i = lane; i < K4; i += 32) cp_async16(row8 + 16 * i, row + 4 * i, 16u);
+        cp_async_commit();
+        cp_async_wait<0>();
+      }
       __syncwarp();
       const float4* v4 = reinterpret_cast<const float4*>(row8);
       for (int i = lane; i < K4; i += 32) m = fmaxf(m, absmax4(v4[i]));
@@ -151,6 +159,13 @@ __device__ __forceinline__ void gq_quantise(const float* __restrict__ x, int K, 
     }
     __syncwarp();
   }
+}
+
+// Token 0's fp32 row staged in place at xs, as one cp.async group.
+__device__ __forceinline__ void gq_stage_first(const float* __restrict__ x, int K, uint8_t* xs,
+                                               int lane) {
+  for (int i = lane; i < K / 4; i += 32) cp_async16(xs + 16 * i, x + 4 * i, 16u);
+  cp_async_commit();
 }
 
 // Segment that warp b belongs to (the last one whose warp_begin <= b).
@@ -223,15 +238,16 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
     slot = (slot + 1) & (kGqStages - 1);
   };
   // The ring's first stages go in before the quantisation when every token's
-  // staged row ends below the ring (the wait for the staging copies then
-  // covers them too, one round trip for both).
+  // staged row ends below the ring.  Token 0's row is copied first, so that its
+  // quantisation waits for that copy alone, not for the weights behind it.
   const bool early_ring = (NT - 1) * p.xstride + 4 * sg.K <= p.area - kGqRingBytes;
   if (early_ring) {
+    gq_stage_first(sg.x, sg.K, xs, lane);
 #pragma unroll 1
     for (int s = 0; s < kGqStages - 1; ++s) issue_next();
   }
   gq_quantise<NT>(sg.x, sg.K, sg.chunks * kGemvChunkK, p.xstride, xs, smem + NT * p.xstride,
-                  p.area - NT * p.xstride, p.area, s_amax, s_xsum, lane);
+                  p.area - NT * p.xstride, p.area, s_amax, s_xsum, early_ring, lane);
   if (!early_ring) {
 #pragma unroll 1
     for (int s = 0; s < kGqStages - 1; ++s) issue_next();
