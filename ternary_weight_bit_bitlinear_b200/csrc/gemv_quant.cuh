@@ -74,8 +74,8 @@ struct GqParams {
 };
 
 // Quantise x [NT][K] (fp32, 16-byte aligned rows) into xs [NT][xstride] int8,
-// zero from K up to kpad; amax and the sum of q of token t go to s_amax[t] and
-// s_xsum[t].  Run by the whole warp.
+// zero from K up to kpad; amax / 127 and the sum of q of token t go to
+// s_a127[t] and s_xsum[t].  Run by the whole warp.
 //
 // In place: token t's row is staged at xs + t * xstride; in round r each lane
 // reads float4 32r + lane and then writes the word of the same index, i.e.
@@ -90,7 +90,7 @@ struct GqParams {
 template <int NT>
 __device__ __forceinline__ void gq_quantise(const float* __restrict__ x, int K, int kpad,
                                             int xstride, uint8_t* xs, uint8_t* win,
-                                            int win_bytes, int area, float* s_amax,
+                                            int win_bytes, int area, float* s_a127,
                                             int* s_xsum, bool first_staged, int lane) {
   const int K4 = K / 4;
 #pragma unroll 1
@@ -154,7 +154,7 @@ __device__ __forceinline__ void gq_quantise(const float* __restrict__ x, int K, 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
     if (lane == 0) {
-      s_amax[t] = m;
+      s_a127[t] = __fdiv_rn(m, 127.0f);
       s_xsum[t] = sum;
     }
     __syncwarp();
@@ -182,7 +182,7 @@ template <int NT>
 __global__ void __launch_bounds__(32)
 gemv_quant_kernel(const __grid_constant__ GqParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float s_amax[NT];
+  __shared__ float s_a127[NT];
   __shared__ int s_xsum[NT];
   const int lane = threadIdx.x;
   const uint32_t sw = static_cast<uint32_t>(lane & 7);
@@ -247,7 +247,7 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
     for (int s = 0; s < kGqStages - 1; ++s) issue_next();
   }
   gq_quantise<NT>(sg.x, sg.K, sg.chunks * kGemvChunkK, p.xstride, xs, smem + NT * p.xstride,
-                  p.area - NT * p.xstride, p.area, s_amax, s_xsum, early_ring, lane);
+                  p.area - NT * p.xstride, p.area, s_a127, s_xsum, early_ring, lane);
   if (!early_ring) {
 #pragma unroll 1
     for (int s = 0; s < kGqStages - 1; ++s) issue_next();
@@ -282,7 +282,7 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
       for (int t = 0; t < NT; ++t) {
         const int a = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) -
                       s_xsum[t];
-        const float scale = __fmul_rn(alpha, __fdiv_rn(s_amax[t], 127.0f));
+        const float scale = __fmul_rn(alpha, s_a127[t]);
         const int64_t o = static_cast<int64_t>(t) * pr.M + row;
         pr.y[o] = __fmul_rn(__int2float_rn(a), scale);
         if (pr.acc) pr.acc[o] = a;
