@@ -68,6 +68,7 @@ struct DeviceInfo {
   bool gq_attr_set[bl::kGemvMaxTokens + 1] = {};
   int gq_smem[bl::kGemvMaxTokens + 1] = {};               // last shared-memory size seen
   int gq_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};      // and its occupancy
+  bool gqs_attr_set[bl::kGqsMaxTokens + 1] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -441,6 +442,33 @@ bitlinear_status gemv_quant_launch(int N, int grid, const bl::GqParams& p, cudaS
   return launch_status();
 }
 
+template <int NT>
+bitlinear_status launch_gemv_quant_split(int grid, const bl::GqParams& p, DeviceInfo* dev,
+                                         cudaStream_t s) {
+  auto kernel = bl::gemv_quant_split_kernel<NT>;
+  if (!dev->gqs_attr_set[NT]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bl::kGqMaxXBytes + bl::kGqsWarps * bl::kGqRingBytes) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    dev->gqs_attr_set[NT] = true;
+  }
+  if (launch_pdl(kernel, grid, bl::kGqsThreads,
+                 static_cast<size_t>(bl::gqs_smem_bytes(NT, p.xstride)), s, p) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  return launch_status();
+}
+
+bitlinear_status gemv_quant_split_launch(int N, int grid, const bl::GqParams& p,
+                                         DeviceInfo* dev, cudaStream_t s) {
+  switch (N) {
+    case 1: return launch_gemv_quant_split<1>(grid, p, dev, s);
+    case 2: return launch_gemv_quant_split<2>(grid, p, dev, s);
+    case 3: return launch_gemv_quant_split<3>(grid, p, dev, s);
+    case 4: return launch_gemv_quant_split<4>(grid, p, dev, s);
+    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  }
+}
+
 // Warps per segment.  Each warp of a segment takes ceil(units / warps) units
 // at most, so a warp's work is that many units of k-chunks, plus about half a
 // unit for staging and quantising its input first (its copy time grows with K
@@ -481,7 +509,9 @@ void gemv_quant_assign(bl::GqParams& p, int warps_total) {
 
 // Fused decode over validated problems sharing N: one launch per at most
 // kGqMaxProblems problems and at most as many input segments as the grid has
-// warps; every warp owns one segment's share of units.
+// warps.  A launch with at least as many units as the one-warp kernel has warp
+// slots gives every warp one segment's share of units; a smaller one (up to 4
+// tokens) runs the split-unit kernel, one 4-warp CTA per unit.
 bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t count,
                                   int64_t N, cudaStream_t s) {
   DeviceInfo* dev = nullptr;
@@ -496,6 +526,7 @@ bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t 
     int n = static_cast<int>(std::min<int64_t>(count - base, bl::kGqMaxProblems));
     bl::GqParams p;
     int grid = 0;
+    int64_t launch_units = 0, launch_cap = 0;
     for (;;) {
       memset(&p, 0, sizeof p);
       int64_t units = 0, kmax = 0;
@@ -538,13 +569,19 @@ bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t 
       const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm;
       if (segs <= cap) {
         grid = static_cast<int>(std::min<int64_t>(cap, units));
+        launch_units = units;
+        launch_cap = cap;
         break;
       }
       n = std::max(1, n / 2);   // more inputs than warps: fewer problems per launch
     }
-    gemv_quant_assign(p, grid);
-    grid = p.seg[p.num_segments - 1].warp_begin + p.seg[p.num_segments - 1].warps;
-    st = gemv_quant_launch(nt, grid, p, s);
+    if (nt <= bl::kGqsMaxTokens && launch_units < launch_cap) {
+      st = gemv_quant_split_launch(nt, static_cast<int>(launch_units), p, dev, s);
+    } else {
+      gemv_quant_assign(p, grid);
+      grid = p.seg[p.num_segments - 1].warp_begin + p.seg[p.num_segments - 1].warps;
+      st = gemv_quant_launch(nt, grid, p, s);
+    }
     if (st != BITLINEAR_OK) return st;
     base += n;
   }

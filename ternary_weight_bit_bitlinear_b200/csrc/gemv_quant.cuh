@@ -292,4 +292,183 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
   cp_async_wait<0>();
 }
 
+// ---------------------------------------------------------------------------
+// Split-unit variant, for launches with fewer units than the kernel above has
+// warp slots (one layer, or one input group of a layer, per launch: the order
+// of a real decoder).  There every warp above would own one unit and work
+// alone on its SM, so one warp's quantisation of a whole input row and its
+// walk through all k-chunks of the unit would be the launch's latency.  Here
+// one CTA of kGqsWarps warps takes one unit:
+//   1. each warp prefetches its share of the k-chunks into L2 (before the
+//      dependent-launch wait) and issues its ring's first stages;
+//   2. all threads reduce amax per token in two passes over x (register
+//      loads, no staging), combine it through shared memory, and quantise
+//      their float4s into the shared int8 copy;
+//   3. warp w streams k-chunks [C w / S, C (w + 1) / S) through its own ring
+//      (gemv.cuh's layout and arithmetic);
+//   4. the other warps leave their int32 sums in their rings, and warp 0 adds
+//      them (integers: the order does not matter) and writes y as above.
+// Shared memory: the int8 copy [NT][xstride], then kGqsWarps rings.
+
+constexpr int kGqsWarps = 4;
+constexpr int kGqsThreads = 32 * kGqsWarps;
+constexpr int kGqsMaxTokens = 4;
+
+__host__ __device__ constexpr int gqs_smem_bytes(int nt, int xstride) {
+  return nt * xstride + kGqsWarps * kGqRingBytes;
+}
+
+// Problem and segment of unit u: the last whose unit_begin <= u.
+__device__ __forceinline__ int gq_problem_of_unit(const GqParams& p, int u) {
+  int lo = 0, hi = p.num_problems - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.prob[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int gq_segment_of_unit(const GqParams& p, int u) {
+  int lo = 0, hi = p.num_segments - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.seg[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kGqsThreads)
+gemv_quant_split_kernel(const __grid_constant__ GqParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float s_m[kGqsWarps][NT];
+  __shared__ int s_q[kGqsWarps][NT];
+  __shared__ float s_a127[NT];
+  __shared__ int s_xsum[NT];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sw = static_cast<uint32_t>(lane & 7);
+  const int unit = blockIdx.x;
+  const GqProblem pr = p.prob[gq_problem_of_unit(p, unit)];
+  const GqSegment sg = p.seg[gq_segment_of_unit(p, unit)];
+  const int row0 = (unit - pr.unit_begin) * kGemvTileRows;
+  const int kc0 = sg.chunks * warp / kGqsWarps;
+  const int kc1 = sg.chunks * (warp + 1) / kGqsWarps;
+  uint8_t* xs = smem;
+  uint8_t* ring = smem + NT * p.xstride + warp * kGqRingBytes;
+
+  // 1. L2 prefetch of this warp's first stages (a hint: nothing is read
+  //    before the wait), then the ring's first stages after it.
+  const GemvCopyPlan cp = gemv_plan(pr, row0, lane);
+#pragma unroll 1
+  for (int kc = kc0; kc < kc1 && kc < kc0 + kGqStages - 1; ++kc) {
+    if (kc * (kGemvChunkBytes / 4) + cp.wword < pr.W) {
+      const uint8_t* src = cp.wsrc + kc * kGemvChunkBytes;
+#pragma unroll 1
+      for (int i = 0; i < cp.vrows; ++i)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(src + i * cp.wstep) : "memory");
+    }
+  }
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+  int ic = kc0, slot = 0;
+  auto issue_next = [&]() {
+    if (ic < kc1) gemv_issue_weights(pr.W, cp, ic++, ring + slot * kGqStageBytes);
+    cp_async_commit();   // one group per stage, empty past this warp's chunks
+    slot = (slot + 1) & (kGqStages - 1);
+  };
+#pragma unroll 1
+  for (int st = 0; st < kGqStages - 1; ++st) issue_next();
+
+  // 2. amax per token over the whole CTA, then the quantisation.
+  const int K4 = sg.K / 4, P4 = sg.chunks * (kGemvChunkK / 4);
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
+    float m = 0.0f;
+    for (int i = tid; i < K4; i += kGqsThreads) m = fmaxf(m, absmax4(x4[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) s_m[warp][t] = m;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kGqsWarps; ++w) m = fmaxf(m, s_m[w][t]);
+    const float s = m == 0.0f ? 0.0f : __fdiv_rn(127.0f, m);
+    const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
+    uint32_t* out = reinterpret_cast<uint32_t*>(xs + t * p.xstride);
+    int sum = 0;
+    for (int i = tid; i < K4; i += kGqsThreads) out[i] = m == 0.0f ? 0u : quant_pack4(x4[i], s, sum);
+    for (int i = K4 + tid; i < P4; i += kGqsThreads) out[i] = 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if (lane == 0) s_q[warp][t] = sum;
+  }
+  __syncthreads();   // the int8 copy and the partial sums are complete
+  if (tid < NT) {
+    float m = 0.0f;
+    int sum = 0;
+#pragma unroll
+    for (int w = 0; w < kGqsWarps; ++w) {
+      m = fmaxf(m, s_m[w][tid]);
+      sum += s_q[w][tid];
+    }
+    s_a127[tid] = __fdiv_rn(m, 127.0f);
+    s_xsum[tid] = sum;
+  }
+
+  // 3. This warp's k-chunks.
+  int acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[t][j] = 0;
+  int cslot = 0;
+  for (int kc = kc0; kc < kc1; ++kc) {
+    issue_next();
+    cp_async_wait<kGqStages - 1>();
+    __syncwarp();
+    const uint8_t* st = ring + cslot * kGqStageBytes;
+    cslot = (cslot + 1) & (kGqStages - 1);
+    gemv_chunk_dot<NT>(st + lane * kGemvChunkBytes, sw, xs + kc * kGemvChunkK, p.xstride, acc);
+    __syncwarp();   // every lane is done with this stage before it is refilled
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+
+  // 4. Partial sums through the rings, the epilogue by warp 0.
+  int* red = reinterpret_cast<int*>(ring);   // [NT][4][32]
+  if (warp > 0) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) red[(t * 4 + j) * 32 + lane] = acc[t][j];
+  }
+  __syncthreads();
+  if (warp != 0) return;
+#pragma unroll 1
+  for (int w = 1; w < kGqsWarps; ++w) {
+    const int* o = reinterpret_cast<const int*>(smem + NT * p.xstride + w * kGqRingBytes);
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[t][j] += o[(t * 4 + j) * 32 + lane];
+  }
+  const int row = row0 + lane;
+  if (row < pr.M) {
+    const float alpha = *pr.alpha;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int a = acc[t][0] + (acc[t][1] >> 2) + (acc[t][2] >> 4) + (acc[t][3] >> 6) -
+                    s_xsum[t];
+      const float scale = __fmul_rn(alpha, s_a127[t]);
+      const int64_t o = static_cast<int64_t>(t) * pr.M + row;
+      pr.y[o] = __fmul_rn(__int2float_rn(a), scale);
+      if (pr.acc) pr.acc[o] = a;
+    }
+  }
+}
+
 }  // namespace bl

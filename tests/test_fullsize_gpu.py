@@ -72,6 +72,19 @@ class Model:
                                     [self.x[(l, _input_proj(p))] for l, p in lst])
         return dict(zip(lst, ys))
 
+    def run_gemv_quant_per_group(self):
+        """The dependent per-layer order: one fused launch per input group
+        (q/k/v, o, gate/up, down).  Launches this small, at one token, run the
+        split-unit kernel (one 4-warp CTA per 32-row unit)."""
+        ys = {}
+        for l in range(self.layers):
+            for projs in ((0, 1, 2), (3,), (4, 5), (6,)):
+                lst = [(l, p) for p in projs]
+                out = api.gemv_quant_grouped([self.w[k] for k in lst],
+                                             self.x[(l, _input_proj(projs[0]))])
+                ys.update(zip(lst, out))
+        return ys
+
     def run_gemm(self, layer):
         lst = [(layer, p) for p in range(7)]
         qs = [self.q[(l, _input_proj(p))] for l, p in lst]
@@ -138,6 +151,19 @@ def test_config2_2b_decode_stream_fused_quant():
     # and the whole stream equals the two-step path bit for bit
     ref = m.run_gemv()
     for k in ys:
+        assert torch.equal(ys[k], ref[k]), k
+
+
+def test_config2_2b_decode_per_group_launches():
+    # the dependent per-layer order (120 small launches, split-unit kernel)
+    # gives the one-launch stream's outputs bit for bit, and the oracle's
+    m = Model(2, 30, 1)
+    ys = m.run_gemv_quant_per_group()
+    for (l, p) in [(0, 1), (5, 3), (17, 4), (29, 6)]:
+        M = m.shape.projections()[p][1]
+        m.check(l, p, ys[(l, p)], _rows(M, 40, 10 * l + p + 2), [0])
+    ref = m.run_gemv()
+    for k in ref:
         assert torch.equal(ys[k], ref[k]), k
 
 

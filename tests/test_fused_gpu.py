@@ -73,6 +73,30 @@ def test_gemv_quant_shapes(M, K, N):
     check(y, acc, oracle.bitlinear(W.numpy(), x.numpy()))
 
 
+@pytest.mark.parametrize("M,K,N", [(160012, 64, 1), (160012, 64, 4), (160012, 640, 3)])
+def test_gemv_quant_one_warp_path_small_k(M, K, N):
+    # More 32-row units (5001) than the one-warp kernel can have resident at
+    # any occupancy (148 SMs x 32 CTAs), so up to 4 tokens these launches take
+    # that kernel rather than the split-unit one that smaller launches of 1-4
+    # tokens take.  Ragged rows (160012 = 5000 x 32 + 12) and a ragged k-chunk.
+    W, (packed, alpha) = layer(M, K, M + K + N)
+    x = inputs.activations(N, K, seed=K + 7 * N, outlier_frac=0.01)
+    y, acc = api.gemv_quant(packed, alpha, x.cuda(), with_acc=True)
+    check(y, acc, oracle.bitlinear(W.numpy(), x.numpy()))
+
+
+@pytest.mark.parametrize("K", [512, 1024, 1536, 2048, 2560, 6912])
+def test_gemv_quant_split_path_chunk_counts(K):
+    # Small launches of 1-4 tokens: one 4-warp CTA per unit, the unit's
+    # k-chunks split over the warps (1, 2, 3, 4, 5 and 14 chunks: some warps get
+    # none, some one, some several).
+    M, N = 200, 2
+    W, (packed, alpha) = layer(M, K, 31 * K + N)
+    x = inputs.activations(N, K, seed=K + 3, outlier_frac=0.01)
+    y, acc = api.gemv_quant(packed, alpha, x.cuda(), with_acc=True)
+    check(y, acc, oracle.bitlinear(W.numpy(), x.numpy()))
+
+
 def test_gemv_quant_equals_two_step_path():
     M, K, N = 2560, 2560, 3
     W, (packed, alpha) = layer(M, K, 77)
