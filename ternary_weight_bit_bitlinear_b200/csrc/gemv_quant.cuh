@@ -313,6 +313,7 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
 constexpr int kGqsWarps = 4;
 constexpr int kGqsThreads = 32 * kGqsWarps;
 constexpr int kGqsMaxTokens = 4;
+constexpr int kGqsRegF4 = 16;   // float4s per thread held in registers (one token, K <= 8192)
 
 __host__ __device__ constexpr int gqs_smem_bytes(int nt, int xstride) {
   return nt * xstride + kGqsWarps * kGqRingBytes;
@@ -379,32 +380,66 @@ gemv_quant_split_kernel(const __grid_constant__ GqParams p) {
 #pragma unroll 1
   for (int st = 0; st < kGqStages - 1; ++st) issue_next();
 
-  // 2. amax per token over the whole CTA, then the quantisation.
+  // 2. amax per token over the whole CTA, then the quantisation.  One token
+  //    with K <= 4 * kGqsRegF4 * kGqsThreads is read once, into registers;
+  //    otherwise x is read twice (the second time from L2).
   const int K4 = sg.K / 4, P4 = sg.chunks * (kGemvChunkK / 4);
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
+  if (NT == 1 && K4 <= kGqsRegF4 * kGqsThreads) {
+    const float4* x4 = reinterpret_cast<const float4*>(sg.x);
+    float4 v[kGqsRegF4];
     float m = 0.0f;
-    for (int i = tid; i < K4; i += kGqsThreads) m = fmaxf(m, absmax4(x4[i]));
+#pragma unroll
+    for (int j = 0; j < kGqsRegF4; ++j) {
+      const int i = tid + j * kGqsThreads;
+      v[j] = i < K4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      m = fmaxf(m, absmax4(v[j]));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (lane == 0) s_m[warp][t] = m;
-  }
-  __syncthreads();
+    if (lane == 0) s_m[warp][0] = m;
+    __syncthreads();
+    m = 0.0f;
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    float m = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kGqsWarps; ++w) m = fmaxf(m, s_m[w][t]);
+    for (int w = 0; w < kGqsWarps; ++w) m = fmaxf(m, s_m[w][0]);
     const float s = m == 0.0f ? 0.0f : __fdiv_rn(127.0f, m);
-    const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
-    uint32_t* out = reinterpret_cast<uint32_t*>(xs + t * p.xstride);
+    uint32_t* out = reinterpret_cast<uint32_t*>(xs);
     int sum = 0;
-    for (int i = tid; i < K4; i += kGqsThreads) out[i] = m == 0.0f ? 0u : quant_pack4(x4[i], s, sum);
+#pragma unroll
+    for (int j = 0; j < kGqsRegF4; ++j) {
+      const int i = tid + j * kGqsThreads;
+      if (i < K4) out[i] = m == 0.0f ? 0u : quant_pack4(v[j], s, sum);
+    }
     for (int i = K4 + tid; i < P4; i += kGqsThreads) out[i] = 0u;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-    if (lane == 0) s_q[warp][t] = sum;
+    if (lane == 0) s_q[warp][0] = sum;
+  } else {
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
+      float m = 0.0f;
+      for (int i = tid; i < K4; i += kGqsThreads) m = fmaxf(m, absmax4(x4[i]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (lane == 0) s_m[warp][t] = m;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float m = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kGqsWarps; ++w) m = fmaxf(m, s_m[w][t]);
+      const float s = m == 0.0f ? 0.0f : __fdiv_rn(127.0f, m);
+      const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
+      uint32_t* out = reinterpret_cast<uint32_t*>(xs + t * p.xstride);
+      int sum = 0;
+      for (int i = tid; i < K4; i += kGqsThreads)
+        out[i] = m == 0.0f ? 0u : quant_pack4(x4[i], s, sum);
+      for (int i = K4 + tid; i < P4; i += kGqsThreads) out[i] = 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+      if (lane == 0) s_q[warp][t] = sum;
+    }
   }
   __syncthreads();   // the int8 copy and the partial sums are complete
   if (tid < NT) {
