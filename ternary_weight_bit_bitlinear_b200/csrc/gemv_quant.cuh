@@ -314,6 +314,7 @@ constexpr int kGqsWarps = 4;
 constexpr int kGqsThreads = 32 * kGqsWarps;
 constexpr int kGqsMaxTokens = 4;
 constexpr int kGqsRegF4 = 16;   // float4s per thread held in registers (one token, K <= 8192)
+constexpr int kGqsPrefetchChunks = 8;
 
 __host__ __device__ constexpr int gqs_smem_bytes(int nt, int xstride) {
   return nt * xstride + kGqsWarps * kGqRingBytes;
@@ -357,11 +358,11 @@ gemv_quant_split_kernel(const __grid_constant__ GqParams p) {
   uint8_t* xs = smem;
   uint8_t* ring = smem + NT * p.xstride + warp * kGqRingBytes;
 
-  // 1. L2 prefetch of this warp's first stages (a hint: nothing is read
-  //    before the wait), then the ring's first stages after it.
+  // 1. L2 prefetch of this warp's k-chunks, up to kGqsPrefetchChunks (a hint:
+  //    nothing is read before the wait), then the ring's first stages after it.
   const GemvCopyPlan cp = gemv_plan(pr, row0, lane);
 #pragma unroll 1
-  for (int kc = kc0; kc < kc1 && kc < kc0 + kGqStages - 1; ++kc) {
+  for (int kc = kc0; kc < kc1 && kc < kc0 + kGqsPrefetchChunks; ++kc) {
     if (kc * (kGemvChunkBytes / 4) + cp.wword < pr.W) {
       const uint8_t* src = cp.wsrc + kc * kGemvChunkBytes;
 #pragma unroll 1
