@@ -301,9 +301,10 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
 // one CTA of kGqsWarps warps takes one unit:
 //   1. each warp prefetches its share of the k-chunks into L2 (before the
 //      dependent-launch wait) and issues its ring's first stages;
-//   2. all threads reduce amax per token in two passes over x (register
-//      loads, no staging), combine it through shared memory, and quantise
-//      their float4s into the shared int8 copy;
+//   2. all threads reduce amax per token, combine it through shared memory
+//      and quantise their float4s into the shared int8 copy; x is read once
+//      into registers when every token's row fits 16 float4s per thread in
+//      total, twice (the second time from L2) otherwise;
 //   3. warp w streams k-chunks [C w / S, C (w + 1) / S) through its own ring
 //      (gemv.cuh's layout and arithmetic);
 //   4. the other warps leave their int32 sums in their rings, and warp 0 adds
@@ -313,7 +314,7 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
 constexpr int kGqsWarps = 4;
 constexpr int kGqsThreads = 32 * kGqsWarps;
 constexpr int kGqsMaxTokens = 4;
-constexpr int kGqsRegF4 = 16;   // float4s per thread held in registers (one token, K <= 8192)
+constexpr int kGqsRegF4 = 16;   // float4s per thread held in registers, over all tokens
 constexpr int kGqsPrefetchChunks = 8;
 
 __host__ __device__ constexpr int gqs_smem_bytes(int nt, int xstride) {
@@ -381,39 +382,46 @@ gemv_quant_split_kernel(const __grid_constant__ GqParams p) {
 #pragma unroll 1
   for (int st = 0; st < kGqStages - 1; ++st) issue_next();
 
-  // 2. amax per token over the whole CTA, then the quantisation.  One token
-  //    with K <= 4 * kGqsRegF4 * kGqsThreads is read once, into registers;
+  // 2. amax per token over the whole CTA, then the quantisation.  Rows with
+  //    K <= 4 * kGqsRegF4 / NT * kGqsThreads are read once, into registers;
   //    otherwise x is read twice (the second time from L2).
   const int K4 = sg.K / 4, P4 = sg.chunks * (kGemvChunkK / 4);
-  if (NT == 1 && K4 <= kGqsRegF4 * kGqsThreads) {
-    const float4* x4 = reinterpret_cast<const float4*>(sg.x);
-    float4 v[kGqsRegF4];
-    float m = 0.0f;
+  constexpr int R = kGqsRegF4 / NT;   // float4s per thread and token
+  if (K4 <= R * kGqsThreads) {
+    float4 v[NT][R];
 #pragma unroll
-    for (int j = 0; j < kGqsRegF4; ++j) {
-      const int i = tid + j * kGqsThreads;
-      v[j] = i < K4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-      m = fmaxf(m, absmax4(v[j]));
+    for (int t = 0; t < NT; ++t) {
+      const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const int i = tid + j * kGqsThreads;
+        v[t][j] = i < K4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        m = fmaxf(m, absmax4(v[t][j]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (lane == 0) s_m[warp][t] = m;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (lane == 0) s_m[warp][0] = m;
     __syncthreads();
-    m = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kGqsWarps; ++w) m = fmaxf(m, s_m[w][0]);
-    const float s = m == 0.0f ? 0.0f : __fdiv_rn(127.0f, m);
-    uint32_t* out = reinterpret_cast<uint32_t*>(xs);
-    int sum = 0;
+    for (int t = 0; t < NT; ++t) {
+      float m = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kGqsRegF4; ++j) {
-      const int i = tid + j * kGqsThreads;
-      if (i < K4) out[i] = m == 0.0f ? 0u : quant_pack4(v[j], s, sum);
+      for (int w = 0; w < kGqsWarps; ++w) m = fmaxf(m, s_m[w][t]);
+      const float s = m == 0.0f ? 0.0f : __fdiv_rn(127.0f, m);
+      uint32_t* out = reinterpret_cast<uint32_t*>(xs + t * p.xstride);
+      int sum = 0;
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const int i = tid + j * kGqsThreads;
+        if (i < K4) out[i] = m == 0.0f ? 0u : quant_pack4(v[t][j], s, sum);
+      }
+      for (int i = K4 + tid; i < P4; i += kGqsThreads) out[i] = 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+      if (lane == 0) s_q[warp][t] = sum;
     }
-    for (int i = K4 + tid; i < P4; i += kGqsThreads) out[i] = 0u;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-    if (lane == 0) s_q[warp][0] = sum;
   } else {
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
