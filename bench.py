@@ -56,7 +56,7 @@ NCU_TRAFFIC = {
              "sha256": "d0ffe60ca94b9a32", "bytes": 522_076_623 + 2_235_136,
              "profile": "profiles/launches_decode_2b.md"},
     "gemv_quant": {"file": "ternary_weight_bit_bitlinear_b200/csrc/gemv_quant.cuh",
-                   "sha256": "c1d58a9d3416cd0c", "bytes": 523_108_124 + 2_584_235,
+                   "sha256": "7f228f2d4b4f408d", "bytes": 523_122_432 + 2_571_093,
                    "profile": "profiles/gemv_quant_2b_decode_stream.md"},
     "gemm": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
                       "ternary_weight_bit_bitlinear_b200/csrc/gemm_pair.cuh"],
