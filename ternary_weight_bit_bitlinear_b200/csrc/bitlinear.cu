@@ -15,6 +15,7 @@
 #include "gemm_pair.cuh"
 #include "gemv.cuh"
 #include "gemv_quant.cuh"
+#include "gemv_split.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
 #include "tl2.cuh"
@@ -69,6 +70,7 @@ struct DeviceInfo {
   int gq_smem[bl::kGemvMaxTokens + 1] = {};               // last shared-memory size seen
   int gq_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};      // and its occupancy
   bool gqs_attr_set[bl::kGqsMaxTokens + 1] = {};
+  bool gemv_split_attr_set[bl::kGemvMaxTokens + 1] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -133,8 +135,21 @@ bitlinear_status launch_gemv_tile(const bl::GemvParams& p, DeviceInfo* dev, cuda
     per_sm = nb;
   }
   // Every warp resident at once, with the same number of units (give or take
-  // one) per warp: units per warp first, then just enough warps.
+  // one) per warp: units per warp first, then just enough warps.  A launch
+  // with fewer units than that takes the split-unit kernel: one CTA per unit.
   const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm * bl::kGemvWarps;
+  if (p.total_units < cap) {
+    auto split = bl::gemv_split_kernel<NT>;
+    if (!dev->gemv_split_attr_set[NT]) {
+      if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return BITLINEAR_ERR_CUDA;
+      dev->gemv_split_attr_set[NT] = true;
+    }
+    if (launch_pdl(split, p.total_units, bl::kGemvThreads, smem, s, p) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    return launch_status();
+  }
   const int64_t upw = (p.total_units + cap - 1) / cap;
   const int64_t warps = (p.total_units + upw - 1) / upw;
   const int grid = static_cast<int>((warps + bl::kGemvWarps - 1) / bl::kGemvWarps);

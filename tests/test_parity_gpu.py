@@ -187,6 +187,28 @@ def test_gemv_parity_all_token_counts(N):
     assert np.array_equal(y.cpu().numpy(), ref["y"])
 
 
+@pytest.mark.parametrize("M,K,N", [(160012, 64, 1), (160012, 640, 4), (160012, 64, 16)])
+def test_gemv_parity_tile_kernel_many_units(M, K, N):
+    # 5001 units: more than gemv_tile_kernel can have warps resident at any
+    # token count (148 SMs x at most 3 CTAs x 4 warps), so these launches take
+    # it rather than the split-unit kernel that the smaller cases here take.
+    ref, (packed, alpha, xq, amax, xsum) = _layer(M, K, N, seed=M + K + N)
+    y, acc = api.gemv(packed, alpha, xq, amax, xsum, with_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("K", [512, 1024, 1536, 2048, 2560, 6912])
+@pytest.mark.parametrize("N", [1, 5, 16])
+def test_gemv_parity_split_kernel_chunk_counts(K, N):
+    # small launches: one 4-warp CTA per unit, its 1 to 14 k-chunks split
+    # over the warps (some warps get none)
+    ref, (packed, alpha, xq, amax, xsum) = _layer(200, K, N, seed=7 * K + N)
+    y, acc = api.gemv(packed, alpha, xq, amax, xsum, with_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
 @pytest.mark.parametrize("M,K,N", [(1024, 1024, 1), (2560, 6912, 1), (640, 2560, 4),
                                    (6912, 2560, 16), (1, 128, 1), (129, 28672, 2)])
 def test_gemv_parity_shapes(M, K, N):
