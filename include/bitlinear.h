@@ -166,6 +166,10 @@ BITLINEAR_API bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* 
  *   y    fp32 [N,M] output: (float)acc * (alpha * (amax[n]/127))
  *   acc  int32 [N,M] output of the raw accumulators, or NULL
  * N > 16 returns BITLINEAR_ERR_UNSUPPORTED_SHAPE.
+ * Two kernels give the same results.  A launch with at least as many 32-row
+ * units as the GPU has resident warps streams them with one warp per unit.
+ * A smaller launch takes one 4-warp CTA per unit, whose warps split the unit's
+ * k-chunks and add their int32 sums at the end.
  */
 BITLINEAR_API bitlinear_status bitlinear_gemv(const uint32_t* packed, const float* alpha,
                                 int64_t M, int64_t K,
