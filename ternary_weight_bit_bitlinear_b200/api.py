@@ -210,8 +210,9 @@ def gemv_quant_grouped(layers, x, with_acc=False, stream=None, outs=None):
     """Fused decode over several layers in one launch.  layers: list of
     (packed, alpha); x: one fp32 tensor [N,K] for all layers or a list with
     one per layer.  Layers that share an input should pass the same tensor and
-    be adjacent (each warp then quantises it once).  Returns a list of y (and
-    of acc)."""
+    be adjacent: in a launch that fills the GPU each warp then quantises one
+    input once (a smaller launch quantises it once per 32-row unit, with all 4
+    warps of the unit's CTA).  Returns a list of y (and of acc)."""
     n = len(layers)
     xs = x if isinstance(x, (list, tuple)) else [x] * n
     N = xs[0].shape[0]
