@@ -46,6 +46,7 @@ SWEEP_CFG = 4
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "source": "fallback"}
 INT8_PER_BF16 = 2.0          # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
+HBM_NOMINAL_GBS = 8000.0     # B200 HBM3e spec figure (context beside the measured copy peak)
 
 # DRAM bytes (read + write) per launch from one ncu capture of each workload's
 # dominant kernel (summaries in profiles/).  They describe the kernel source
@@ -727,6 +728,7 @@ def run_ours(args, rank, world, local_rank):
                 "parallelism": "replicas" if world > 1 else "single GPU",
             },
             "pct_of_measured_hbm": round(100 * gbs / world / hbm_peak, 2),
+            "pct_of_nominal_hbm_8000": round(100 * gbs / world / HBM_NOMINAL_GBS, 2),
             "roofline": {
                 "bound": "hbm",
                 "kernel": "gemv_quant (fused quantise + GEMV, grouped, 210 layers, K=2560 and 6912)",
