@@ -68,7 +68,8 @@ typedef enum {
     BITLINEAR_ERR_MISALIGNED = 3,        /* pointer not 16-byte aligned */
     BITLINEAR_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than required */
     BITLINEAR_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
-    BITLINEAR_ERR_DEVICE_TIMEOUT = 6     /* a kernel gave up a bounded wait */
+    BITLINEAR_ERR_DEVICE_TIMEOUT = 6,    /* a kernel gave up a bounded wait */
+    BITLINEAR_ERR_NONFINITE = 7          /* packed weights held inf or NaN */
 } bitlinear_status;
 
 /* Static, human-readable name of a status code.  Never NULL. */
@@ -92,7 +93,10 @@ BITLINEAR_API size_t bitlinear_pack_workspace_bytes(int64_t M, int64_t K);
  *   alpha    fp32 [1] output: mean|W| rounded to nearest-even once, from an
  *            exact, order-independent sum; 0 when W is all zero (every code 0)
  *   workspace, workspace_bytes: scratch of bitlinear_pack_workspace_bytes()
- * If W holds inf or NaN, *alpha is written as NaN and every code is 0.
+ * If W holds inf or NaN, *alpha is written as NaN, every code is 0, and the
+ * device error word records it: a later bitlinear_device_error() reports
+ * BITLINEAR_ERR_NONFINITE (the call itself cannot know without waiting for
+ * the device, and it returns before the kernels run).
  * Tie rule: |W/alpha| == 0.5 exactly gives code 0 (round half to even).
  */
 BITLINEAR_API bitlinear_status bitlinear_pack_weights(const float* W, int64_t M, int64_t K,
@@ -380,12 +384,27 @@ BITLINEAR_API bitlinear_status bitlinear_pack_weights_noalloc(const float* W, in
 /* ------------------------------------------------------------ diagnostics */
 
 /*
- * Read (and, if clear != 0, reset) the device-side error word that kernels set
- * when a bounded wait gives up.  Synchronises the device.  *status_out is
- * BITLINEAR_OK or BITLINEAR_ERR_DEVICE_TIMEOUT; the return value reports
- * whether the read itself worked.
+ * Read (and, if clear != 0, reset) the device-side error words: kernels set
+ * them when a bounded wait gives up, and the pack step when the weights hold
+ * inf or NaN.  Synchronises the device.  *status_out is BITLINEAR_OK,
+ * BITLINEAR_ERR_DEVICE_TIMEOUT (if any wait gave up) or else
+ * BITLINEAR_ERR_NONFINITE; the return value reports whether the read itself
+ * worked.
  */
 BITLINEAR_API bitlinear_status bitlinear_device_error(int* status_out, int clear);
+
+/*
+ * Wall-time limit, in nanoseconds, of every bounded wait in the kernels
+ * launched after this call (process-wide; 0 restores the default of 2 s).
+ * Returns the previous limit.  A wait that runs out makes its kernel wind
+ * down: it stops issuing work, waits (with a fixed 2 s limit) for the copies
+ * and tensor-core operations it has in flight, releases its tensor memory and
+ * returns, leaving its outputs incomplete and BITLINEAR_ERR_DEVICE_TIMEOUT in
+ * the device error word.  Normal waits last microseconds; a short limit is a
+ * way to exercise that path (or to bound the cost of a stalled device) without
+ * a fault.  Launches already enqueued keep the limit they were given.
+ */
+BITLINEAR_API unsigned long long bitlinear_set_wait_limit(unsigned long long limit_ns);
 
 #ifdef __cplusplus
 }

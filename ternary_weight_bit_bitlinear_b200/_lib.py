@@ -19,6 +19,7 @@ ERR_MISALIGNED = 3
 ERR_WORKSPACE = 4
 ERR_CUDA = 5
 ERR_DEVICE_TIMEOUT = 6
+ERR_NONFINITE = 7
 
 
 class Problem(ctypes.Structure):
@@ -107,6 +108,8 @@ def load(path: str = LIB_PATH):
     L.bitlinear_gemv_tl2_grouped.restype = st
     L.bitlinear_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
     L.bitlinear_device_error.restype = st
+    L.bitlinear_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+    L.bitlinear_set_wait_limit.restype = ctypes.c_ulonglong
     _lib = L
     return L
 
@@ -260,6 +263,12 @@ def bitlinear_gemv_tl2_grouped(problems, count, N, stream=None):
 
 def bitlinear_pack_workspace_bytes(M, K):
     return load().bitlinear_pack_workspace_bytes(M, K)
+
+
+def bitlinear_set_wait_limit(limit_ns):
+    """Set the wall-time limit of the kernels' bounded waits (0: the default);
+    returns the previous limit."""
+    return load().bitlinear_set_wait_limit(int(limit_ns))
 
 
 def bitlinear_device_error(clear=True):

@@ -31,6 +31,34 @@ def _need(t, dtype, name):
         raise ValueError("%s must be contiguous" % name)
 
 
+def _on(device, **tensors):
+    """Every given tensor (None skipped) must sit on `device`: the kernels run
+    on one GPU and dereference all pointers there."""
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError("%s is on %s, the weights on %s: all operands must share one "
+                             "device" % (name, t.device, device))
+
+
+def _check_out(out, N, M, device, name="out"):
+    """A caller-supplied output must be fp32 [N, M], contiguous, on `device`
+    (the kernels write N*M floats through its pointer)."""
+    if out is None:
+        return
+    if not isinstance(out, torch.Tensor) or tuple(out.shape) != (N, M):
+        raise ValueError("%s must have shape (%d, %d), got %s"
+                         % (name, N, M, tuple(getattr(out, "shape", ()))))
+    _need(out, torch.float32, name)
+    _on(device, **{name: out})
+
+
+def _check_token_vector(t, N, dtype, name):
+    """amax / xsum: one entry per token, read for every n < N."""
+    _need(t, dtype, name)
+    if t.numel() != N:
+        raise ValueError("%s must hold N = %d entries, got %d" % (name, N, t.numel()))
+
+
 def packed_row_words(K):
     """Words per packed row: K/16 rounded up to a multiple of 4 (rows end on a
     16-byte boundary; the padding fields hold code 0)."""
@@ -98,15 +126,19 @@ def _matmul(fn, name, packed, alpha, xq, amax, xsum, M, with_acc, stream, out=No
     _need(packed, torch.int32, "packed")
     _need(alpha, torch.float32, "alpha")
     _need(xq, torch.int8, "xq")
-    _need(amax, torch.float32, "amax")
-    _need(xsum, torch.int32, "xsum")
     N, K = xq.shape
+    _check_token_vector(amax, N, torch.float32, "amax")
+    _check_token_vector(xsum, N, torch.int32, "xsum")
     if packed.shape != (M, packed_row_words(K)):
         raise ValueError("packed must be [M, packed_row_words(K)] = [%d, %d], got %s"
                          % (M, packed_row_words(K), tuple(packed.shape)))
-    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=xq.device)
-    acc = torch.empty((N, M), dtype=torch.int32, device=xq.device) if with_acc else None
-    _lib.check(fn(packed, alpha, M, K, xq, amax, xsum, N, y, acc, stream), name)
+    dev = packed.device
+    _on(dev, alpha=alpha, xq=xq, amax=amax, xsum=xsum)
+    _check_out(out, N, M, dev)
+    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=dev)
+    acc = torch.empty((N, M), dtype=torch.int32, device=dev) if with_acc else None
+    with torch.cuda.device(dev):
+        _lib.check(fn(packed, alpha, M, K, xq, amax, xsum, N, y, acc, stream), name)
     return (y, acc) if with_acc else y
 
 
@@ -122,24 +154,34 @@ def _grouped(fn, name, layers, xq, amax, xsum, with_acc, stream, outs):
     xqs = xq if isinstance(xq, (list, tuple)) else [xq] * n
     amaxs = amax if isinstance(amax, (list, tuple)) else [amax] * n
     xsums = xsum if isinstance(xsum, (list, tuple)) else [xsum] * n
+    if not (len(xqs) == len(amaxs) == len(xsums) == n) or (outs is not None and len(outs) != n):
+        raise ValueError("one xq, amax, xsum (and out) per layer, or one for all")
     N = xqs[0].shape[0]
+    dev = layers[0][0].device if n else None
     ys, accs, entries = [], [], []
     for i, (packed, alpha) in enumerate(layers):
         _need(packed, torch.int32, "packed")
         _need(alpha, torch.float32, "alpha")
         _need(xqs[i], torch.int8, "xq")
+        _check_token_vector(amaxs[i], N, torch.float32, "amax")
+        _check_token_vector(xsums[i], N, torch.int32, "xsum")
         M, K = packed.shape[0], xqs[i].shape[1]
         if xqs[i].shape[0] != N or packed.shape[1] != packed_row_words(K):
             raise ValueError("layer %d: packed [M, packed_row_words(K)] must match xq [N, K];"
                              " N shared" % i)
+        _on(dev, packed=packed, alpha=alpha, xq=xqs[i], amax=amaxs[i], xsum=xsums[i])
+        if outs is not None:
+            _check_out(outs[i], N, M, dev, "outs[%d]" % i)
         y = outs[i] if outs is not None else torch.empty((N, M), dtype=torch.float32,
-                                                           device=packed.device)
-        acc = torch.empty((N, M), dtype=torch.int32, device=packed.device) if with_acc else None
+                                                           device=dev)
+        acc = torch.empty((N, M), dtype=torch.int32, device=dev) if with_acc else None
         ys.append(y)
         accs.append(acc)
         entries.append((packed, alpha, M, K, xqs[i], amaxs[i], xsums[i], y, acc))
     arr = _lib.make_problems(entries)
-    _lib.check(fn(arr, n, N, stream), name)
+    if n:
+        with torch.cuda.device(dev):
+            _lib.check(fn(arr, n, N, stream), name)
     return (ys, accs) if with_acc else ys
 
 
@@ -199,10 +241,14 @@ def gemv_quant(packed, alpha, x, M=None, with_acc=False, stream=None, out=None):
     if packed.shape != (M, packed_row_words(K)):
         raise ValueError("packed must be [M, packed_row_words(K)] = [%d, %d], got %s"
                          % (M, packed_row_words(K), tuple(packed.shape)))
-    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=x.device)
-    acc = torch.empty((N, M), dtype=torch.int32, device=x.device) if with_acc else None
-    _lib.check(_lib.bitlinear_gemv_quant(packed, alpha, M, K, x, N, y, acc, stream),
-               "bitlinear_gemv_quant")
+    dev = packed.device
+    _on(dev, alpha=alpha, x=x)
+    _check_out(out, N, M, dev)
+    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=dev)
+    acc = torch.empty((N, M), dtype=torch.int32, device=dev) if with_acc else None
+    with torch.cuda.device(dev):
+        _lib.check(_lib.bitlinear_gemv_quant(packed, alpha, M, K, x, N, y, acc, stream),
+                   "bitlinear_gemv_quant")
     return (y, acc) if with_acc else y
 
 
@@ -210,12 +256,14 @@ def gemv_quant_grouped(layers, x, with_acc=False, stream=None, outs=None):
     """Fused decode over several layers in one launch.  layers: list of
     (packed, alpha); x: one fp32 tensor [N,K] for all layers or a list with
     one per layer.  Layers that share an input should pass the same tensor and
-    be adjacent: in a launch that fills the GPU each warp then quantises one
-    input once (a smaller launch quantises it once per 32-row unit, with all 4
-    warps of the unit's CTA).  Returns a list of y (and of acc)."""
+    be adjacent, so that the kernel quantises it once for the rows it streams.
+    Returns a list of y (and of acc)."""
     n = len(layers)
     xs = x if isinstance(x, (list, tuple)) else [x] * n
+    if len(xs) != n or (outs is not None and len(outs) != n):
+        raise ValueError("one x (and out) per layer, or one x for all")
     N = xs[0].shape[0]
+    dev = layers[0][0].device if n else None
     ys, accs, entries = [], [], []
     for i, (packed, alpha) in enumerate(layers):
         _need(packed, torch.int32, "packed")
@@ -225,15 +273,20 @@ def gemv_quant_grouped(layers, x, with_acc=False, stream=None, outs=None):
         if xs[i].shape[0] != N or packed.shape[1] != packed_row_words(K):
             raise ValueError("layer %d: packed [M, packed_row_words(K)] must match x [N, K];"
                              " N shared" % i)
+        _on(dev, packed=packed, alpha=alpha, x=xs[i])
+        if outs is not None:
+            _check_out(outs[i], N, M, dev, "outs[%d]" % i)
         y = outs[i] if outs is not None else torch.empty((N, M), dtype=torch.float32,
-                                                           device=packed.device)
-        acc = torch.empty((N, M), dtype=torch.int32, device=packed.device) if with_acc else None
+                                                           device=dev)
+        acc = torch.empty((N, M), dtype=torch.int32, device=dev) if with_acc else None
         ys.append(y)
         accs.append(acc)
         entries.append((packed, alpha, M, K, xs[i], y, acc))
     arr = _lib.make_fused_problems(entries)
-    _lib.check(_lib.bitlinear_gemv_quant_grouped(arr, n, N, stream),
-               "bitlinear_gemv_quant_grouped")
+    if n:
+        with torch.cuda.device(dev):
+            _lib.check(_lib.bitlinear_gemv_quant_grouped(arr, n, N, stream),
+                       "bitlinear_gemv_quant_grouped")
     return (ys, accs) if with_acc else ys
 
 
@@ -263,15 +316,19 @@ def gemv_tl2(tl2, alpha, xq, amax, M=None, with_acc=False, stream=None, out=None
     _need(tl2, torch.uint8, "tl2")
     _need(alpha, torch.float32, "alpha")
     _need(xq, torch.int8, "xq")
-    _need(amax, torch.float32, "amax")
     M = tl2.shape[0] if M is None else M
     N, K = xq.shape
+    _check_token_vector(amax, N, torch.float32, "amax")
     if tl2.shape != (M, tl2_row_bytes(K)):
         raise ValueError("tl2 must be [M, tl2_row_bytes(K)] = [%d, %d]" % (M, tl2_row_bytes(K)))
-    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=xq.device)
-    acc = torch.empty((N, M), dtype=torch.int32, device=xq.device) if with_acc else None
-    _lib.check(_lib.bitlinear_gemv_tl2(tl2, alpha, M, K, xq, amax, N, y, acc, stream),
-               "bitlinear_gemv_tl2")
+    dev = tl2.device
+    _on(dev, alpha=alpha, xq=xq, amax=amax)
+    _check_out(out, N, M, dev)
+    y = out if out is not None else torch.empty((N, M), dtype=torch.float32, device=dev)
+    acc = torch.empty((N, M), dtype=torch.int32, device=dev) if with_acc else None
+    with torch.cuda.device(dev):
+        _lib.check(_lib.bitlinear_gemv_tl2(tl2, alpha, M, K, xq, amax, N, y, acc, stream),
+                   "bitlinear_gemv_tl2")
     return (y, acc) if with_acc else y
 
 

@@ -30,6 +30,12 @@ def sources():
             if f.endswith((".cu", ".cuh"))] + [os.path.join(INCLUDE, "bitlinear.h")]
 
 
+def units():
+    """The translation units: the C ABI (bitlinear.cu) and one launcher unit
+    per kernel family (launch_*.cu), compiled in parallel."""
+    return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith(".cu")]
+
+
 def up_to_date():
     if not os.path.exists(LIB):
         return False
@@ -38,16 +44,29 @@ def up_to_date():
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/bitlinear.cu into libbitlinear.so unless it is up to date."""
+    """Compile every unit of csrc/ and link libbitlinear.so, unless it is up
+    to date."""
     if not force and up_to_date():
         return LIB
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    procs, objs = [], []
+    for src in units():
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".%d.o" % os.getpid())
+        cmd = [NVCC, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+            print(" ".join(cmd))
+        procs.append((src, subprocess.Popen(cmd)))
+        objs.append(obj)
+    failed = [src for src, p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, "nvcc " + " ".join(failed))
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [NVCC, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-shared", "-cudart", "static",
-           "-o", tmp, os.path.join(CSRC, "bitlinear.cu")]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd))
-    subprocess.check_call(cmd)
+    subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                           "-cudart", "static", "-o", tmp, *objs])
+    for obj in objs:
+        os.remove(obj)
     os.replace(tmp, LIB)
     return LIB
 

@@ -1,79 +1,30 @@
 // bitlinear.cu -- the C ABI of libbitlinear.so (declared in include/bitlinear.h):
-// argument checks, launch configuration and TMA descriptor set-up around the
-// sm_100a kernels in pack.cuh, quant.cuh, gemv.cuh and gemm.cuh.
+// argument checks, problem tables, launch configuration and TMA descriptor
+// set-up around the sm_100a kernels.  The weight-packing and quantiser kernels
+// (pack.cuh, quant.cuh) are launched from here; the GEMV, fused decode, GEMM
+// and TL2 kernels from their own units (launch_*.cu, see internal.h).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstdint>
-#include <algorithm>
+#include <cstring>
 #include <mutex>
 #include <utility>
 #include <vector>
 
-#include "bitlinear.h"
-#include "gemm.cuh"
-#include "gemm_pair.cuh"
-#include "gemv.cuh"
-#include "gemv_quant.cuh"
-#include "gemv_split.cuh"
+#include "internal.h"
 #include "pack.cuh"
 #include "quant.cuh"
-#include "tl2.cuh"
+
+namespace blh {
 
 namespace {
-
-constexpr int64_t kMaxK = 131072;
-constexpr int64_t kMaxElems = int64_t(1) << 40;
-constexpr int kMaxDevices = 64;
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
-
-// Launch with programmatic stream serialisation (see pdl_wait_prior_grid).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem,
-                       cudaStream_t s, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(static_cast<unsigned>(block));
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
-
-bitlinear_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? BITLINEAR_OK : BITLINEAR_ERR_CUDA;
-}
-
-// Words per packed row: K/16 rounded up to a multiple of 4 (16 bytes).
-int64_t packed_row_words(int64_t K) { return 4 * ((K + 63) / 64); }
-
-bitlinear_status check_mk(int64_t M, int64_t K) {
-  if (M < 0 || K < 0) return BITLINEAR_ERR_INVALID_ARG;
-  if (M == 0 || K == 0 || K % 16 != 0 || K > kMaxK) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  if (M > INT_MAX / 2 || M * K > kMaxElems) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  return BITLINEAR_OK;
-}
-
-// Per-device facts, looked up once per device.
-struct DeviceInfo {
-  int sms = 0;
-  bool gemm_attr_set[4] = {false, false, false, false};
-  int gemv_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};   // 0: not set up yet
-  int tl2_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};    // 0: not set up yet
-  bool gq_attr_set[bl::kGemvMaxTokens + 1] = {};
-  int gq_smem[bl::kGemvMaxTokens + 1] = {};               // last shared-memory size seen
-  int gq_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};      // and its occupancy
-  bool gqs_attr_set[bl::kGqsMaxTokens + 1] = {};
-  bool gemv_split_attr_set[bl::kGemvMaxTokens + 1] = {};
-};
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
+std::atomic<unsigned long long> g_wait_limit_ns{bl::kWaitLimitNs};
+}  // namespace
 
 bitlinear_status device_info(DeviceInfo** out) {
   int dev = 0;
@@ -88,6 +39,34 @@ bitlinear_status device_info(DeviceInfo** out) {
     d.sms = sms;
   }
   *out = &d;
+  return BITLINEAR_OK;
+}
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
+}  // namespace blh
+
+namespace {
+
+using blh::DeviceInfo;
+using blh::device_info;
+using blh::launch_pdl;
+using blh::launch_status;
+using blh::kMaxDevices;
+
+constexpr int64_t kMaxK = 131072;
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Words per packed row: K/16 rounded up to a multiple of 4 (16 bytes).
+int64_t packed_row_words(int64_t K) { return 4 * ((K + 63) / 64); }
+
+bitlinear_status check_mk(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return BITLINEAR_ERR_INVALID_ARG;
+  if (M == 0 || K == 0 || K % 16 != 0 || K > kMaxK) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  if (M > INT_MAX / 2 || M * K > kMaxElems) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   return BITLINEAR_OK;
 }
 
@@ -117,58 +96,6 @@ bool encode_u8_2d(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t row
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
-}
-
-template <int NT>
-bitlinear_status launch_gemv_tile(const bl::GemvParams& p, DeviceInfo* dev, cudaStream_t s) {
-  auto kernel = bl::gemv_tile_kernel<NT>;
-  constexpr int smem = bl::GemvCfg<NT>::kSmemBytes;
-  int& per_sm = dev->gemv_blocks_per_sm[NT];
-  if (per_sm == 0) {
-    int nb = 0;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, bl::kGemvThreads, smem) !=
-            cudaSuccess ||
-        nb < 1)
-      return BITLINEAR_ERR_CUDA;
-    per_sm = nb;
-  }
-  // Every warp resident at once, with the same number of units (give or take
-  // one) per warp: units per warp first, then just enough warps.  A launch
-  // with fewer units than that takes the split-unit kernel: one CTA per unit.
-  const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm * bl::kGemvWarps;
-  if (p.total_units < cap) {
-    auto split = bl::gemv_split_kernel<NT>;
-    if (!dev->gemv_split_attr_set[NT]) {
-      if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-          cudaSuccess)
-        return BITLINEAR_ERR_CUDA;
-      dev->gemv_split_attr_set[NT] = true;
-    }
-    if (launch_pdl(split, p.total_units, bl::kGemvThreads, smem, s, p) != cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
-    return launch_status();
-  }
-  const int64_t upw = (p.total_units + cap - 1) / cap;
-  const int64_t warps = (p.total_units + upw - 1) / upw;
-  const int grid = static_cast<int>((warps + bl::kGemvWarps - 1) / bl::kGemvWarps);
-  if (launch_pdl(kernel, grid, bl::kGemvThreads, smem, s, p) != cudaSuccess)
-    return BITLINEAR_ERR_CUDA;
-  return launch_status();
-}
-
-bitlinear_status launch_gemv_n(int N, const bl::GemvParams& p, DeviceInfo* dev, cudaStream_t s) {
-  switch (N) {
-#define BL_GEMV_CASE(n) \
-  case n: return launch_gemv_tile<n>(p, dev, s);
-    BL_GEMV_CASE(1) BL_GEMV_CASE(2) BL_GEMV_CASE(3) BL_GEMV_CASE(4)
-    BL_GEMV_CASE(5) BL_GEMV_CASE(6) BL_GEMV_CASE(7) BL_GEMV_CASE(8)
-    BL_GEMV_CASE(9) BL_GEMV_CASE(10) BL_GEMV_CASE(11) BL_GEMV_CASE(12)
-    BL_GEMV_CASE(13) BL_GEMV_CASE(14) BL_GEMV_CASE(15) BL_GEMV_CASE(16)
-#undef BL_GEMV_CASE
-    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  }
 }
 
 // Decode GEMV over problems that share N (all validated): one launch
@@ -203,7 +130,7 @@ bitlinear_status gemv_group(const bitlinear_problem* probs, int64_t count, int64
     if (units > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     p.num_problems = n;
     p.total_units = static_cast<int>(units);
-    st = launch_gemv_n(static_cast<int>(N), p, dev, s);
+    st = blh::launch_gemv(static_cast<int>(N), p, dev, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;
@@ -222,40 +149,6 @@ bool encode_f32_2d(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t ro
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
-}
-
-template <int BN, int STAGES>
-bitlinear_status launch_gemm(const bl::GemmParams& p, DeviceInfo* dev, int slot, cudaStream_t s) {
-  auto kernel = bl::gemm_i8_tcgen05_kernel<BN, STAGES>;
-  const int smem = static_cast<int>(sizeof(bl::GemmSmem<BN, STAGES>)) + 1024;
-  if (!dev->gemm_attr_set[slot]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
-    dev->gemm_attr_set[slot] = true;
-  }
-  const int grid = p.total_tiles < dev->sms ? p.total_tiles : dev->sms;
-  if (launch_pdl(kernel, grid, bl::kGemmThreads, smem, s, p) != cudaSuccess)
-    return BITLINEAR_ERR_CUDA;
-  return launch_status();
-}
-
-// CTA-pair GEMM for wide token blocks: two CTAs (a compile-time cluster) per
-// 256 x 256 tile, one pair per two SMs.
-template <int STAGES>
-bitlinear_status launch_gemm_pair(const bl::GemmParams& p, DeviceInfo* dev, cudaStream_t s) {
-  auto kernel = bl::gemm_i8_pair_kernel<STAGES>;
-  const int smem = static_cast<int>(sizeof(bl::GemmPairSmem<STAGES>)) + 1024;
-  if (!dev->gemm_attr_set[1]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
-    dev->gemm_attr_set[1] = true;
-  }
-  const int pairs = p.total_tiles < dev->sms / 2 ? p.total_tiles : dev->sms / 2;
-  if (launch_pdl(kernel, 2 * pairs, bl::kGemmThreads, smem, s, p) != cudaSuccess)
-    return BITLINEAR_ERR_CUDA;
-  return launch_status();
 }
 
 bitlinear_status check_matmul_args(const uint32_t* packed, const float* alpha, int64_t M,
@@ -377,11 +270,9 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     if (tiles > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     p.num_problems = n;
     p.total_tiles = static_cast<int>(tiles);
+    p.wait_ns = blh::wait_limit_ns();
     build_gemm_schedule(p, wide ? dev->sms / 2 : dev->sms);
-    st = wide      ? launch_gemm_pair<5>(p, dev, s)
-         : BN == 32 ? launch_gemm<32, 16>(p, dev, 2, s)
-         : BN == 64 ? launch_gemm<64, 12>(p, dev, 3, s)
-                    : launch_gemm<128, 7>(p, dev, 0, s);
+    st = blh::launch_gemm(wide ? 1 : BN == 32 ? 2 : BN == 64 ? 3 : 0, p, dev, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;
@@ -405,84 +296,6 @@ bitlinear_status check_fused_problem(const bitlinear_fused_problem& q, int64_t N
 // copy round trip): above it the row goes through the ring's space in
 // pieces, which keeps the area, and so the warps per SM, unchanged.
 constexpr int kGqInPlaceMaxArea = 28 * 1024;
-
-template <int NT>
-bitlinear_status gemv_quant_blocks_per_sm(int area, DeviceInfo* dev, int* out) {
-  auto kernel = bl::gemv_quant_kernel<NT>;
-  if (!dev->gq_attr_set[NT]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bl::kGqMaxXBytes + bl::kGqRingBytes) != cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
-    dev->gq_attr_set[NT] = true;
-  }
-  if (dev->gq_smem[NT] != area) {
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, 32, area) != cudaSuccess ||
-        nb < 1)
-      return BITLINEAR_ERR_CUDA;
-    dev->gq_smem[NT] = area;
-    dev->gq_blocks_per_sm[NT] = nb;
-  }
-  *out = dev->gq_blocks_per_sm[NT];
-  return BITLINEAR_OK;
-}
-
-bitlinear_status gemv_quant_occupancy(int N, int area, DeviceInfo* dev, int* out) {
-  switch (N) {
-#define BL_GQ_CASE(n) \
-  case n: return gemv_quant_blocks_per_sm<n>(area, dev, out);
-    BL_GQ_CASE(1) BL_GQ_CASE(2) BL_GQ_CASE(3) BL_GQ_CASE(4)
-    BL_GQ_CASE(5) BL_GQ_CASE(6) BL_GQ_CASE(7) BL_GQ_CASE(8)
-    BL_GQ_CASE(9) BL_GQ_CASE(10) BL_GQ_CASE(11) BL_GQ_CASE(12)
-    BL_GQ_CASE(13) BL_GQ_CASE(14) BL_GQ_CASE(15) BL_GQ_CASE(16)
-#undef BL_GQ_CASE
-    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  }
-}
-
-bitlinear_status gemv_quant_launch(int N, int grid, const bl::GqParams& p, cudaStream_t s) {
-  cudaError_t e = cudaErrorInvalidValue;
-  switch (N) {
-#define BL_GQ_CASE(n) \
-  case n: e = launch_pdl(bl::gemv_quant_kernel<n>, grid, 32, static_cast<size_t>(p.area), s, p); \
-    break;
-    BL_GQ_CASE(1) BL_GQ_CASE(2) BL_GQ_CASE(3) BL_GQ_CASE(4)
-    BL_GQ_CASE(5) BL_GQ_CASE(6) BL_GQ_CASE(7) BL_GQ_CASE(8)
-    BL_GQ_CASE(9) BL_GQ_CASE(10) BL_GQ_CASE(11) BL_GQ_CASE(12)
-    BL_GQ_CASE(13) BL_GQ_CASE(14) BL_GQ_CASE(15) BL_GQ_CASE(16)
-#undef BL_GQ_CASE
-    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  }
-  if (e != cudaSuccess) return BITLINEAR_ERR_CUDA;
-  return launch_status();
-}
-
-template <int NT>
-bitlinear_status launch_gemv_quant_split(int grid, const bl::GqParams& p, DeviceInfo* dev,
-                                         cudaStream_t s) {
-  auto kernel = bl::gemv_quant_split_kernel<NT>;
-  if (!dev->gqs_attr_set[NT]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bl::kGqMaxXBytes + bl::kGqsWarps * bl::kGqRingBytes) != cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
-    dev->gqs_attr_set[NT] = true;
-  }
-  if (launch_pdl(kernel, grid, bl::kGqsThreads,
-                 static_cast<size_t>(bl::gqs_smem_bytes(NT, p.xstride)), s, p) != cudaSuccess)
-    return BITLINEAR_ERR_CUDA;
-  return launch_status();
-}
-
-bitlinear_status gemv_quant_split_launch(int N, int grid, const bl::GqParams& p,
-                                         DeviceInfo* dev, cudaStream_t s) {
-  switch (N) {
-    case 1: return launch_gemv_quant_split<1>(grid, p, dev, s);
-    case 2: return launch_gemv_quant_split<2>(grid, p, dev, s);
-    case 3: return launch_gemv_quant_split<3>(grid, p, dev, s);
-    case 4: return launch_gemv_quant_split<4>(grid, p, dev, s);
-    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  }
-}
 
 // Warps per segment.  Each warp of a segment takes ceil(units / warps) units
 // at most, so a warp's work is that many units of k-chunks, plus about half a
@@ -579,7 +392,7 @@ bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t 
       const int in_place = (nt - 1) * p.xstride + 4 * static_cast<int>(kmax);
       p.area = in_place > plain && in_place <= kGqInPlaceMaxArea ? in_place : plain;
       int per_sm = 0;
-      st = gemv_quant_occupancy(nt, p.area, dev, &per_sm);
+      st = blh::gemv_quant_occupancy(nt, p.area, dev, &per_sm);
       if (st != BITLINEAR_OK) return st;
       const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm;
       if (segs <= cap) {
@@ -591,11 +404,11 @@ bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t 
       n = std::max(1, n / 2);   // more inputs than warps: fewer problems per launch
     }
     if (nt <= bl::kGqsMaxTokens && launch_units < launch_cap) {
-      st = gemv_quant_split_launch(nt, static_cast<int>(launch_units), p, dev, s);
+      st = blh::gemv_quant_split_launch(nt, static_cast<int>(launch_units), p, dev, s);
     } else {
       gemv_quant_assign(p, grid);
       grid = p.seg[p.num_segments - 1].warp_begin + p.seg[p.num_segments - 1].warps;
-      st = gemv_quant_launch(nt, grid, p, s);
+      st = blh::gemv_quant_launch(nt, grid, p, s);
     }
     if (st != BITLINEAR_OK) return st;
     base += n;
@@ -614,44 +427,6 @@ bitlinear_status check_tl2_problem(const bitlinear_tl2_problem& q, int64_t N) {
   if (!aligned4(q.alpha) || !aligned4(q.amax)) return BITLINEAR_ERR_MISALIGNED;
   (void)N;
   return BITLINEAR_OK;
-}
-
-template <int NT>
-bitlinear_status launch_gemv_tl2(const bl::Tl2Params& p, DeviceInfo* dev, cudaStream_t s) {
-  auto kernel = bl::gemv_tl2_kernel<NT>;
-  constexpr int smem = bl::Tl2Cfg<NT>::kSmemBytes;
-  int& per_sm = dev->tl2_blocks_per_sm[NT];
-  if (per_sm == 0) {
-    int nb = 0;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, bl::kTl2Threads, smem) !=
-            cudaSuccess ||
-        nb < 1)
-      return BITLINEAR_ERR_CUDA;
-    per_sm = nb;
-  }
-  const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm * bl::kTl2Warps;
-  const int64_t upw = (p.total_units + cap - 1) / cap;
-  const int64_t warps = (p.total_units + upw - 1) / upw;
-  const int grid = static_cast<int>((warps + bl::kTl2Warps - 1) / bl::kTl2Warps);
-  if (launch_pdl(kernel, grid, bl::kTl2Threads, smem, s, p) != cudaSuccess)
-    return BITLINEAR_ERR_CUDA;
-  return launch_status();
-}
-
-bitlinear_status launch_gemv_tl2_n(int N, const bl::Tl2Params& p, DeviceInfo* dev,
-                                   cudaStream_t s) {
-  switch (N) {
-#define BL_TL2_CASE(n) \
-  case n: return launch_gemv_tl2<n>(p, dev, s);
-    BL_TL2_CASE(1) BL_TL2_CASE(2) BL_TL2_CASE(3) BL_TL2_CASE(4)
-    BL_TL2_CASE(5) BL_TL2_CASE(6) BL_TL2_CASE(7) BL_TL2_CASE(8)
-    BL_TL2_CASE(9) BL_TL2_CASE(10) BL_TL2_CASE(11) BL_TL2_CASE(12)
-    BL_TL2_CASE(13) BL_TL2_CASE(14) BL_TL2_CASE(15) BL_TL2_CASE(16)
-#undef BL_TL2_CASE
-    default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-  }
 }
 
 bitlinear_status gemv_tl2_group(const bitlinear_tl2_problem* probs, int64_t count, int64_t N,
@@ -686,7 +461,7 @@ bitlinear_status gemv_tl2_group(const bitlinear_tl2_problem* probs, int64_t coun
     if (units > INT_MAX) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
     p.num_problems = n;
     p.total_units = static_cast<int>(units);
-    st = launch_gemv_tl2_n(static_cast<int>(N), p, dev, s);
+    st = blh::launch_gemv_tl2(static_cast<int>(N), p, dev, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;
@@ -705,11 +480,12 @@ const char* bitlinear_status_string(int status) {
     case BITLINEAR_ERR_WORKSPACE: return "workspace missing or too small";
     case BITLINEAR_ERR_CUDA: return "CUDA error";
     case BITLINEAR_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case BITLINEAR_ERR_NONFINITE: return "non-finite weights (inf or NaN)";
     default: return "unknown status";
   }
 }
 
-int bitlinear_version(void) { return 100; }
+int bitlinear_version(void) { return 101; }
 
 size_t bitlinear_pack_workspace_bytes(int64_t M, int64_t K) {
   (void)M;
@@ -924,9 +700,8 @@ bitlinear_status bitlinear_tl2_from_packed(const uint32_t* packed, int64_t M, in
   const int64_t total = M * (nb + (K - bl::kTl2Block * nb + 63) / 64);
   int64_t g = (total + 255) / 256;
   if (g > dev->sms * 16) g = dev->sms * 16;
-  bl::tl2_convert_kernel<<<static_cast<int>(g), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      packed, M, K, static_cast<int>(packed_row_words(K)), tl2);
-  return launch_status();
+  return blh::launch_tl2_convert(packed, M, K, static_cast<int>(packed_row_words(K)), tl2,
+                                 static_cast<int>(g), reinterpret_cast<cudaStream_t>(stream));
 }
 
 bitlinear_status bitlinear_gemv_tl2(const uint8_t* tl2, const float* alpha, int64_t M, int64_t K,
@@ -956,16 +731,28 @@ bitlinear_status bitlinear_gemv_tl2_grouped(const bitlinear_tl2_problem* problem
 bitlinear_status bitlinear_device_error(int* status_out, int clear) {
   if (!status_out) return BITLINEAR_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return BITLINEAR_ERR_CUDA;
-  unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, bl::g_device_error, sizeof v) != cudaSuccess)
+  // One error word per unit of the library; this unit's holds the pack step's.
+  unsigned int v = 0, w = 0;
+  if (blh::read_error_word(bl::g_device_error, &w, clear != 0) != cudaSuccess)
     return BITLINEAR_ERR_CUDA;
-  *status_out = (v & bl::kDeviceTimeout) ? BITLINEAR_ERR_DEVICE_TIMEOUT : BITLINEAR_OK;
-  if (clear && v) {
-    unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(bl::g_device_error, &zero, sizeof zero) != cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
+  v |= w;
+  cudaError_t (*const readers[])(unsigned int*, bool) = {
+      blh::device_error_gemv, blh::device_error_gemv_quant, blh::device_error_gemm,
+      blh::device_error_tl2};
+  for (auto rd : readers) {
+    w = 0;
+    if (rd(&w, clear != 0) != cudaSuccess) return BITLINEAR_ERR_CUDA;
+    v |= w;
   }
+  *status_out = (v & bl::kDeviceTimeout)     ? BITLINEAR_ERR_DEVICE_TIMEOUT
+                : (v & bl::kDeviceNonFinite) ? BITLINEAR_ERR_NONFINITE
+                                             : BITLINEAR_OK;
   return BITLINEAR_OK;
+}
+
+unsigned long long bitlinear_set_wait_limit(unsigned long long limit_ns) {
+  const unsigned long long v = limit_ns ? limit_ns : bl::kWaitLimitNs;
+  return blh::g_wait_limit_ns.exchange(v);
 }
 
 }  // extern "C"
@@ -976,24 +763,17 @@ bitlinear_status bitlinear_device_error(int* status_out, int clear) {
 static __device__ __align__(256) unsigned char g_noalloc_pack_scratch[bl::kPackWorkspaceBytes];
 
 namespace {
-void* g_noalloc_pack_ptr[kMaxDevices] = {};
-std::mutex g_noalloc_mutex;
-
 // Device address of the scratch array for the current device.  Host code may
 // not pass the symbol itself to a kernel: on the host it names a stand-in,
-// not device memory.  Looked up once per device, with that device current.
+// not device memory.  Looked up on every call, with the caller's device
+// current, so a device reset or a new primary context never leaves a stale
+// address behind (the lookup is a host-side table read once the module is
+// loaded).
 bitlinear_status noalloc_pack_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_pack_scratch) != cudaSuccess || !p)
     return BITLINEAR_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_pack_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_pack_scratch) != cudaSuccess || !p)
-      return BITLINEAR_ERR_CUDA;
-    g_noalloc_pack_ptr[dev] = p;
-  }
-  *out = g_noalloc_pack_ptr[dev];
+  *out = p;
   return BITLINEAR_OK;
 }
 }  // namespace

@@ -62,6 +62,7 @@ struct GemmParams {
   // sched_begin[b+1]) in that order (built on the host, longest tiles first,
   // each to the least-loaded CTA); otherwise tiles b, b + grid, b + 2 grid...
   int use_sched;
+  unsigned long long wait_ns;   // limit of every bounded wait of the launch
   uint16_t sched_begin[kGemmMaxGrid + 1];
   uint16_t sched[kGemmMaxSched];
 };
@@ -109,6 +110,18 @@ struct GemmSmem {
   uint32_t tmem_slot;
   int abort;
 };
+
+// Before the CTA releases its shared memory: wait for the TMA loads still in
+// flight.  Only the last STAGES loads issued can be (the producer waited for
+// each stage to be consumed before refilling it); load i completes phase
+// (i / STAGES) & 1 of full[i % STAGES], and nothing re-arms those barriers
+// after the producer stops.  On the normal path every one of them has been
+// consumed already and the waits return at once.
+template <int STAGES>
+__device__ __forceinline__ void gemm_drain_loads(uint64_t* full, int issued) {
+  for (int i = issued - 1; i >= 0 && i >= issued - STAGES; --i)
+    mbar_drain(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
+}
 
 template <int BN>
 __device__ __forceinline__ void gemm_locate(const GemmParams& p, int tile, int& pi, int& m_blk,
@@ -170,21 +183,24 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
+      int issued = 0;
       for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti) {
         const int tile = gemm_my_tile(p, ti);
         int pi, m_blk, n_blk;
         gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
         const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort)) goto producer_done;
+          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort, p.wait_ns)) goto producer_done;
           mbar_arrive_expect_tx(&s.full[stage], kStageTx);
           tma_load_2d(s.apk[stage], &p.tmA[pi], &s.full[stage], kb * kGemmPackedRowBytes,
                       m_blk * kGemmBM);
           tma_load_2d(s.b[stage], &p.tmB[pi], &s.full[stage], kb * kGemmBK, n_blk * BN);
+          ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-    producer_done:;
+    producer_done:
+      gemm_drain_loads<STAGES>(s.full, issued);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -198,13 +214,13 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
         gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
         const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
         const uint32_t ab = it & 1, ap = (it >> 1) & 1;
-        if (!mbar_wait(&s.tempty[ab], ap ^ 1u, abort)) break;
+        if (!mbar_wait(&s.tempty[ab], ap ^ 1u, abort, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * BN;
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&s.full[stage], phase, abort) ||
-              !mbar_wait(&s.ufull[ub], uphase, abort)) {
+          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
+              !mbar_wait(&s.ufull[ub], uphase, abort, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -226,13 +242,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       }
       // Everything issued must finish before tensor memory is released.
       mma_commit(&s.drain);
-      unsigned long long t0 = global_timer_ns();
-      while (!mbar_try_wait(&s.drain, 0)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-          atomicOr(&g_device_error, kDeviceTimeout);
-          break;
-        }
-      }
+      mbar_drain(&s.drain, 0);
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ unpackers
@@ -246,8 +256,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(&s.full[stage], phase, abort) ||
-            !mbar_wait(&s.uempty[ub], uphase ^ 1u, abort))
+        if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
+            !mbar_wait(&s.uempty[ub], uphase ^ 1u, abort, p.wait_ns))
           goto unpack_done;
         const uint4* src = reinterpret_cast<const uint4*>(s.apk[stage] + u * kGemmPackedRowBytes);
         const uint4 h0 = src[half], h1 = src[half ^ 1];
@@ -286,7 +296,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       // by value: registers, not re-read from parameter space after each store
       const GemmProblem pr = p.prob[pi];
       const uint32_t ab = it & 1, ap = (it >> 1) & 1;
-      if (!mbar_wait(&s.tfull[ab], ap, abort)) break;
+      if (!mbar_wait(&s.tfull[ab], ap, abort, p.wait_ns)) break;
       tc_fence_after();
       const int m = m_blk * kGemmBM + r_in_tile;
       // this warp's copy of the tile's per-token scale and sum

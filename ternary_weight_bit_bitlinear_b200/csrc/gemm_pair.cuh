@@ -113,24 +113,38 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // The two producers must issue the same number of loads: rank 1's
+      // activation loads complete on rank 0's barriers, and rank 0 drains them
+      // before the pair exits.  So they do not follow the CTA's abort flag
+      // (which is per CTA) and wait on `empty` (committed to both CTAs alike)
+      // with the drain limit: both stop at the same stage when the commits stop.
+      volatile int no_abort = 0;
       uint32_t stage = 0, phase = 0;
+      int issued = 0;
       for (int ti = 0; ti < ntiles; ++ti) {
         const int tile = gemm_my_tile(p, pair, npairs, ti);
         int pi, m_blk, n_blk;
         gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
         const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_cluster(&s.empty[stage], phase ^ 1u, abort)) goto producer_done;
+          if (!mbar_wait_cluster(&s.empty[stage], phase ^ 1u, &no_abort, kDrainLimitNs))
+            goto producer_done;
           mbar_arrive_expect_tx(&s.afull[stage], kATx);
           tma_load_2d(s.apk[stage], &p.tmA[pi], &s.afull[stage], kb * kGemmPackedRowBytes,
                       m_blk * kPairBM + static_cast<int>(rank) * kGemmBM);
           if (rank == 0) mbar_arrive_expect_tx(&s.bfull[stage], kBTx);
           tma_load_2d_pair(s.b[stage], &p.tmB[pi], &s.bfull[stage], kb * kGemmBK,
                            n_blk * kPairBN + static_cast<int>(rank) * kPairHalfN);
+          ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-    producer_done:;
+    producer_done:
+      // This CTA's weight loads land on its own afull barriers; both CTAs'
+      // activation loads count on rank 0's bfull barriers, so rank 0 waits for
+      // those of the pair (the two producers issue the same sequence).
+      gemm_drain_loads<STAGES>(s.afull, issued);
+      if (rank == 0) gemm_drain_loads<STAGES>(s.bfull, issued);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (rank 0)
@@ -144,13 +158,13 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
         gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
         const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
         const uint32_t ab = it & 1, ap = (it >> 1) & 1;
-        if (!mbar_wait_cluster(&s.tempty[ab], ap ^ 1u, abort)) break;
+        if (!mbar_wait_cluster(&s.tempty[ab], ap ^ 1u, abort, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * kPairBN;
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_cluster(&s.bfull[stage], phase, abort) ||
-              !mbar_wait_cluster(&s.ufull[ub], uphase, abort)) {
+          if (!mbar_wait_cluster(&s.bfull[stage], phase, abort, p.wait_ns) ||
+              !mbar_wait_cluster(&s.ufull[ub], uphase, abort, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -185,8 +199,8 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
       gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(&s.afull[stage], phase, abort) ||
-            !mbar_wait_cluster(&s.uempty[ub], uphase ^ 1u, abort))
+        if (!mbar_wait(&s.afull[stage], phase, abort, p.wait_ns) ||
+            !mbar_wait_cluster(&s.uempty[ub], uphase ^ 1u, abort, p.wait_ns))
           goto unpack_done;
         const uint4* src = reinterpret_cast<const uint4*>(s.apk[stage] + u * kGemmPackedRowBytes);
         const uint4 h0 = src[half], h1 = src[half ^ 1];
@@ -224,7 +238,7 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
       gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
       const GemmProblem pr = p.prob[pi];   // by value: registers, not parameter-space reloads
       const uint32_t ab = it & 1, ap = (it >> 1) & 1;
-      if (!mbar_wait_cluster(&s.tfull[ab], ap, abort)) break;
+      if (!mbar_wait_cluster(&s.tfull[ab], ap, abort, p.wait_ns)) break;
       tc_fence_after();
       const int m_base = m_blk * kPairBM + static_cast<int>(rank) * kGemmBM;
       const int m = m_base + r_in_tile;
@@ -295,15 +309,7 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
 
   // The pair's last MMAs write both CTAs' tensor memory and read both shared
   // memories: each CTA waits for them, then both meet before anything is freed.
-  if (warp == 1 && lane == 0) {
-    const unsigned long long t0 = global_timer_ns();
-    while (!mbar_try_wait_cluster(&s.drain, 0)) {
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(&g_device_error, kDeviceTimeout);
-        break;
-      }
-    }
-  }
+  if (warp == 1 && lane == 0) mbar_drain(&s.drain, 0);
   tc_fence_before();
   cluster_sync();
   tc_fence_after();

@@ -34,7 +34,7 @@
 #pragma once
 
 #include "gemv.cuh"
-#include "quant.cuh"
+#include "quant_math.cuh"
 
 namespace bl {
 

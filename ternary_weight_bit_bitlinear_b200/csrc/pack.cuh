@@ -25,7 +25,7 @@ constexpr int kBinsThreads = 256;
 constexpr int kBinsWarps = kBinsThreads / 32;
 
 // Per-warp shared histograms keep same-address atomics inside one warp.
-__global__ void __launch_bounds__(kBinsThreads)
+static __global__ void __launch_bounds__(kBinsThreads)
 abs_bins_kernel(const float4* __restrict__ w4, int64_t n4,
                 unsigned long long* __restrict__ bins, unsigned int* __restrict__ flag) {
   __shared__ unsigned long long hist[kBinsWarps][kBins];
@@ -65,12 +65,13 @@ abs_bins_kernel(const float4* __restrict__ w4, int64_t n4,
 // The numerator is a 384-bit integer D; restoring division by `count`, one
 // quotient bit per numerator bit from the top, continued into fractional bit
 // positions until the bit below the fp32 unit in the last place is known.
-__global__ void alpha_finalize_kernel(const unsigned long long* __restrict__ bins,
+static __global__ void alpha_finalize_kernel(const unsigned long long* __restrict__ bins,
                                       const unsigned int* __restrict__ flag, uint64_t count,
                                       float* __restrict__ alpha) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   if (*flag) {
     *alpha = __int_as_float(0x7FC00000);   // NaN marks a non-finite weight
+    atomicOr(&g_device_error, kDeviceNonFinite);
     return;
   }
   constexpr int kLimbs = 12;   // 384 bits; the numerator needs < 320
@@ -140,7 +141,7 @@ __global__ void alpha_finalize_kernel(const unsigned long long* __restrict__ bin
 // One thread per packed word.  A row holds `wp` words: the first `kw` =
 // K/16 carry 16 consecutive weights each, the rest (when K is not a multiple
 // of 64) pad the row to a 16-byte boundary with code-0 fields (01).
-__global__ void __launch_bounds__(256)
+static __global__ void __launch_bounds__(256)
 ternarize_pack_kernel(const float4* __restrict__ w4, int64_t rows, int kw, int wp,
                       const float* __restrict__ alpha_ptr, uint32_t* __restrict__ packed) {
   const float alpha = *alpha_ptr;

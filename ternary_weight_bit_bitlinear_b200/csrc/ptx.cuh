@@ -10,13 +10,20 @@
 namespace bl {
 
 // Device-side error word: a kernel that gives up a bounded wait ORs
-// kDeviceTimeout into it; bitlinear_device_error() reads it back.
-__device__ unsigned int g_device_error = 0;
+// kDeviceTimeout into it, the pack step ORs kDeviceNonFinite when the weights
+// hold inf or NaN; bitlinear_device_error() reads it back.  Each translation
+// unit of the library is its own device module and has its own copy (static):
+// the host reads all of them.
+static __device__ unsigned int g_device_error = 0;
 constexpr unsigned int kDeviceTimeout = 1u;
+constexpr unsigned int kDeviceNonFinite = 2u;
 
-// A wait gives up after this much wall time (ns, %globaltimer).  Normal waits
-// in these kernels last microseconds.
+// Default wall-time limit of a bounded wait (ns, %globaltimer).  Normal waits
+// in these kernels last microseconds.  The limit a launch uses travels in its
+// parameters (bitlinear_set_wait_limit changes it); draining the work a CTA
+// has already issued uses kDrainLimitNs, whatever that setting.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -77,22 +84,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up (returns
-// false, sets *abort and the device error word) after kWaitLimitNs, or as soon
-// as another role of the same CTA has given up (*abort != 0).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// false, sets *abort and the device error word) after limit_ns, or as soon as
+// another role of the same CTA has given up (*abort != 0).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0) {
+    if ((i & 15u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicOr(&g_device_error, kDeviceTimeout);
         return false;
       }
     }
   }
+}
+
+// Wait, without an abort flag, for a phase that work this CTA has already
+// issued will complete (its own copies or MMAs in flight), before the memory
+// they touch is released.  Gives up after kDrainLimitNs.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kDrainLimitNs) {
+      atomicOr(&g_device_error, kDeviceTimeout);
+      return false;
+    }
+  }
+  return true;
 }
 
 // ------------------------------------------------------------------ TMA
@@ -299,14 +321,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 // mbar_wait for barriers that the other CTA of the pair arrives on, directly
 // or through a multicast commit.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
+                                                  volatile int* abort,
+                                                  unsigned long long limit_ns) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   unsigned long long t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((i & 255u) == 0) {
+    if ((i & 15u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicOr(&g_device_error, kDeviceTimeout);
         return false;

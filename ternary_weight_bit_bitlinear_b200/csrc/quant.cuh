@@ -18,6 +18,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "quant_math.cuh"
 
 namespace bl {
 
@@ -40,24 +41,7 @@ struct QuantParams {
   int count;
 };
 
-__device__ __forceinline__ int quant_one(float x, float s) {
-  int v = __float2int_rn(__fmul_rn(x, s));   // NaN (0 * inf) -> 0; +-inf saturate
-  return max(-128, min(127, v));
-}
-
-__device__ __forceinline__ uint32_t quant_pack4(float4 v, float s, int& sum) {
-  const int a = quant_one(v.x, s), b = quant_one(v.y, s), c = quant_one(v.z, s),
-            d = quant_one(v.w, s);
-  sum += a + b + c + d;
-  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | (static_cast<uint32_t>(d) << 24);
-}
-
-__device__ __forceinline__ float absmax4(float4 v) {
-  return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-}
-
-__global__ void __launch_bounds__(kQuantThreads)
+static __global__ void __launch_bounds__(kQuantThreads)
 quant_rows_kernel(const __grid_constant__ QuantParams p) {
   __shared__ float red_f[kQuantThreads / 32];
   __shared__ int red_i[kQuantThreads / 32];
@@ -126,7 +110,7 @@ quant_rows_kernel(const __grid_constant__ QuantParams p) {
 // Per-tensor maximum of |x| over n4 float4s, folded into *out (the bits of a
 // non-negative float order like unsigned integers, so atomicMax on them is
 // the float maximum).  *out must start at 0.
-__global__ void __launch_bounds__(kQuantThreads)
+static __global__ void __launch_bounds__(kQuantThreads)
 tensor_absmax_kernel(const float4* __restrict__ x, int64_t n4, unsigned int* __restrict__ out) {
   __shared__ float red[kQuantThreads / 32];
   pdl_wait_prior_grid();

@@ -56,7 +56,7 @@ __device__ __forceinline__ int i2_field(const uint32_t* row, int64_t k) {
   return (row[k >> 4] >> (8 * (k & 3) + 2 * ((k & 15) >> 2))) & 3;
 }
 
-__global__ void __launch_bounds__(256)
+static __global__ void __launch_bounds__(256)
 tl2_convert_kernel(const uint32_t* __restrict__ packed, int64_t rows, int64_t K, int wp,
                    uint8_t* __restrict__ out) {
   const int64_t nb = tl2_blocks(K);

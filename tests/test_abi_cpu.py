@@ -34,11 +34,23 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.bitlinear_version() == 100
-    for code in range(7):
-        assert _lib.status_string(code)
+    assert L.bitlinear_version() == 101
+    names = {_lib.status_string(code) for code in range(8)}
+    assert len(names) == 8 and "unknown status" not in names
     assert _lib.status_string(0) == "ok"
+    assert "non-finite" in _lib.status_string(_lib.ERR_NONFINITE)
     assert _lib.status_string(99) == "unknown status"
+
+
+def test_wait_limit_setting_is_host_only(L):
+    # A process-wide host setting: no CUDA call, so it works without a device.
+    default = _lib.bitlinear_set_wait_limit(5000)
+    try:
+        assert default == 2_000_000_000
+        assert _lib.bitlinear_set_wait_limit(7000) == 5000
+    finally:
+        assert _lib.bitlinear_set_wait_limit(0) == 7000
+    assert _lib.bitlinear_set_wait_limit(0) == default   # 0 restored the default
 
 
 def test_missing_library_raises(tmp_path):

@@ -80,11 +80,14 @@ def test_pack_edge_cases():
     a_ref = oracle.absmean(W)
     assert alpha.cpu().numpy()[0] == a_ref
     assert np.array_equal(words(packed), oracle.pack(oracle.ternarize(W, a_ref)))
-    # non-finite -> alpha NaN, codes 0
+    # non-finite -> alpha NaN, codes 0, and the device error word says so
+    assert _lib.bitlinear_device_error(clear=True) == _lib.OK
     W = np.ones((128, 128), np.float32)
     W[3, 5] = np.inf
     packed, alpha = api.pack_weights(dev_t(W))
     assert np.isnan(alpha.item()) and (words(packed) == 0x55555555).all()
+    assert _lib.bitlinear_device_error(clear=True) == _lib.ERR_NONFINITE
+    assert _lib.bitlinear_device_error(clear=True) == _lib.OK
 
 
 # ----------------------------------------------------------------------------- quant_act
