@@ -292,126 +292,103 @@ bitlinear_status check_fused_problem(const bitlinear_fused_problem& q, int64_t N
   return BITLINEAR_OK;
 }
 
-// Largest shared-memory area for which a token row is staged in place (one
-// copy round trip): above it the row goes through the ring's space in
-// pieces, which keeps the area, and so the warps per SM, unchanged.
-constexpr int kGqInPlaceMaxArea = 28 * 1024;
-
-// Warps per segment.  Each warp of a segment takes ceil(units / warps) units
-// at most, so a warp's work is that many units of k-chunks, plus about half a
-// unit for staging and quantising its input first (its copy time grows with K
-// like a unit's).  Starting from one warp each, the segment with the largest
-// estimate gets just enough warps for its largest share to drop by one unit,
-// until the warps run out; this minimises the largest estimate.
-void gemv_quant_assign(bl::GqParams& p, int warps_total) {
-  const int n = p.num_segments;
-  std::vector<int> w(n, 1);
-  int left = warps_total - n;
-  auto load = [&](int g) {
-    const int per = (p.seg[g].units + w[g] - 1) / w[g];
-    return (2 * per + 1) * p.seg[g].chunks;   // twice (per + 1/2) units of chunks
-  };
-  std::vector<std::pair<int, int>> heap;   // (load, segment), max-heap
-  for (int g = 0; g < n; ++g) heap.push_back({load(g), g});
-  std::make_heap(heap.begin(), heap.end());
-  while (!heap.empty()) {
-    std::pop_heap(heap.begin(), heap.end());
-    const int g = heap.back().second;
-    heap.pop_back();
-    const int per = (p.seg[g].units + w[g] - 1) / w[g];
-    if (per <= 1) continue;                 // one unit per warp already: cannot drop
-    const int need = (p.seg[g].units + per - 2) / (per - 1) - w[g];
-    if (need > left) break;                 // the largest estimate cannot drop any further
-    w[g] += need;
-    left -= need;
-    heap.push_back({load(g), g});
-    std::push_heap(heap.begin(), heap.end());
+// Plan of one fused launch: its problems and segments (runs of consecutive
+// problems on one input), the CTA size with the most warps resident per SM
+// (fewest warps per CTA on a tie: more CTAs to share the work), and each CTA's
+// range of units, cut so that every range holds about the same number of
+// (unit, k-chunk) pairs.
+bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, int nt,
+                                 DeviceInfo* dev, bl::GqParams& p, int* grid, int* warps) {
+  memset(&p, 0, sizeof p);
+  int64_t units = 0, kmax = 0;
+  int segs = 0;
+  std::vector<int64_t> seg_pairs;
+  for (int i = 0; i < n; ++i) {
+    const bitlinear_fused_problem& q = probs[i];
+    bl::GqProblem& g = p.prob[i];
+    g.packed = q.packed;
+    g.alpha = q.alpha;
+    g.y = q.y;
+    g.acc = q.acc;
+    g.M = static_cast<int>(q.M);
+    g.W = static_cast<int>(packed_row_words(q.K));
+    g.unit_begin = static_cast<int>(units);
+    const int64_t u = (q.M + bl::kGemvTileRows - 1) / bl::kGemvTileRows;
+    const bool same = segs > 0 && p.seg[segs - 1].x == q.x && p.seg[segs - 1].K == q.K;
+    if (!same) {
+      bl::GqSegment& sg = p.seg[segs++];
+      sg.x = q.x;
+      sg.K = static_cast<int>(q.K);
+      sg.chunks = static_cast<int>((q.K + bl::kGemvChunkK - 1) / bl::kGemvChunkK);
+      sg.unit_begin = static_cast<int>(units);
+      sg.prob_begin = i;
+      seg_pairs.push_back(0);
+    }
+    p.seg[segs - 1].units += static_cast<int>(u);
+    seg_pairs.back() += u * p.seg[segs - 1].chunks;
+    units += u;
+    kmax = std::max<int64_t>(kmax, q.K);
+    if (units > INT_MAX / 2) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   }
-  int begin = 0;
-  for (int g = 0; g < n; ++g) {
-    p.seg[g].warp_begin = begin;
-    p.seg[g].warps = w[g];
-    begin += w[g];
+  p.num_problems = n;
+  p.num_segments = segs;
+  p.xstride = static_cast<int>((kmax + bl::kGemvChunkK - 1) / bl::kGemvChunkK * bl::kGemvChunkK);
+  // CTA size: the most warps resident per SM.
+  int best_w = 0, best_per_sm = 0, best_resident = 0;
+  for (int w = 4; w <= bl::gq_max_warps(nt); w += 2) {
+    int per_sm = 0;
+    bitlinear_status st =
+        blh::gemv_quant_occupancy(nt, w, bl::gq_smem_bytes(nt, w, p.xstride), dev, &per_sm);
+    if (st != BITLINEAR_OK) return st;
+    if (per_sm * w > best_resident) {
+      best_resident = per_sm * w;
+      best_w = w;
+      best_per_sm = per_sm;
+    }
   }
+  if (best_w == 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
+  p.area = bl::gq_smem_bytes(nt, best_w, p.xstride);
+  int64_t ctas = std::min<int64_t>(static_cast<int64_t>(dev->sms) * best_per_sm, units);
+  ctas = std::min<int64_t>(ctas, bl::kGqMaxCtas);
+  // Unit ranges: CTA c starts at the first unit whose pairs-before count
+  // reaches c * total / ctas (rounded to the nearer unit boundary); empty
+  // ranges are dropped.
+  int64_t total = 0;
+  for (int64_t v : seg_pairs) total += v;
+  int g = 0;
+  p.bounds[0] = 0;
+  int sg = 0;
+  int64_t seg_pair_begin = 0;
+  for (int64_t c = 1; c < ctas; ++c) {
+    const int64_t t = total * c / ctas;
+    while (sg + 1 < segs && seg_pair_begin + seg_pairs[sg] <= t) seg_pair_begin += seg_pairs[sg++];
+    const int64_t C = p.seg[sg].chunks;
+    const int64_t u = p.seg[sg].unit_begin + (t - seg_pair_begin + C / 2) / C;
+    const int b = static_cast<int>(std::min<int64_t>(u, units));
+    if (b > p.bounds[g]) p.bounds[++g] = b;
+  }
+  if (units > p.bounds[g]) p.bounds[++g] = static_cast<int>(units);
+  *grid = g;
+  *warps = best_w;
+  return BITLINEAR_OK;
 }
 
 // Fused decode over validated problems sharing N: one launch per at most
-// kGqMaxProblems problems and at most as many input segments as the grid has
-// warps.  A launch with at least as many units as the one-warp kernel has warp
-// slots gives every warp one segment's share of units; a smaller one (up to 4
-// tokens) runs the split-unit kernel, one 4-warp CTA per unit.
+// kGqMaxProblems problems.
 bitlinear_status gemv_quant_group(const bitlinear_fused_problem* probs, int64_t count,
                                   int64_t N, cudaStream_t s) {
   DeviceInfo* dev = nullptr;
   bitlinear_status st = device_info(&dev);
   if (st != BITLINEAR_OK) return st;
   const int nt = static_cast<int>(N);
-  int64_t base = 0;
-  while (base < count) {
-    // Shared-memory area from the largest K of this launch's first problems.
-    // Start from as many problems as the table holds; shrink to the number of
-    // segments the grid can give one warp each.
-    int n = static_cast<int>(std::min<int64_t>(count - base, bl::kGqMaxProblems));
-    bl::GqParams p;
-    int grid = 0;
-    int64_t launch_units = 0, launch_cap = 0;
-    for (;;) {
-      memset(&p, 0, sizeof p);
-      int64_t units = 0, kmax = 0;
-      int segs = 0;
-      for (int i = 0; i < n; ++i) {
-        const bitlinear_fused_problem& q = probs[base + i];
-        bl::GqProblem& g = p.prob[i];
-        g.packed = q.packed;
-        g.alpha = q.alpha;
-        g.y = q.y;
-        g.acc = q.acc;
-        g.M = static_cast<int>(q.M);
-        g.W = static_cast<int>(packed_row_words(q.K));
-        g.unit_begin = static_cast<int>(units);
-        const int64_t u = (q.M + bl::kGemvTileRows - 1) / bl::kGemvTileRows;
-        const bool same = segs > 0 && p.seg[segs - 1].x == q.x && p.seg[segs - 1].K == q.K;
-        if (!same) {
-          bl::GqSegment& sg = p.seg[segs++];
-          sg.x = q.x;
-          sg.K = static_cast<int>(q.K);
-          sg.chunks = static_cast<int>((q.K + bl::kGemvChunkK - 1) / bl::kGemvChunkK);
-          sg.unit_begin = static_cast<int>(units);
-          sg.prob_begin = i;
-        }
-        p.seg[segs - 1].units += static_cast<int>(u);
-        units += u;
-        kmax = std::max<int64_t>(kmax, q.K);
-        if (units > INT_MAX / 2) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
-      }
-      p.num_problems = n;
-      p.num_segments = segs;
-      const int64_t chunks = (kmax + bl::kGemvChunkK - 1) / bl::kGemvChunkK;
-      p.xstride = static_cast<int>(chunks * bl::kGemvChunkK);
-      const int plain = nt * p.xstride + bl::kGqRingBytes;
-      const int in_place = (nt - 1) * p.xstride + 4 * static_cast<int>(kmax);
-      p.area = in_place > plain && in_place <= kGqInPlaceMaxArea ? in_place : plain;
-      int per_sm = 0;
-      st = blh::gemv_quant_occupancy(nt, p.area, dev, &per_sm);
-      if (st != BITLINEAR_OK) return st;
-      const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm;
-      if (segs <= cap) {
-        grid = static_cast<int>(std::min<int64_t>(cap, units));
-        launch_units = units;
-        launch_cap = cap;
-        break;
-      }
-      n = std::max(1, n / 2);   // more inputs than warps: fewer problems per launch
-    }
-    if (nt <= bl::kGqsMaxTokens && launch_units < launch_cap) {
-      st = blh::gemv_quant_split_launch(nt, static_cast<int>(launch_units), p, dev, s);
-    } else {
-      gemv_quant_assign(p, grid);
-      grid = p.seg[p.num_segments - 1].warp_begin + p.seg[p.num_segments - 1].warps;
-      st = blh::gemv_quant_launch(nt, grid, p, s);
-    }
+  bl::GqParams p;
+  for (int64_t base = 0; base < count; base += bl::kGqMaxProblems) {
+    const int n = static_cast<int>(std::min<int64_t>(count - base, bl::kGqMaxProblems));
+    int grid = 0, warps = 0;
+    st = gemv_quant_plan(probs + base, n, nt, dev, p, &grid, &warps);
     if (st != BITLINEAR_OK) return st;
-    base += n;
+    st = blh::gemv_quant_launch(nt, grid, warps, p, s);
+    if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;
 }

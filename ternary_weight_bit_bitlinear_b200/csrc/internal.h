@@ -31,9 +31,8 @@ struct DeviceInfo {
   int gemv_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};   // 0: not set up yet
   int tl2_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};    // 0: not set up yet
   bool gq_attr_set[bl::kGemvMaxTokens + 1] = {};
-  int gq_smem[bl::kGemvMaxTokens + 1] = {};               // last shared-memory size seen
-  int gq_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};      // and its occupancy
-  bool gqs_attr_set[bl::kGqsMaxTokens + 1] = {};
+  int gq_area[bl::kGemvMaxTokens + 1][bl::kGqMaxWarps + 1] = {};   // last shared-memory size
+  int gq_occ[bl::kGemvMaxTokens + 1][bl::kGqMaxWarps + 1] = {};    // and its CTAs per SM
   bool gemv_split_attr_set[bl::kGemvMaxTokens + 1] = {};
 };
 
@@ -69,11 +68,11 @@ inline bitlinear_status launch_status() {
 // launch_gemv.cu: decode GEMV on int8 activations (tile or split-unit kernel).
 bitlinear_status launch_gemv(int N, const bl::GemvParams& p, DeviceInfo* dev, cudaStream_t s);
 
-// launch_gemv_quant.cu: the fused quantise + GEMV decode kernels.
-bitlinear_status gemv_quant_occupancy(int N, int area, DeviceInfo* dev, int* out);
-bitlinear_status gemv_quant_launch(int N, int grid, const bl::GqParams& p, cudaStream_t s);
-bitlinear_status gemv_quant_split_launch(int N, int grid, const bl::GqParams& p,
-                                         DeviceInfo* dev, cudaStream_t s);
+// launch_gemv_quant.cu: the fused quantise + GEMV decode kernel.  CTAs of
+// `warps` warps with `area` bytes of dynamic shared memory each.
+bitlinear_status gemv_quant_occupancy(int N, int warps, int area, DeviceInfo* dev, int* out);
+bitlinear_status gemv_quant_launch(int N, int grid, int warps, const bl::GqParams& p,
+                                   cudaStream_t s);
 
 // launch_gemm.cu: tensor-core GEMMs.  variant: 0 = 128-token tiles, 1 = CTA
 // pairs, 2 = 32-token tiles, 3 = 64-token tiles.

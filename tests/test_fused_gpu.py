@@ -74,11 +74,10 @@ def test_gemv_quant_shapes(M, K, N):
 
 
 @pytest.mark.parametrize("M,K,N", [(160012, 64, 1), (160012, 64, 4), (160012, 640, 3)])
-def test_gemv_quant_one_warp_path_small_k(M, K, N):
-    # More 32-row units (5001) than the one-warp kernel can have resident at
-    # any occupancy (148 SMs x 32 CTAs), so up to 4 tokens these launches take
-    # that kernel rather than the split-unit one that smaller launches of 1-4
-    # tokens take.  Ragged rows (160012 = 5000 x 32 + 12) and a ragged k-chunk.
+def test_gemv_quant_many_units_small_k(M, K, N):
+    # Many more 32-row units (5001) than CTAs: every CTA takes a range of
+    # several units, its warps a share of their k-chunks.  Ragged rows
+    # (160012 = 5000 x 32 + 12) and a ragged k-chunk.
     W, (packed, alpha) = layer(M, K, M + K + N)
     x = inputs.activations(N, K, seed=K + 7 * N, outlier_frac=0.01)
     y, acc = api.gemv_quant(packed, alpha, x.cuda(), with_acc=True)
@@ -86,10 +85,11 @@ def test_gemv_quant_one_warp_path_small_k(M, K, N):
 
 
 @pytest.mark.parametrize("K", [512, 1024, 1536, 2048, 2560, 6912])
-def test_gemv_quant_split_path_chunk_counts(K):
-    # Small launches of 1-4 tokens: one 4-warp CTA per unit, the unit's
-    # k-chunks split over the warps (1, 2, 3, 4, 5 and 14 chunks: some warps get
-    # none, some one, some several).
+def test_gemv_quant_split_units_chunk_counts(K):
+    # Small launches (7 units, fewer than CTAs): one unit per CTA, the unit's
+    # k-chunks split over the CTA's warps (1, 2, 3, 4, 5 and 14 chunks: some
+    # warps get none, some one, some several, and the warp holding chunk 0 adds
+    # the others' partial sums).
     M, N = 200, 2
     W, (packed, alpha) = layer(M, K, 31 * K + N)
     x = inputs.activations(N, K, seed=K + 3, outlier_frac=0.01)
@@ -167,7 +167,8 @@ def test_gemv_quant_grouped_mixed_k(N):
 
 def test_gemv_quant_grouped_many_problems():
     # 300 layers (two launches), each with its own input, rows of one stacked
-    # activation buffer: every warp re-quantises at each layer boundary
+    # activation buffer: a CTA whose range crosses a layer boundary quantises
+    # the next input before it goes on
     K, M, L = 640, 96, 300
     X = inputs.activations(L, K, seed=61, outlier_frac=0.02)
     W, (packed, alpha) = layer(M, K, 62)
@@ -177,6 +178,29 @@ def test_gemv_quant_grouped_many_problems():
     ref = oracle.bitlinear(W.numpy(), X.numpy())
     assert np.array_equal(torch.cat(accs).cpu().numpy(), ref["acc"])
     assert np.array_equal(torch.cat(ys).cpu().numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("N", [1, 2, 4])
+def test_gemv_quant_ctas_span_several_inputs(N):
+    # 256 layers of 5 units each (1280 units, more than the CTAs of a launch),
+    # each with its own input: CTA ranges cross two or three inputs, which the
+    # CTA quantises one after the other; units split between warps and between
+    # inputs at every boundary.
+    K, M, L = 1024, 160, 256
+    X = inputs.activations(L * N, K, seed=63 + N, outlier_frac=0.02)
+    W, (packed, alpha) = layer(M, K, 64)
+    Xd = X.cuda()
+    ys, accs = api.gemv_quant_grouped([(packed, alpha)] * L,
+                                      [Xd[i * N:(i + 1) * N] for i in range(L)], with_acc=True)
+    codes = oracle.ternarize(W.numpy(), oracle.absmean(W.numpy()))
+    for i in (0, 1, 2, 97, 128, 200, 255):
+        ref = oracle.bitlinear(W.numpy(), X[i * N:(i + 1) * N].numpy())
+        assert np.array_equal(accs[i].cpu().numpy(), ref["acc"]), i
+        assert np.array_equal(ys[i].cpu().numpy(), ref["y"]), i
+    # every layer: the int32 sums against the oracle's integer product
+    q, _, _ = oracle.quant_act(X.numpy())
+    acc_all = oracle.matmul_i32(codes, q)                      # [L*N, M]
+    assert np.array_equal(torch.cat(accs).cpu().numpy(), acc_all)
 
 
 def test_gemv_quant_same_pointer_different_k():
