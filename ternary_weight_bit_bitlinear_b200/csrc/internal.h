@@ -31,6 +31,7 @@ struct DeviceInfo {
   int gemv_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};   // 0: not set up yet
   int tl2_blocks_per_sm[bl::kGemvMaxTokens + 1] = {};    // 0: not set up yet
   bool gq_attr_set[bl::kGemvMaxTokens + 1] = {};
+  int gq_max_dyn[bl::kGemvMaxTokens + 1] = {};            // dynamic shared memory limit
   int gq_area[bl::kGemvMaxTokens + 1][bl::kGqMaxWarps + 1] = {};   // last shared-memory size
   int gq_occ[bl::kGemvMaxTokens + 1][bl::kGqMaxWarps + 1] = {};    // and its CTAs per SM
   bool gemv_split_attr_set[bl::kGemvMaxTokens + 1] = {};

@@ -5,16 +5,40 @@
 namespace blh {
 namespace {
 
-constexpr int kMaxDynSmem = 227 * 1024;
+// Dynamic shared memory a CTA of this kernel may use: the device's opt-in
+// maximum per block less the kernel's static shared memory.
+template <int NT>
+bitlinear_status max_dyn_smem(DeviceInfo* dev, int* out) {
+  auto kernel = bl::gemv_quant_kernel<NT>;
+  if (!dev->gq_attr_set[NT]) {
+    int dev_id = 0, optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaGetDevice(&dev_id) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev_id) !=
+            cudaSuccess ||
+        cudaFuncGetAttributes(&fa, kernel) != cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    const int dyn = optin - static_cast<int>(fa.sharedSizeBytes);
+    if (dyn <= 0 ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) !=
+            cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    dev->gq_max_dyn[NT] = dyn;
+    dev->gq_attr_set[NT] = true;
+  }
+  *out = dev->gq_max_dyn[NT];
+  return BITLINEAR_OK;
+}
 
 template <int NT>
 bitlinear_status occupancy_nt(int warps, int area, DeviceInfo* dev, int* out) {
   auto kernel = bl::gemv_quant_kernel<NT>;
-  if (!dev->gq_attr_set[NT]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) !=
-        cudaSuccess)
-      return BITLINEAR_ERR_CUDA;
-    dev->gq_attr_set[NT] = true;
+  int dyn = 0;
+  bitlinear_status st = max_dyn_smem<NT>(dev, &dyn);
+  if (st != BITLINEAR_OK) return st;
+  if (area > dyn) {
+    *out = 0;
+    return BITLINEAR_OK;
   }
   if (dev->gq_area[NT][warps] != area) {
     int nb = 0;
@@ -31,7 +55,7 @@ bitlinear_status occupancy_nt(int warps, int area, DeviceInfo* dev, int* out) {
 }  // namespace
 
 bitlinear_status gemv_quant_occupancy(int N, int warps, int area, DeviceInfo* dev, int* out) {
-  if (warps < 1 || warps > bl::gq_max_warps(N) || area > kMaxDynSmem) {
+  if (warps < 1 || warps > bl::gq_max_warps(N)) {
     *out = 0;
     return BITLINEAR_OK;
   }
