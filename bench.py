@@ -493,14 +493,18 @@ def measure_crossover(dev, s, reps=30):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     out = {"workload": "8B-shaped layer (q 4096x4096, k/v 1024x4096, o 4096x4096, gate/up "
                        "14336x4096, down 4096x14336), 7 projections per grouped launch",
-           "N": [], "gemv_us": [], "gemm_us": [], "gemv_gbs": [], "gemm_gbs": [],
-           "gemm_tops": []}
+           "N": [], "gemv_us": [], "gemv_quant_us": [], "gemm_us": [], "gemv_gbs": [],
+           "gemm_gbs": [], "gemm_tops": [],
+           "paths": "gemv: CUDA cores on int8 activations; gemv_quant: CUDA cores from fp32 "
+                    "activations, quantiser fused; gemm: tensor cores on int8 activations "
+                    "(A in tensor memory up to 32 tokens)"}
     for N in wl.tokens:
-        xs = {}
+        xs, xf = {}, {}
         for p in (0, 3, 4, 6):
             K = wl.model.ffn if p == 6 else wl.model.hidden
             x = inputs.activations(N, K, inputs.act_seed(SWEEP_CFG, 0, p), device=dev,
                                    outlier_frac=wl.outlier_frac)
+            xf[p] = x
             xs[p] = api.quant_act(x)
         ents = []
         for p, (packed, alpha, M, K) in enumerate(layers):
@@ -508,20 +512,25 @@ def measure_crossover(dev, s, reps=30):
             ents.append((packed, alpha, M, K, xq, am, xsum,
                          torch.empty((N, M), device=dev), None))
         prob = _lib.make_problems(ents)
+        fents = [(packed, alpha, M, K, xf[input_proj(p)], torch.empty((N, M), device=dev), None)
+                 for p, (packed, alpha, M, K) in enumerate(layers)]
+        fprob = _lib.make_fused_problems(fents)
         res = {}
-        for path, fn in (("gemv", _lib.bitlinear_gemv_grouped),
-                         ("gemm", _lib.bitlinear_gemm_grouped)):
-            if path == "gemv" and N > api.GEMV_MAX_TOKENS:
+        for path, fn in (("gemv", lambda: _lib.bitlinear_gemv_grouped(prob, len(ents), N, s)),
+                         ("gemv_quant",
+                          lambda: _lib.bitlinear_gemv_quant_grouped(fprob, len(fents), N, s)),
+                         ("gemm", lambda: _lib.bitlinear_gemm_grouped(prob, len(ents), N, s))):
+            if path != "gemm" and N > api.GEMV_MAX_TOKENS:
                 res[path] = None
                 continue
             for _ in range(3):
-                _lib.check(fn(prob, len(ents), N, s), path)
+                _lib.check(fn(), path)
             tot = 0.0
             for _ in range(reps):
                 flush_l2(flush)
                 a, b = events(2)
                 a.record(s)
-                _lib.check(fn(prob, len(ents), N, s), path)
+                _lib.check(fn(), path)
                 b.record(s)
                 torch.cuda.synchronize()
                 tot += a.elapsed_time(b)
@@ -529,6 +538,8 @@ def measure_crossover(dev, s, reps=30):
         flops = sum(2 * M * N * K for (_, _, M, K) in layers)
         out["N"].append(N)
         out["gemv_us"].append(None if res["gemv"] is None else round(res["gemv"] * 1e3, 2))
+        out["gemv_quant_us"].append(None if res["gemv_quant"] is None else
+                                    round(res["gemv_quant"] * 1e3, 2))
         out["gemm_us"].append(round(res["gemm"] * 1e3, 2))
         out["gemv_gbs"].append(None if res["gemv"] is None else
                                round(packed_bytes / (res["gemv"] * 1e-3) / 1e9, 1))

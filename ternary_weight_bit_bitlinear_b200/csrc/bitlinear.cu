@@ -218,13 +218,15 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
   DeviceInfo* dev = nullptr;
   bitlinear_status st = device_info(&dev);
   if (st != BITLINEAR_OK) return st;
-  // Wide token blocks: 256-token tiles on CTA pairs.  Narrow ones: one CTA per
-  // 128-row tile, 32, 64 or 128 tokens wide -- the narrower the tile, the
-  // smaller its activation stage and the deeper the ring of weight stages the
-  // same shared memory holds (16, 12 or 7), which is what streams the weights
-  // when there are few tokens.
+  // Up to 32 tokens: one 128-row tile of all tokens per CTA, the expanded
+  // weights in tensor memory (gemm_small.cuh), 16 or 32 tokens wide.  Wide
+  // token blocks: 256-token tiles on CTA pairs.  In between: one CTA per
+  // 128-row tile, 64 or 128 tokens wide -- the narrower the tile, the smaller
+  // its activation stage and the deeper the ring of weight stages the same
+  // shared memory holds.
+  const bool small = N <= 32;
   const bool wide = N > 128;
-  const int BN = wide ? bl::kPairBN : N <= 32 ? 32 : N <= 64 ? 64 : 128;
+  const int BN = small ? (N <= 16 ? 16 : 32) : wide ? bl::kPairBN : N <= 64 ? 64 : 128;
   const int BMt = wide ? bl::kPairBM : bl::kGemmBM;
   const int64_t n_tiles = (N + BN - 1) / BN;
   for (int64_t base = 0; base < count; base += bl::kGemmMaxProblems) {
@@ -243,7 +245,7 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     int64_t tiles = 0;
     for (int i = 0; i < n; ++i) {
       const bitlinear_problem& q = probs[base + order[i]];
-      const bool direct = q.M % 4 != 0;
+      const bool direct = small || q.M % 4 != 0;   // the small kernel stores directly
       if (!encode_u8_2d(&p.tmA[i], q.packed, static_cast<uint64_t>(packed_row_words(q.K) * 4),
                         static_cast<uint64_t>(q.M), bl::kGemmPackedRowBytes, bl::kGemmBM,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
@@ -272,7 +274,7 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     p.total_tiles = static_cast<int>(tiles);
     p.wait_ns = blh::wait_limit_ns();
     build_gemm_schedule(p, wide ? dev->sms / 2 : dev->sms);
-    st = blh::launch_gemm(wide ? 1 : BN == 32 ? 2 : BN == 64 ? 3 : 0, p, dev, s);
+    st = blh::launch_gemm(small ? (BN == 16 ? 4 : 5) : wide ? 1 : BN == 64 ? 3 : 0, p, dev, s);
     if (st != BITLINEAR_OK) return st;
   }
   return BITLINEAR_OK;

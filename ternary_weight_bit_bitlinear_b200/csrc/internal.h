@@ -76,7 +76,8 @@ bitlinear_status gemv_quant_launch(int N, int grid, int warps, const bl::GqParam
                                    cudaStream_t s);
 
 // launch_gemm.cu: tensor-core GEMMs.  variant: 0 = 128-token tiles, 1 = CTA
-// pairs, 2 = 32-token tiles, 3 = 64-token tiles.
+// pairs, 3 = 64-token tiles (A unpacked into shared memory); 4 = 16 tokens,
+// 5 = 32 tokens (A in tensor memory).
 bitlinear_status launch_gemm(int variant, const bl::GemmParams& p, DeviceInfo* dev,
                              cudaStream_t s);
 

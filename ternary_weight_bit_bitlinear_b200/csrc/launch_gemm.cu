@@ -1,6 +1,8 @@
 // launch_gemm.cu -- launchers of the tensor-core GEMMs (gemm.cuh: one CTA per
-// 128-row tile; gemm_pair.cuh: CTA pairs per 256 x 256 tile).
+// 128-row tile; gemm_pair.cuh: CTA pairs per 256 x 256 tile; gemm_small.cuh:
+// A in tensor memory for up to 32 tokens).
 #include "internal.h"
+#include "gemm_small.cuh"
 
 namespace blh {
 namespace {
@@ -40,6 +42,23 @@ bitlinear_status launch_pair(const bl::GemmParams& p, DeviceInfo* dev, cudaStrea
   return launch_status();
 }
 
+template <int BN>
+bitlinear_status launch_small(const bl::GemmParams& p, DeviceInfo* dev, int slot,
+                              cudaStream_t s) {
+  auto kernel = bl::gemm_small_kernel<BN>;
+  const int smem = static_cast<int>(sizeof(bl::SmallSmem<BN>)) + 1024;
+  if (!dev->gemm_attr_set[slot]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return BITLINEAR_ERR_CUDA;
+    dev->gemm_attr_set[slot] = true;
+  }
+  const int grid = p.total_tiles < dev->sms ? p.total_tiles : dev->sms;
+  if (launch_pdl(kernel, grid, bl::kSmallThreads, smem, s, p) != cudaSuccess)
+    return BITLINEAR_ERR_CUDA;
+  return launch_status();
+}
+
 }  // namespace
 
 bitlinear_status launch_gemm(int variant, const bl::GemmParams& p, DeviceInfo* dev,
@@ -47,8 +66,9 @@ bitlinear_status launch_gemm(int variant, const bl::GemmParams& p, DeviceInfo* d
   switch (variant) {
     case 0: return launch_single<128, 7>(p, dev, 0, s);
     case 1: return launch_pair<5>(p, dev, s);
-    case 2: return launch_single<32, 16>(p, dev, 2, s);
     case 3: return launch_single<64, 12>(p, dev, 3, s);
+    case 4: return launch_small<16>(p, dev, 4, s);
+    case 5: return launch_small<32>(p, dev, 5, s);
     default: return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   }
 }

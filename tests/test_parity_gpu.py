@@ -276,7 +276,7 @@ def test_gemv_grouped_mixed_k(N):
         assert np.array_equal(y.cpu().numpy(), ref["y"])
 
 
-@pytest.mark.parametrize("N", [1, 100, 512])
+@pytest.mark.parametrize("N", [1, 20, 100, 512])
 def test_gemm_grouped_mixed_k(N):
     shapes = [(512, 1024), (256, 4096), (384, 2816), (128, 128)]
     layers, refs, xq, amax, xsum = _mixed_layers(shapes, N, seed=400 + N)
@@ -298,7 +298,10 @@ def test_gemm_grouped_more_than_one_launch():
 
 @pytest.mark.parametrize("M,K,N", [(128, 128, 1), (256, 512, 200), (384, 1024, 129),
                                    (128, 256, 16), (1024, 2560, 512), (512, 4096, 300),
-                                   (256, 6912, 77)])
+                                   (256, 6912, 77),
+                                   # up to 32 tokens: A in tensor memory, 16 or 32 wide
+                                   (512, 2048, 4), (512, 2048, 25), (256, 14336, 32),
+                                   (200, 1040, 2), (1000, 3072, 17), (4096, 4096, 8)])
 def test_gemm_parity(M, K, N):
     ref, (packed, alpha, xq, amax, xsum) = _layer(M, K, N, seed=3 * M + K + N)
     y, acc = api.gemm(packed, alpha, xq, amax, xsum, with_acc=True)

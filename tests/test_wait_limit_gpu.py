@@ -41,8 +41,9 @@ def _case(M, K, N, seed):
     return W, packed, alpha, x, xq, amax, xsum
 
 
-# N = 32: one CTA per 128-row tile (32-token tiles); N = 256: CTA pairs.
-@pytest.mark.parametrize("M,N", [(128, 32), (256, 256)])
+# N = 32: A in tensor memory (gemm_small); N = 128: one CTA per 128-row tile,
+# A unpacked into shared memory; N = 256: CTA pairs.
+@pytest.mark.parametrize("M,N", [(128, 32), (128, 128), (256, 256)])
 def test_short_limit_times_out_then_recovers(M, N):
     K = 131072
     W, packed, alpha, x, xq, amax, xsum = _case(M, K, N, seed=9100 + N)
