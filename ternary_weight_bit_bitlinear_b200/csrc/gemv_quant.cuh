@@ -264,12 +264,14 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
   };
 
   // L2 prefetch of the first stages (before the wait on the preceding kernel).
+  // The problem cursor only moves forward, so it is put back afterwards: the
+  // prefetched pairs may already reach the next problem.
   if (copy_valid()) {
-    GqItem pi = ii;
+    const int save_pi = ipi;
     int pq = iq;
 #pragma unroll 1
-    for (int st = 0; st < kGqStages - 1 && pq < pi.qe; ++st, ++pq) {
-      const int unit = pi.ub + pq / pi.chunks, kc = pq % pi.chunks;
+    for (int st = 0; st < kGqStages - 1 && pq < ii.qe; ++st, ++pq) {
+      const int unit = ii.ub + pq / ii.chunks, kc = pq % ii.chunks;
       copy_plan_for(unit);
       if (kc * (kGemvChunkBytes / 4) + icp.wword < ipr.W) {
         const uint8_t* src = icp.wsrc + kc * kGemvChunkBytes;
@@ -278,6 +280,8 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
           asm volatile("prefetch.global.L2 [%0];" ::"l"(src + i * icp.wstep) : "memory");
       }
     }
+    ipi = save_pi;
+    iunit = -1;
   }
   pdl_wait_prior_grid();
   pdl_allow_next_grid();

@@ -203,6 +203,25 @@ def test_gemv_quant_ctas_span_several_inputs(N):
     assert np.array_equal(torch.cat(accs).cpu().numpy(), acc_all)
 
 
+@pytest.mark.parametrize("N", [1, 3])
+def test_gemv_quant_many_small_problems_in_segments(N):
+    # 240 problems of 2 units (M = 40) and 3 k-chunks (K = 1536) in segments of
+    # three that share an input (like q, k, v): warp shares start and end at
+    # every position, so a warp's first stages often reach the next problem
+    # and the next segment.
+    K, M, L = 1536, 40, 240
+    X = inputs.activations((L // 3) * N, K, seed=65 + N, outlier_frac=0.02)
+    Ws = [inputs.latent_weights(M, K, seed=1000 + i) for i in range(4)]
+    packs = [api.pack_weights(W.cuda()) for W in Ws]
+    Xd = X.cuda()
+    xs = [Xd[(i // 3) * N:(i // 3 + 1) * N] for i in range(L)]
+    ys, accs = api.gemv_quant_grouped([packs[i % 4] for i in range(L)], xs, with_acc=True)
+    for i in range(L):
+        ref = oracle.bitlinear(Ws[i % 4].numpy(), X[(i // 3) * N:(i // 3 + 1) * N].numpy())
+        assert np.array_equal(accs[i].cpu().numpy(), ref["acc"]), i
+        assert np.array_equal(ys[i].cpu().numpy(), ref["y"]), i
+
+
 def test_gemv_quant_same_pointer_different_k():
     # two layers read prefixes of one buffer with different K: the kernel must
     # quantise each separately (amax is per row of the K it is given)
