@@ -222,9 +222,9 @@ class DecodeStream:
     linear: weights, fp32 inputs per layer, output buffers and the problem
     tables of every call the benchmark makes."""
 
-    def __init__(self, device, cfg, launch_layers=None, int8_path=False, tl2=False):
+    def __init__(self, device, cfg, launch_layers=None, int8_path=False, tl2=False, layers=None):
         wl = inputs.WORKLOADS[cfg]
-        self.cfg, self.shape, self.layers = cfg, wl.model, wl.layers
+        self.cfg, self.shape, self.layers = cfg, wl.model, layers or wl.layers
         self.launch_layers = launch_layers or self.layers
         h, f, L = self.shape.hidden, self.shape.ffn, self.layers
         self.weights = []            # [layer][proj] -> (packed, alpha, M, K)
@@ -412,6 +412,16 @@ class PrefillLayer:
 
 # ----------------------------------------------------------------------------- measurements
 
+def soft(fn, *a, **k):
+    """Run one secondary measurement; a failure becomes a string in the JSON
+    line instead of losing the whole line."""
+    try:
+        return fn(*a, **k)
+    except Exception as exc:  # noqa: BLE001
+        torch.cuda.synchronize()
+        return "failed: %s" % exc
+
+
 def measure_prefill(dev, s, peaks, cfg, N, reps, breakdown=True):
     """One layer at N tokens on the tensor cores: the seven projections in one
     grouped GEMM launch, timed with events around it, L2 flushed before every
@@ -522,6 +532,10 @@ def measure_crossover(dev, s, reps=30):
                          ("gemm", lambda: _lib.bitlinear_gemm_grouped(prob, len(ents), N, s))):
             if path != "gemm" and N > api.GEMV_MAX_TOKENS:
                 res[path] = None
+                continue
+            if path == "gemv_quant" and not all(api.gemv_quant_fits(N, K)
+                                                for (_, _, _, K) in layers):
+                res[path] = None      # the fused kernel's int8 copy of x does not fit
                 continue
             for _ in range(3):
                 _lib.check(fn(), path)
@@ -641,6 +655,27 @@ def run_ours(args, rank, world, local_rank):
     def max_over_ranks(v):
         return rank_max(v, dist, dev)
 
+    if args.only in ("headline", "chain"):
+        # profiling runs: the fused decode step (or the per-group chain) on the
+        # first --layers layers of the 70B-shaped stream, nothing else
+        dec = DecodeStream(dev, HEADLINE_CFG, launch_layers=HEADLINE_LAUNCH_LAYERS,
+                           layers=args.layers)
+        if args.only == "headline":
+            for _ in range(args.warmup):
+                dec.step(s)
+            ms = back_to_back_ms(dec.step, s, args.steps)
+            print(json.dumps({"partial_run": "headline", "layers": dec.layers,
+                              "ms_per_step": round(ms, 5),
+                              "gbs": round(dec.packed_bytes / (ms * 1e-3) / 1e9, 1)}))
+        else:
+            tabs = dec.chain_tables()
+            for _ in range(args.warmup):
+                dec.chain_step(s, tabs)
+            ms = back_to_back_ms(lambda st: dec.chain_step(st, tabs), s, args.steps)
+            print(json.dumps({"partial_run": "chain", "layers": dec.layers,
+                              "ms_per_step": round(ms, 5),
+                              "gbs": round(dec.packed_bytes / (ms * 1e-3) / 1e9, 1)}))
+        return
     if args.only == "prefill":
         print(json.dumps({"partial_run": "prefill",
                           "prefill": measure_prefill(dev, s, peaks, PREFILL_CFG, 512, 20),
@@ -719,9 +754,29 @@ def run_ours(args, rank, world, local_rank):
     del dec
     torch.cuda.empty_cache()
 
-    prefill_70b = measure_prefill(dev, s, peaks, HEADLINE_CFG, 2048, 10, breakdown=False)
+    prefill_70b = soft(measure_prefill, dev, s, peaks, HEADLINE_CFG, 2048, 10, breakdown=False)
+    s2 = soft(measure_stream_2b, dev, s, K, hbm_peak)
+    prefill = soft(measure_prefill, dev, s, peaks, PREFILL_CFG, 512, max(10, min(200, K // 50)))
+    crossover = soft(measure_crossover, dev, s)
+    single = soft(measure_single, dev, s)
 
-    # ================================================================ 2B stream
+    # ---- CPU oracle baseline (rank 0, N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = soft(cpu_baseline, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        emit(args, world, peaks, headline, ms_per_step, gbs, K, K2, e2e_ms, h2d, d2h,
+             prefill_70b, s2, prefill, crossover, single, cpu)
+    assert _lib.bitlinear_device_error(clear=True) == _lib.OK
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure_stream_2b(dev, s, K, hbm_peak):
+    """The 2B-shaped 30-layer stream: fused step, two-step path, per-launch
+    rooflines, the dependent per-group chain and the TL2-style storage."""
     d2 = DecodeStream(dev, STREAM2B_CFG, int8_path=True, tl2=True)
     for _ in range(3):
         d2.step(s)
@@ -789,108 +844,100 @@ def run_ours(args, rank, world, local_rank):
                         "weights_per_s_as_2bit_gbs": round(d2.packed_bytes /
                                                            (per["gemv_tl2"] * 1e-3) / 1e9, 1)},
     })
-    launches_2b = 2 * k2 + k2 * 4 + 3 * 3
+    s2["launches"] = 2 * k2 + k2 * 4 + 3 * 3
     del d2
     torch.cuda.empty_cache()
+    return s2
 
-    prefill = measure_prefill(dev, s, peaks, PREFILL_CFG, 512, max(10, min(200, K // 50)))
-    crossover = measure_crossover(dev, s)
-    single = measure_single(dev, s)
 
-    # ---- CPU oracle baseline (rank 0, N=1 only)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(budget_s=args.cpu_seconds)
-
-    if rank == 0:
-        h = headline
-        sus_gbs = h["packed_bytes"] / (h["sus_ms"] * 1e-3) / 1e9
-        chain_ms = h["chain_ms"]
-        out = {
-            "metric": METRIC,
-            "value": round(gbs, 1),
-            "unit": "GB/s",
-            "n_gpus": world,
-            "steps": K,
-            "warmup": args.warmup,
-            "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "i8",
-            "data": "synthetic (seeded N(0,0.02) latent weights, N(0,1) activations)",
-            "config": {
-                "workload": "70B-shaped decode weight stream: 80 layers x 7 projections "
-                            "(q/o 8192x8192, k/v 1024x8192, gate/up 28672x8192, down "
-                            "8192x28672), N=1",
-                "layers": 80, "tokens": 1,
-                "packed_bytes_per_step": h["packed_bytes"],
-                "launches_per_step": h["ncalls"],
-                "l2": "no flush: 17.11 GB of packed weights per step > 126 MB L2",
-                "parallelism": "replicas" if world > 1 else "single GPU",
-            },
-            "headline_basis": "value = packed weight bytes per step / back-to-back step time "
-                              "(K steps, events at the ends; consecutive launches overlap their "
-                              "start-up through programmatic dependent launch). roofline.achieved "
-                              "= all bytes the fused kernel must move / its mean launch time, "
-                              "events around every launch (no overlap).",
-            "pct_of_measured_hbm": round(100 * gbs / world / hbm_peak, 2),
-            "pct_of_nominal_hbm_8000": round(100 * gbs / world / HBM_NOMINAL_GBS, 2),
-            "roofline": {
-                "bound": "hbm",
-                "kernel": "gemv_quant (fused quantise + GEMV, grouped, 20 layers = 140 linears "
-                          "per launch, K=8192 and 28672)",
-                "achieved": round(h["fused_gbs"], 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(h["fused_gbs"] / hbm_peak, 4),
-                "peak_note": "hbm_gbs %s (burst copy)" % peaks["source"],
-                "bytes_per_launch": round(h["alg_bytes"] / h["ncalls"]),
-                "avg_launch_ms": round(h["launch_ms"], 5),
-                "timing": "events around each launch, %d steps x %d launches" % (K2, h["ncalls"]),
-                "traffic": None,
-                "traffic_note": "ncu DRAM bytes of this kernel on this workload: see profiles/",
-            },
-            "sustained": {
-                "what": "the headline step back to back for >= %.0f s" % SUSTAINED_S,
-                "steps": h["sus_steps"], "ms_per_step": round(h["sus_ms"], 5),
-                "gbs": round(sus_gbs, 1), "frac_of_measured_hbm": round(sus_gbs / hbm_peak, 4),
-                "peak_note": "against hbm_gbs (burst copy); MEASURED_PEAKS has no sustained "
-                             "copy figure",
-                "clocks": h["sclk"],
-            },
-            "decode_chain": {
-                "what": "the same 560 linears in the order a decoder imposes: per layer "
-                        "q/k/v, then o, then gate/up, then down, each group one fused launch "
-                        "(320 launches), one CUDA graph",
-                "ms_per_step": rounded(chain_ms),
-                "gbs": None if isinstance(chain_ms, str) else
-                round(h["packed_bytes"] / (chain_ms * 1e-3) / 1e9, 1),
-                "frac_of_measured_hbm": None if isinstance(chain_ms, str) else
-                round(h["packed_bytes"] / (chain_ms * 1e-3) / 1e9 / hbm_peak, 4),
-            },
-            "e2e": {"value": round(whole_job_gbs(world, h["packed_bytes"], e2e_ms), 1),
-                    "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "how": "per step: pinned host -> device copy of every fp32 layer input, "
-                           "the fused launches, device -> host copy of every output; two buffer "
-                           "sets and two copy streams overlap step i's copies with step i-1's "
-                           "launches"},
-            "prefill_70b": prefill_70b,
-            "prefill": prefill,
-            "stream_2b": s2,
-            "crossover": crossover,
-            "single_1024": single,
-            "gpu_launches": K * h["ncalls"],
-            "gpu_launches_other_passes": {"sustained": h["sus_steps"] * h["ncalls"],
-                                          "per_launch_timing": K2 * h["ncalls"],
-                                          "stream_2b": launches_2b},
-            "clocks": h["clk"],
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(out), flush=True)
-    assert _lib.bitlinear_device_error(clear=True) == _lib.OK
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+def emit(args, world, peaks, h, ms_per_step, gbs, K, K2, e2e_ms, h2d, d2h, prefill_70b, s2,
+         prefill, crossover, single, cpu):
+    """Print the one JSON line (rank 0)."""
+    hbm_peak = peaks["hbm_gbs"]
+    sus_gbs = h["packed_bytes"] / (h["sus_ms"] * 1e-3) / 1e9
+    chain_ms = h["chain_ms"]
+    out = {
+        "metric": METRIC,
+        "value": round(gbs, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "i8",
+        "data": "synthetic (seeded N(0,0.02) latent weights, N(0,1) activations)",
+        "config": {
+            "workload": "70B-shaped decode weight stream: 80 layers x 7 projections "
+                        "(q/o 8192x8192, k/v 1024x8192, gate/up 28672x8192, down "
+                        "8192x28672), N=1",
+            "layers": 80, "tokens": 1,
+            "packed_bytes_per_step": h["packed_bytes"],
+            "launches_per_step": h["ncalls"],
+            "l2": "no flush: 17.11 GB of packed weights per step > 126 MB L2",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+        },
+        "headline_basis": "value = packed weight bytes per step / back-to-back step time "
+                          "(K steps, events at the ends; consecutive launches overlap their "
+                          "start-up through programmatic dependent launch). roofline.achieved "
+                          "= all bytes the fused kernel must move / its mean launch time, "
+                          "events around every launch (no overlap).",
+        "pct_of_measured_hbm": round(100 * gbs / world / hbm_peak, 2),
+        "pct_of_nominal_hbm_8000": round(100 * gbs / world / HBM_NOMINAL_GBS, 2),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "gemv_quant (fused quantise + GEMV, grouped, 20 layers = 140 linears "
+                      "per launch, K=8192 and 28672)",
+            "achieved": round(h["fused_gbs"], 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(h["fused_gbs"] / hbm_peak, 4),
+            "peak_note": "hbm_gbs %s (burst copy)" % peaks["source"],
+            "bytes_per_launch": round(h["alg_bytes"] / h["ncalls"]),
+            "avg_launch_ms": round(h["launch_ms"], 5),
+            "timing": "events around each launch, %d steps x %d launches" % (K2, h["ncalls"]),
+            "traffic": None,
+            "traffic_note": "ncu DRAM bytes of this kernel on this workload: see profiles/",
+        },
+        "sustained": {
+            "what": "the headline step back to back for >= %.0f s" % SUSTAINED_S,
+            "steps": h["sus_steps"], "ms_per_step": round(h["sus_ms"], 5),
+            "gbs": round(sus_gbs, 1), "frac_of_measured_hbm": round(sus_gbs / hbm_peak, 4),
+            "peak_note": "against hbm_gbs (burst copy); MEASURED_PEAKS has no sustained "
+                         "copy figure",
+            "clocks": h["sclk"],
+        },
+        "decode_chain": {
+            "what": "the same 560 linears in the order a decoder imposes: per layer "
+                    "q/k/v, then o, then gate/up, then down, each group one fused launch "
+                    "(320 launches), one CUDA graph",
+            "ms_per_step": rounded(chain_ms),
+            "gbs": None if isinstance(chain_ms, str) else
+            round(h["packed_bytes"] / (chain_ms * 1e-3) / 1e9, 1),
+            "frac_of_measured_hbm": None if isinstance(chain_ms, str) else
+            round(h["packed_bytes"] / (chain_ms * 1e-3) / 1e9 / hbm_peak, 4),
+        },
+        "e2e": {"value": round(whole_job_gbs(world, h["packed_bytes"], e2e_ms), 1),
+                "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "per step: pinned host -> device copy of every fp32 layer input, "
+                       "the fused launches, device -> host copy of every output; two buffer "
+                       "sets and two copy streams overlap step i's copies with step i-1's "
+                       "launches"},
+        "prefill_70b": prefill_70b,
+        "prefill": prefill,
+        "stream_2b": s2,
+        "crossover": crossover,
+        "single_1024": single,
+        "gpu_launches": K * h["ncalls"],
+        "gpu_launches_other_passes": {"sustained": h["sus_steps"] * h["ncalls"],
+                                      "per_launch_timing": K2 * h["ncalls"],
+                                      "stream_2b": s2.get("launches")
+                                      if isinstance(s2, dict) else None},
+        "clocks": h["clk"],
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(out), flush=True)
 
 
 def measure_e2e(dec, s, steps):
@@ -1100,8 +1147,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "crossover"], default="all",
+    ap.add_argument("--only", choices=["all", "headline", "chain", "prefill", "crossover"],
+                    default="all",
                     help="profiling runs: time only one part and print a partial line")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="with --only headline|chain: layers of the 70B-shaped stream (default 80)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
