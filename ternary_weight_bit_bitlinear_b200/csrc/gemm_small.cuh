@@ -15,15 +15,18 @@
 //
 //   warp 0        TMA producer: packed weights (128 rows x 32 bytes) and int8
 //                 activations (BN x 128, 128-byte swizzle) into a deep ring;
-//   warps 4-7     unpackers: warp w owns tensor-memory lanes 32 (w % 4) ..
-//                 +31, one weight row per lane; per k-block it reads its 32
-//                 packed bytes, expands them to 32 words of codes+1 (four int8
-//                 per word, in k order) and stores them with one tcgen05.st
-//                 into one of kSmallABufs A buffers (32 columns each);
+//   warps 4-11    unpackers, in kSmallUnpackGroups groups of four that take
+//                 alternate k-blocks: warp w owns tensor-memory lanes
+//                 32 (w % 4) .. +31, one weight row per lane; per k-block it
+//                 reads its 32 packed bytes, expands them to 32 words of
+//                 codes+1 (four int8 per word, in k order) and stores them with
+//                 one tcgen05.st into one of kSmallABufs A buffers (32 columns
+//                 each).  A store must complete before its buffer is handed to
+//                 the MMA, so one group alone would serialise on that latency;
 //   warp 1        MMA issuer: 4 x tcgen05.mma kind::i8 (K = 32) per k-block,
 //                 A from tensor memory, B from the ring; commits free the ring
 //                 stage and the A buffer; accumulators double-buffered;
-//   warps 2,3,8,9 epilogue, one per lane quarter: tcgen05.ld of BN columns,
+//   warps 2,3,12,13  epilogue, one per lane quarter: tcgen05.ld of BN columns,
 //                 subtract the token's sum of q (the +1 code offset), rescale
 //                 by alpha * amax / 127, store y (lane = row: coalesced).
 //
@@ -37,7 +40,8 @@
 
 namespace bl {
 
-constexpr int kSmallThreads = 10 * 32;
+constexpr int kSmallUnpackGroups = 2;
+constexpr int kSmallThreads = (6 + 4 * kSmallUnpackGroups) * 32;   // 14 warps
 constexpr int kSmallABufs = 14;          // A tiles in tensor memory, 32 columns each
 constexpr int kSmallAColBase = 64;       // after two accumulators of up to 32 columns
 constexpr uint32_t kSmallTmemCols = 512;
@@ -168,17 +172,24 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
       mma_commit(&s.drain);
       mbar_drain(&s.drain, 0);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 4 + 4 * kSmallUnpackGroups) {
     // ------------------------------------------------------------ unpackers
     const uint32_t quarter = static_cast<uint32_t>(warp & 3);
+    const int group = (warp - 4) >> 2;   // takes the k-blocks whose sequence number % groups == group
     const int u = static_cast<int>(quarter) * 32 + lane;   // weight row within the tile
     const int half = (u >> 2) & 1;   // read order of the two 16-byte halves: no bank conflict
     uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
+    int seq = 0;
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-      for (int kb = 0; kb < kblocks; ++kb) {
+      for (int kb = 0; kb < kblocks; ++kb, ++seq) {
+        if (seq % kSmallUnpackGroups != group) {   // the other group's k-block
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+          if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
+          continue;
+        }
         if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
             !mbar_wait(&s.aempty[ab], aphase ^ 1u, abort, p.wait_ns))
           goto unpack_done;
@@ -210,7 +221,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
   unpack_done:;
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
-    const uint32_t quarter = static_cast<uint32_t>(warp & 3);   // warps 2, 3, 8, 9
+    const uint32_t quarter = static_cast<uint32_t>(warp & 3);   // warps 2, 3, 12, 13
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
