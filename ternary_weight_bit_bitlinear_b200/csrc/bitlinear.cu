@@ -15,6 +15,7 @@
 #include <vector>
 
 #include "internal.h"
+#include "gemm_small.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
 
@@ -246,9 +247,12 @@ bitlinear_status gemm_group(const bitlinear_problem* probs, int64_t count, int64
     for (int i = 0; i < n; ++i) {
       const bitlinear_problem& q = probs[base + order[i]];
       const bool direct = small || q.M % 4 != 0;   // the small kernel stores directly
+      // packed weights: one k-block (32 bytes) per row, or for the small kernel
+      // four k-blocks (128 bytes, swizzled) per row
       if (!encode_u8_2d(&p.tmA[i], q.packed, static_cast<uint64_t>(packed_row_words(q.K) * 4),
-                        static_cast<uint64_t>(q.M), bl::kGemmPackedRowBytes, bl::kGemmBM,
-                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
+                        static_cast<uint64_t>(q.M),
+                        small ? bl::kSmallGroupBytes : bl::kGemmPackedRowBytes, bl::kGemmBM,
+                        small ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) ||
           !encode_u8_2d(&p.tmB[i], q.xq, static_cast<uint64_t>(q.K), static_cast<uint64_t>(N),
                         bl::kGemmBK, wide ? bl::kPairHalfN : BN,
                         CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -337,7 +341,7 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
   p.xstride = static_cast<int>((kmax + bl::kGemvChunkK - 1) / bl::kGemvChunkK * bl::kGemvChunkK);
   // CTA size: the most warps resident per SM.
   int best_w = 0, best_per_sm = 0, best_resident = 0;
-  for (int w = 4; w <= bl::gq_max_warps(nt); w += 2) {
+  for (int w = 4; w <= bl::gq_max_warps(nt); ++w) {
     int per_sm = 0;
     bitlinear_status st =
         blh::gemv_quant_occupancy(nt, w, bl::gq_smem_bytes(nt, w, p.xstride), dev, &per_sm);

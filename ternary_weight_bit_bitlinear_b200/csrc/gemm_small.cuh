@@ -10,22 +10,29 @@
 // the prefill GEMM of gemm.cuh is where the expanded weights live: the unpack
 // warps write them from registers straight into tensor memory (tcgen05.st),
 // and the MMAs read A from there, so no expanded tile is written to or read
-// from shared memory.  Shared memory carries only the TMA ring: 4 KB of packed
-// weights and BN x 128 bytes of activations per k-block of 128 weights.
+// from shared memory.
 //
-//   warp 0        TMA producer: packed weights (128 rows x 32 bytes) and int8
-//                 activations (BN x 128, 128-byte swizzle) into a deep ring;
+// The ring moves k-groups of four k-blocks (512 weights): per stage one TMA
+// box of 128 weight rows x 128 packed bytes (128-byte swizzle, so the row
+// reads below are conflict-free) and the group's activation tiles (BN x 128
+// int8 each, 128-byte swizzle).  Whole 128-byte rows keep the number of
+// memory requests per weight byte low: rows 32 bytes wide (one k-block) left
+// DRAM at a seventh of its bandwidth, most of each row's sectors missing L2
+// one 32-byte request at a time.
+//
+//   warp 0        TMA producer;
 //   warps 4-11    unpackers, in kSmallUnpackGroups groups of four that take
-//                 alternate k-blocks: warp w owns tensor-memory lanes
-//                 32 (w % 4) .. +31, one weight row per lane; per k-block it
-//                 reads its 32 packed bytes, expands them to 32 words of
-//                 codes+1 (four int8 per word, in k order) and stores them with
-//                 one tcgen05.st into one of kSmallABufs A buffers (32 columns
-//                 each).  A store must complete before its buffer is handed to
-//                 the MMA, so one group alone would serialise on that latency;
+//                 alternate k-groups: warp w owns tensor-memory lanes
+//                 32 (w % 4) .. +31, one weight row per lane; per k-group it
+//                 reads its row's 128 packed bytes, expands each k-block's 32
+//                 bytes to 32 words of codes+1 (four int8 per word, in k order)
+//                 and stores them with one tcgen05.st into one of kSmallABufs A
+//                 buffers (32 columns each), then waits once for the group's
+//                 stores and hands the buffers to the MMA;
 //   warp 1        MMA issuer: 4 x tcgen05.mma kind::i8 (K = 32) per k-block,
-//                 A from tensor memory, B from the ring; commits free the ring
-//                 stage and the A buffer; accumulators double-buffered;
+//                 A from tensor memory, B from the ring; commits free each A
+//                 buffer and, after a group's last k-block, its ring stage;
+//                 accumulators double-buffered;
 //   warps 2,3,12,13  epilogue, one per lane quarter: tcgen05.ld of BN columns,
 //                 subtract the token's sum of q (the +1 code offset), rescale
 //                 by alpha * amax / 127, store y (lane = row: coalesced).
@@ -42,18 +49,20 @@ namespace bl {
 
 constexpr int kSmallUnpackGroups = 2;
 constexpr int kSmallThreads = (6 + 4 * kSmallUnpackGroups) * 32;   // 14 warps
-constexpr int kSmallABufs = 14;          // A tiles in tensor memory, 32 columns each
+constexpr int kSmallGroupKb = 4;                                   // k-blocks per ring stage
+constexpr int kSmallGroupBytes = kSmallGroupKb * kGemmPackedRowBytes;   // 128 per row
+constexpr int kSmallABufs = 12;          // A tiles in tensor memory, 32 columns each
 constexpr int kSmallAColBase = 64;       // after two accumulators of up to 32 columns
 constexpr uint32_t kSmallTmemCols = 512;
 
-__host__ __device__ constexpr int small_stages(int bn) { return bn <= 16 ? 24 : 20; }
+__host__ __device__ constexpr int small_stages(int bn) { return bn <= 16 ? 8 : 6; }
 
 template <int BN>
 struct SmallSmem {
   static constexpr int S = small_stages(BN);
   // each array up to the barriers is a multiple of 1024 bytes
-  uint8_t b[S][BN * kGemmBK];                          // activations, 128-byte swizzle
-  uint8_t apk[S][kGemmBM * kGemmPackedRowBytes];       // packed weights, 4 KB
+  uint8_t apk[S][kGemmBM * kSmallGroupBytes];          // packed weights, 16 KB, swizzled
+  uint8_t b[S][kSmallGroupKb][BN * kGemmBK];           // activations, 128-byte swizzle
   uint64_t full[S];
   uint64_t empty[S];                                   // MMA commit + 4 unpack warps
   uint64_t afull[kSmallABufs];                         // 4 unpack warps
@@ -78,7 +87,6 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  constexpr uint32_t kStageTx = kGemmBM * kGemmPackedRowBytes + BN * kGemmBK;
   volatile int* abort = &s.abort;
 
   if (threadIdx.x == 0) {
@@ -121,12 +129,16 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
         int pi, m_blk, n_blk;
         gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
         const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallGroupKb) {
+          const int nkb = min(kSmallGroupKb, kblocks - kb0);
           if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort, p.wait_ns)) goto producer_done;
-          mbar_arrive_expect_tx(&s.full[stage], kStageTx);
-          tma_load_2d(s.apk[stage], &p.tmA[pi], &s.full[stage], kb * kGemmPackedRowBytes,
+          mbar_arrive_expect_tx(&s.full[stage],
+                                kGemmBM * kSmallGroupBytes + nkb * BN * kGemmBK);
+          tma_load_2d(s.apk[stage], &p.tmA[pi], &s.full[stage], kb0 * kGemmPackedRowBytes,
                       m_blk * kGemmBM);
-          tma_load_2d(s.b[stage], &p.tmB[pi], &s.full[stage], kb * kGemmBK, n_blk * BN);
+          for (int j = 0; j < nkb; ++j)
+            tma_load_2d(s.b[stage][j], &p.tmB[pi], &s.full[stage], (kb0 + j) * kGemmBK,
+                        n_blk * BN);
           ++issued;
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
@@ -148,23 +160,30 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + db * BN;
         bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
-              !mbar_wait(&s.afull[ab], aphase, abort, p.wait_ns)) {
+        for (int kb0 = 0; kb0 < kblocks && ok; kb0 += kSmallGroupKb) {
+          const int nkb = min(kSmallGroupKb, kblocks - kb0);
+          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t a_tmem = tmem_base + kSmallAColBase + 32 * ab;
-          const uint32_t b_addr = smem_u32(s.b[stage]);
+          for (int j = 0; j < nkb; ++j) {
+            if (!mbar_wait(&s.afull[ab], aphase, abort, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_tmem = tmem_base + kSmallAColBase + 32 * ab;
+            const uint32_t b_addr = smem_u32(s.b[stage][j]);
 #pragma unroll
-          for (int kk = 0; kk < kGemmBK / 32; ++kk)
-            mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_k_sw128(b_addr + 32 * kk), idesc,
-                      (kb | kk) != 0);
+            for (int kk = 0; kk < kGemmBK / 32; ++kk)
+              mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_k_sw128(b_addr + 32 * kk), idesc,
+                        (kb0 + j + kk) != 0);
+            mma_commit(&s.aempty[ab]);
+            if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
+          }
+          if (!ok) break;
           mma_commit(&s.empty[stage]);
-          mma_commit(&s.aempty[ab]);
           if (++stage == S) { stage = 0; phase ^= 1u; }
-          if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
         }
         if (!ok) break;
         mma_commit(&s.tfull[db]);
@@ -175,47 +194,63 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
   } else if (warp >= 4 && warp < 4 + 4 * kSmallUnpackGroups) {
     // ------------------------------------------------------------ unpackers
     const uint32_t quarter = static_cast<uint32_t>(warp & 3);
-    const int group = (warp - 4) >> 2;   // takes the k-blocks whose sequence number % groups == group
+    const int group = (warp - 4) >> 2;   // takes the k-groups whose sequence number % groups == group
     const int u = static_cast<int>(quarter) * 32 + lane;   // weight row within the tile
-    const int half = (u >> 2) & 1;   // read order of the two 16-byte halves: no bank conflict
+    const uint32_t sw = static_cast<uint32_t>(u & 7);       // the row's 128-byte swizzle
+    const uint32_t lane_addr = (quarter * 32u) << 16;
     uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
     int seq = 0;
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-      for (int kb = 0; kb < kblocks; ++kb, ++seq) {
-        if (seq % kSmallUnpackGroups != group) {   // the other group's k-block
+      for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallGroupKb, ++seq) {
+        const int nkb = min(kSmallGroupKb, kblocks - kb0);
+        if (seq % kSmallUnpackGroups != group) {   // the other group's k-group
           if (++stage == S) { stage = 0; phase ^= 1u; }
-          if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
+          ab += nkb;
+          if (ab >= kSmallABufs) { ab -= kSmallABufs; aphase ^= 1u; }
           continue;
         }
-        if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
-            !mbar_wait(&s.aempty[ab], aphase ^ 1u, abort, p.wait_ns))
-          goto unpack_done;
-        tc_fence_after();
-        const uint4* src = reinterpret_cast<const uint4*>(s.apk[stage] + u * kGemmPackedRowBytes);
-        const uint4 h0 = src[half], h1 = src[half ^ 1];
-        const uint4 p0 = half ? h1 : h0, p1 = half ? h0 : h1;
-        const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        uint32_t r[32];
+        if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns)) goto unpack_done;
+        // the row's 128 bytes: 16-byte chunk c at chunk c ^ (row % 8)
+        const uint8_t* row = s.apk[stage] + u * kSmallGroupBytes;
+        uint4 c[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {   // column 4j + i holds weights 16j + 4i .. +3
-          r[4 * j + 0] = words[j] & 0x03030303u;
-          r[4 * j + 1] = (words[j] >> 2) & 0x03030303u;
-          r[4 * j + 2] = (words[j] >> 4) & 0x03030303u;
-          r[4 * j + 3] = (words[j] >> 6) & 0x03030303u;
+        for (int q = 0; q < 8; ++q)
+          c[q] = *reinterpret_cast<const uint4*>(row + ((static_cast<uint32_t>(q) ^ sw) << 4));
+        uint32_t ab_first = ab, aphase_first = aphase;
+#pragma unroll
+        for (int j = 0; j < kSmallGroupKb; ++j) {
+          if (j < nkb) {
+            if (!mbar_wait(&s.aempty[ab], aphase ^ 1u, abort, p.wait_ns)) goto unpack_done;
+            tc_fence_after();
+            const uint32_t words[8] = {c[2 * j].x,     c[2 * j].y,     c[2 * j].z,
+                                       c[2 * j].w,     c[2 * j + 1].x, c[2 * j + 1].y,
+                                       c[2 * j + 1].z, c[2 * j + 1].w};
+            uint32_t r[32];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {   // column 4w + i holds weights 16w + 4i .. +3
+              r[4 * w + 0] = words[w] & 0x03030303u;
+              r[4 * w + 1] = (words[w] >> 2) & 0x03030303u;
+              r[4 * w + 2] = (words[w] >> 4) & 0x03030303u;
+              r[4 * w + 3] = (words[w] >> 6) & 0x03030303u;
+            }
+            tmem_st_32x32b_x32(tmem_base + lane_addr + kSmallAColBase + 32 * ab, r);
+            if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
+          }
         }
-        tmem_st_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + kSmallAColBase + 32 * ab, r);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&s.afull[ab]);
+          for (int j = 0; j < nkb; ++j) {
+            mbar_arrive(&s.afull[ab_first]);
+            if (++ab_first == kSmallABufs) { ab_first = 0; aphase_first ^= 1u; }
+          }
           mbar_arrive(&s.empty[stage]);   // this warp has read its packed rows
         }
         if (++stage == S) { stage = 0; phase ^= 1u; }
-        if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
       }
     }
   unpack_done:;

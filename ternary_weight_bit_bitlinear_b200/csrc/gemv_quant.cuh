@@ -49,7 +49,7 @@ constexpr int kGqStageBytes = kGemvTileRows * kGemvChunkBytes;        // 4 KB of
 constexpr int kGqRingBytes = kGqStages * kGqStageBytes;
 constexpr int kGqMaxProblems = 256;
 constexpr int kGqMaxCtas = 640;
-constexpr int kGqMaxWarps = 16;
+constexpr int kGqMaxWarps = 12;          // 12 x 16 KB of rings already fill shared memory
 constexpr int kGqMaxXBytes = 65536;   // tokens x K (rounded up to 512) held per CTA
 constexpr int kGqRegF4 = 16;          // float4s per thread kept in registers while quantising
 
@@ -132,6 +132,7 @@ __device__ __forceinline__ void gq_quantise_cta(const GqSegment& sg, uint8_t* xs
   const int warp = tid >> 5, lane = tid & 31, nwarps = nthreads >> 5;
   const int K4 = sg.K / 4, P4 = sg.chunks * (kGemvChunkK / 4);
   constexpr int R = kGqRegF4 / NT > 0 ? kGqRegF4 / NT : 1;   // float4s per thread and token
+  constexpr int RB = R > 8 ? 8 : R;   // loads per thread in flight when reading in batches
   const bool in_regs = K4 <= R * nthreads;
   float4 v[NT][R];
   float m[NT];
@@ -149,10 +150,21 @@ __device__ __forceinline__ void gq_quantise_cta(const GqSegment& sg, uint8_t* xs
       }
     }
   } else {
+    // longer rows: batches of RB loads per thread in flight, read again below
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
-      for (int i = tid; i < K4; i += nthreads) m[t] = fmaxf(m[t], absmax4(x4[i]));
+#pragma unroll 1
+      for (int b = tid; b < K4; b += RB * nthreads) {
+        float4 w[RB];
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          const int i = b + j * nthreads;
+          w[j] = i < K4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < RB; ++j) m[t] = fmaxf(m[t], absmax4(w[j]));
+      }
     }
   }
 #pragma unroll
@@ -179,8 +191,20 @@ __device__ __forceinline__ void gq_quantise_cta(const GqSegment& sg, uint8_t* xs
       }
     } else {
       const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
-      for (int i = tid; i < K4; i += nthreads)
-        out[i] = mt == 0.0f ? 0u : quant_pack4(x4[i], s, sum[t]);
+#pragma unroll 1
+      for (int b = tid; b < K4; b += RB * nthreads) {
+        float4 w[RB];
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          const int i = b + j * nthreads;
+          w[j] = i < K4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          const int i = b + j * nthreads;
+          if (i < K4) out[i] = mt == 0.0f ? 0u : quant_pack4(w[j], s, sum[t]);
+        }
+      }
     }
     for (int i = K4 + tid; i < P4; i += nthreads) out[i] = 0u;
 #pragma unroll
@@ -213,7 +237,7 @@ __device__ __forceinline__ void gq_epilogue(const GqProblem& pr, int row, const 
   }
 }
 
-// Warps a CTA may have: up to 16 for 1..4 tokens; 4 beyond, where each
+// Warps a CTA may have: up to 12 for 1..4 tokens; 4 beyond, where each
 // thread's accumulators take most of its registers.
 __host__ __device__ constexpr int gq_max_warps(int nt) { return nt <= 4 ? kGqMaxWarps : 4; }
 
@@ -237,10 +261,13 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
                                         [&](int i) { return p.seg[i].unit_begin; })
                            : 0;
 
-  // ---- copy side: this warp's pairs, item after item, kGqStages - 1 ahead
+  // ---- copy side: this warp's pairs, item after item, kGqStages - 1 ahead.
+  // (iu, ikc) is the unit and k-chunk of pair iq of the current item, kept
+  // incrementally: one division per item, none per pair.
   int iseg = seg0;
   GqItem ii = gq_item(p, iseg, u0, u1, warp, nwarps);
   int iq = ii.qb;
+  int iu = ii.ub + ii.qb / ii.chunks, ikc = ii.qb % ii.chunks;
   int ipi = p.seg[iseg].prob_begin;
   int iunit = -1;
   GqProblem ipr;
@@ -252,6 +279,8 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
       if (ii.ue >= u1 || iseg + 1 >= p.num_segments) return false;
       ii = gq_item(p, ++iseg, u0, u1, warp, nwarps);
       iq = ii.qb;
+      iu = ii.ub + ii.qb / ii.chunks;
+      ikc = ii.qb % ii.chunks;
     }
     return u0 < u1;
   };
@@ -268,17 +297,17 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
   // prefetched pairs may already reach the next problem.
   if (copy_valid()) {
     const int save_pi = ipi;
-    int pq = iq;
+    int pq = iq, pu = iu, pkc = ikc;
 #pragma unroll 1
     for (int st = 0; st < kGqStages - 1 && pq < ii.qe; ++st, ++pq) {
-      const int unit = ii.ub + pq / ii.chunks, kc = pq % ii.chunks;
-      copy_plan_for(unit);
-      if (kc * (kGemvChunkBytes / 4) + icp.wword < ipr.W) {
-        const uint8_t* src = icp.wsrc + kc * kGemvChunkBytes;
+      copy_plan_for(pu);
+      if (pkc * (kGemvChunkBytes / 4) + icp.wword < ipr.W) {
+        const uint8_t* src = icp.wsrc + pkc * kGemvChunkBytes;
 #pragma unroll 1
         for (int i = 0; i < icp.vrows; ++i)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(src + i * icp.wstep) : "memory");
       }
+      if (++pkc == ii.chunks) { pkc = 0; ++pu; }
     }
     ipi = save_pi;
     iunit = -1;
@@ -290,10 +319,10 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
   int slot = 0;
   auto issue_next = [&]() {
     if (copy_valid()) {
-      const int unit = ii.ub + iq / ii.chunks, kc = iq % ii.chunks;
-      copy_plan_for(unit);
-      gemv_issue_weights(ipr.W, icp, kc, ring + slot * kGqStageBytes);
+      copy_plan_for(iu);
+      gemv_issue_weights(ipr.W, icp, ikc, ring + slot * kGqStageBytes);
       ++iq;
+      if (++ikc == ii.chunks) { ikc = 0; ++iu; }
     }
     cp_async_commit();   // one group per stage, empty once the sequence is done
     slot = (slot + 1) & (kGqStages - 1);
