@@ -51,9 +51,19 @@ constexpr int kSmallUnpackGroups = 2;
 constexpr int kSmallThreads = (6 + 4 * kSmallUnpackGroups) * 32;   // 14 warps
 constexpr int kSmallGroupKb = 4;                                   // k-blocks per ring stage
 constexpr int kSmallGroupBytes = kSmallGroupKb * kGemmPackedRowBytes;   // 128 per row
-constexpr int kSmallABufs = 12;          // A tiles in tensor memory, 32 columns each
-constexpr int kSmallAColBase = 64;       // after two accumulators of up to 32 columns
+// Each tile accumulates into kSmallAcc independent accumulators (MMA kk of every
+// k-block into accumulator kk), summed in the epilogue: consecutive MMAs then
+// do not wait for each other's result, which short MMAs (N = 16 or 32) would
+// otherwise do once per K = 32 step.
+constexpr int kSmallAcc = 4;
+static_assert(kSmallAcc == kGemmBK / 32, "one accumulator per K = 32 step of a k-block");
 constexpr uint32_t kSmallTmemCols = 512;
+// Tensor memory: two sets of kSmallAcc accumulators of BN columns, then the A
+// buffers (32 columns each) in what is left.
+__host__ __device__ constexpr int small_acol_base(int bn) { return 2 * kSmallAcc * bn; }
+__host__ __device__ constexpr int small_abufs(int bn) {
+  return (static_cast<int>(kSmallTmemCols) - small_acol_base(bn)) / 32;
+}
 
 __host__ __device__ constexpr int small_stages(int bn) { return bn <= 16 ? 8 : 6; }
 
@@ -65,8 +75,8 @@ struct SmallSmem {
   uint8_t b[S][kSmallGroupKb][BN * kGemmBK];           // activations, 128-byte swizzle
   uint64_t full[S];
   uint64_t empty[S];                                   // MMA commit + 4 unpack warps
-  uint64_t afull[kSmallABufs];                         // 4 unpack warps
-  uint64_t aempty[kSmallABufs];                        // MMA commit
+  uint64_t afull[small_abufs(BN)];                     // 4 unpack warps
+  uint64_t aempty[small_abufs(BN)];                    // MMA commit
   uint64_t tfull[2];
   uint64_t tempty[2];                                  // 4 epilogue warps
   uint64_t drain;
@@ -80,6 +90,8 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Smem = SmallSmem<BN>;
   constexpr int S = Smem::S;
+  constexpr int kSmallABufs = small_abufs(BN);
+  constexpr uint32_t kSmallAColBase = small_acol_base(BN);
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
   const uint32_t base = smem_u32(smem_raw);
@@ -158,7 +170,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
         const uint32_t db = ti & 1, dp = (ti >> 1) & 1;
         if (!mbar_wait(&s.tempty[db], dp ^ 1u, abort, p.wait_ns)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + db * BN;
+        const uint32_t d_tmem = tmem_base + db * kSmallAcc * BN;
         bool ok = true;
         for (int kb0 = 0; kb0 < kblocks && ok; kb0 += kSmallGroupKb) {
           const int nkb = min(kSmallGroupKb, kblocks - kb0);
@@ -175,9 +187,9 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
             const uint32_t a_tmem = tmem_base + kSmallAColBase + 32 * ab;
             const uint32_t b_addr = smem_u32(s.b[stage][j]);
 #pragma unroll
-            for (int kk = 0; kk < kGemmBK / 32; ++kk)
-              mma_i8_ts(d_tmem, a_tmem + 8 * kk, smem_desc_k_sw128(b_addr + 32 * kk), idesc,
-                        (kb0 + j + kk) != 0);
+            for (int kk = 0; kk < kGemmBK / 32; ++kk)   // accumulator kk (kSmallAcc == 4)
+              mma_i8_ts(d_tmem + kk * BN, a_tmem + 8 * kk, smem_desc_k_sw128(b_addr + 32 * kk),
+                        idesc, (kb0 + j) != 0);
             mma_commit(&s.aempty[ab]);
             if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
           }
@@ -273,11 +285,20 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
       if (!mbar_wait(&s.tfull[db], dp, abort, p.wait_ns)) break;
       tc_fence_after();
       uint32_t r[BN];
-      const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + db * BN;
-      if constexpr (BN == 16) {
-        tmem_ld_32x32b_x16(taddr, r);
-      } else {
-        tmem_ld_32x32b_x32(taddr, r);
+      const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + db * kSmallAcc * BN;
+#pragma unroll
+      for (int j = 0; j < BN; ++j) r[j] = 0;
+#pragma unroll
+      for (int a = 0; a < kSmallAcc; ++a) {   // the accumulators' int32 sums
+        uint32_t t[BN];
+        if constexpr (BN == 16) {
+          tmem_ld_32x32b_x16(taddr + a * BN, t);
+        } else {
+          tmem_ld_32x32b_x32(taddr + a * BN, t);
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < BN; ++j) r[j] += t[j];
       }
       tmem_ld_wait();
       tc_fence_before();
