@@ -339,42 +339,36 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
   p.num_problems = n;
   p.num_segments = segs;
   p.xstride = static_cast<int>((kmax + bl::kGemvChunkK - 1) / bl::kGemvChunkK * bl::kGemvChunkK);
-  // CTA size: the most warps resident per SM.
-  int best_w = 0, best_per_sm = 0, best_resident = 0;
+  // CTA size: the most warps resident per SM, among sizes that fit at least
+  // two CTAs per SM when there are any (a CTA that starts on an SM quantises
+  // its input while the other one streams weights); fewest warps on a tie.
+  int best_w = 0, best_per_sm = 0, best_score = 0;
   for (int w = 4; w <= bl::gq_max_warps(nt); ++w) {
     int per_sm = 0;
     bitlinear_status st =
         blh::gemv_quant_occupancy(nt, w, bl::gq_smem_bytes(nt, w, p.xstride), dev, &per_sm);
     if (st != BITLINEAR_OK) return st;
-    if (per_sm * w > best_resident) {
-      best_resident = per_sm * w;
+    const int score = per_sm * w + (per_sm >= 2 ? 1000 : 0);
+    if (per_sm > 0 && score > best_score) {
+      best_score = score;
       best_w = w;
       best_per_sm = per_sm;
     }
   }
   if (best_w == 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   p.area = bl::gq_smem_bytes(nt, best_w, p.xstride);
-  int64_t ctas = std::min<int64_t>(static_cast<int64_t>(dev->sms) * best_per_sm, units);
-  ctas = std::min<int64_t>(ctas, bl::kGqMaxCtas);
-  // Unit ranges: CTA c starts at the first unit whose pairs-before count
-  // reaches c * total / ctas (rounded to the nearer unit boundary); empty
-  // ranges are dropped.
+  // kGqOversub CTAs per resident slot (at most one per unit), so that SMs that
+  // drain their first range early take later ones.
+  p.total_units = static_cast<int>(units);
   int64_t total = 0;
-  for (int64_t v : seg_pairs) total += v;
-  int g = 0;
-  p.bounds[0] = 0;
-  int sg = 0;
-  int64_t seg_pair_begin = 0;
-  for (int64_t c = 1; c < ctas; ++c) {
-    const int64_t t = total * c / ctas;
-    while (sg + 1 < segs && seg_pair_begin + seg_pairs[sg] <= t) seg_pair_begin += seg_pairs[sg++];
-    const int64_t C = p.seg[sg].chunks;
-    const int64_t u = p.seg[sg].unit_begin + (t - seg_pair_begin + C / 2) / C;
-    const int b = static_cast<int>(std::min<int64_t>(u, units));
-    if (b > p.bounds[g]) p.bounds[++g] = b;
+  for (int g = 0; g < segs; ++g) {
+    p.seg[g].pair_begin = total;
+    total += seg_pairs[g];
   }
-  if (units > p.bounds[g]) p.bounds[++g] = static_cast<int>(units);
-  *grid = g;
+  p.total_pairs = total;
+  const int64_t slots = static_cast<int64_t>(dev->sms) * best_per_sm;
+  *grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(slots * bl::kGqOversub, units),
+                                             INT_MAX / 2));
   *warps = best_w;
   return BITLINEAR_OK;
 }

@@ -13,10 +13,16 @@
 // problems that read the same input (pointer and K -- q, k and v, or gate and
 // up, given side by side).  A unit is 32 rows of one problem over all of its K,
 // and a pair is one unit and one k-chunk of 512 weights (128 bytes per row), so
-// a segment holds units x ceil(K / 512) pairs.  The host cuts the launch's
-// units into one contiguous range per CTA with about the same number of pairs
-// each (bounds[]).  A CTA's range meets one or more segments; each such
-// meeting is an item, and the CTA takes its items in order:
+// a segment holds units x ceil(K / 512) pairs.  The launch's units are cut
+// into one contiguous range per CTA with about the same number of pairs each:
+// CTA c starts at the unit nearest to pair (total pairs) x c / (CTAs), which
+// every CTA computes from the segment table.  The host launches several
+// times more CTAs than fit on the GPU at once (kGqOversub), so the block
+// scheduler hands the later ranges to whichever SMs finish first: SMs do not
+// all draw the same share of HBM bandwidth, and equal static shares left the
+// slowest SMs finishing a quarter of a launch after the fastest.  A CTA's
+// range meets one or more segments; each such meeting is an item, and the
+// CTA takes its items in order:
 //   1. all its threads quantise the item's input, once, into the CTA's int8
 //      copy in shared memory (amax and the sum of q per token reduced across
 //      the CTA);
@@ -48,7 +54,7 @@ constexpr int kGqStages = 4;                                          // power o
 constexpr int kGqStageBytes = kGemvTileRows * kGemvChunkBytes;        // 4 KB of weights
 constexpr int kGqRingBytes = kGqStages * kGqStageBytes;
 constexpr int kGqMaxProblems = 256;
-constexpr int kGqMaxCtas = 640;
+constexpr int kGqOversub = 4;         // CTAs launched per CTA slot of the GPU
 constexpr int kGqMaxWarps = 12;          // 12 x 16 KB of rings already fill shared memory
 constexpr int kGqMaxXBytes = 65536;   // tokens x K (rounded up to 512) held per CTA
 constexpr int kGqRegF4 = 16;          // float4s per thread kept in registers while quantising
@@ -69,12 +75,14 @@ struct GqSegment {
   int chunks;              // k-chunks per unit: ceil(K / 512)
   int unit_begin, units;   // the segment's units, numbered across the launch
   int prob_begin;          // first problem of the segment
+  long long pair_begin;    // (unit, k-chunk) pairs of the segments before this one
 };
 
 struct GqParams {
   GqProblem prob[kGqMaxProblems];
   GqSegment seg[kGqMaxProblems];
-  int bounds[kGqMaxCtas + 1];   // CTA c takes units [bounds[c], bounds[c+1])
+  long long total_pairs;
+  int total_units;
   int num_problems;
   int num_segments;
   int xstride;             // bytes per token of the int8 copy: 512 x the launch's largest chunks
@@ -98,6 +106,22 @@ __device__ __forceinline__ int gq_last_le(int n, int v, F begin) {
     if (begin(mid) <= v) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+// First unit of CTA c's range (c in [0, ctas]): the unit boundary nearest to
+// pair total_pairs * c / ctas.  Nondecreasing in c; 0 at c = 0 and every unit
+// at c = ctas.  The host sizes the grid with the same rule in mind (a CTA
+// whose range comes out empty returns at once).
+__device__ __forceinline__ int gq_unit_bound(const GqParams& p, int c, int ctas) {
+  if (c <= 0) return 0;
+  if (c >= ctas) return p.total_units;
+  const long long t = p.total_pairs * c / ctas;
+  const int sg = gq_last_le(p.num_segments, 0, [&](int i) {
+    return p.seg[i].pair_begin <= t ? 0 : 1;   // segments whose pairs start at or before t
+  });
+  const long long C = p.seg[sg].chunks;
+  const long long u = p.seg[sg].unit_begin + (t - p.seg[sg].pair_begin + C / 2) / C;
+  return static_cast<int>(u < p.total_units ? u : p.total_units);
 }
 
 // One item of a CTA: the units [ub, ue) of segment `seg`, `chunks` k-chunks
@@ -256,7 +280,8 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
   int* part_all = reinterpret_cast<int*>(smem + NT * p.xstride);
   uint8_t* ring = smem + NT * p.xstride + gq_partial_bytes(NT, nwarps) + warp * kGqRingBytes;
 
-  const int u0 = p.bounds[blockIdx.x], u1 = p.bounds[blockIdx.x + 1];
+  const int u0 = gq_unit_bound(p, blockIdx.x, gridDim.x);
+  const int u1 = gq_unit_bound(p, blockIdx.x + 1, gridDim.x);
   const int seg0 = u0 < u1 ? gq_last_le(p.num_segments, u0,
                                         [&](int i) { return p.seg[i].unit_begin; })
                            : 0;
