@@ -678,9 +678,17 @@ def run_ours(args, rank, world, local_rank):
         return
     if args.only == "prefill":
         print(json.dumps({"partial_run": "prefill",
-                          "prefill": measure_prefill(dev, s, peaks, PREFILL_CFG, 512, 20),
-                          "prefill_70b": measure_prefill(dev, s, peaks, HEADLINE_CFG, 2048, 10,
-                                                         breakdown=False)}))
+                          "prefill": measure_prefill(dev, s, peaks, PREFILL_CFG, 512,
+                                                     args.steps)}))
+        return
+    if args.only == "prefill70":
+        print(json.dumps({"partial_run": "prefill70",
+                          "prefill_70b": measure_prefill(dev, s, peaks, HEADLINE_CFG, 2048,
+                                                         args.steps, breakdown=False)}))
+        return
+    if args.only == "stream2b":
+        print(json.dumps({"partial_run": "stream2b",
+                          "stream_2b": measure_stream_2b(dev, s, args.steps, hbm_peak)}))
         return
     if args.only == "crossover":
         print(json.dumps({"partial_run": "crossover", "crossover": measure_crossover(dev, s)}))
@@ -1147,7 +1155,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "headline", "chain", "prefill", "crossover"],
+    ap.add_argument("--only", choices=["all", "headline", "chain", "prefill", "prefill70",
+                                       "stream2b", "crossover"],
                     default="all",
                     help="profiling runs: time only one part and print a partial line")
     ap.add_argument("--layers", type=int, default=None,

@@ -357,8 +357,11 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
   }
   if (best_w == 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   p.area = bl::gq_smem_bytes(nt, best_w, p.xstride);
-  // kGqOversub CTAs per resident slot (at most one per unit), so that SMs that
-  // drain their first range early take later ones.
+  // Up to kGqOversub CTAs per resident slot, so that SMs that drain their
+  // first range early take later ones -- but only while every warp keeps at
+  // least kGqMinPairsPerWarp pairs: each CTA quantises its inputs once, and on
+  // short launches (a decoder's per-group launches) more CTAs only repeat that
+  // work.  At most one CTA per unit.
   p.total_units = static_cast<int>(units);
   int64_t total = 0;
   for (int g = 0; g < segs; ++g) {
@@ -367,8 +370,9 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
   }
   p.total_pairs = total;
   const int64_t slots = static_cast<int64_t>(dev->sms) * best_per_sm;
-  *grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(slots * bl::kGqOversub, units),
-                                             INT_MAX / 2));
+  const int64_t by_work = total / (static_cast<int64_t>(best_w) * bl::kGqMinPairsPerWarp);
+  const int64_t ctas = std::max<int64_t>(slots, std::min<int64_t>(by_work, slots * bl::kGqOversub));
+  *grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(ctas, units), INT_MAX / 2));
   *warps = best_w;
   return BITLINEAR_OK;
 }

@@ -26,13 +26,14 @@
 //                 32 (w % 4) .. +31, one weight row per lane; per k-group it
 //                 reads its row's 128 packed bytes, expands each k-block's 32
 //                 bytes to 32 words of codes+1 (four int8 per word, in k order)
-//                 and stores them with one tcgen05.st into one of kSmallABufs A
-//                 buffers (32 columns each), then waits once for the group's
-//                 stores and hands the buffers to the MMA;
+//                 and stores them with one tcgen05.st into one of the four A
+//                 buffers (32 columns each) of the group's slot, then waits once
+//                 for the group's stores and hands the slot to the MMA;
 //   warp 1        MMA issuer: 4 x tcgen05.mma kind::i8 (K = 32) per k-block,
-//                 A from tensor memory, B from the ring; commits free each A
-//                 buffer and, after a group's last k-block, its ring stage;
-//                 accumulators double-buffered;
+//                 A from tensor memory, B from the ring; one commit per k-group
+//                 frees the A slot and one its ring stage (barrier waits and
+//                 commits, not the MMAs, took most of this thread's time when
+//                 they were per k-block); accumulators double-buffered;
 //   warps 2,3,12,13  epilogue, one per lane quarter: tcgen05.ld of BN columns,
 //                 subtract the token's sum of q (the +1 code offset), rescale
 //                 by alpha * amax / 127, store y (lane = row: coalesced).
@@ -64,6 +65,8 @@ __host__ __device__ constexpr int small_acol_base(int bn) { return 2 * kSmallAcc
 __host__ __device__ constexpr int small_abufs(int bn) {
   return (static_cast<int>(kSmallTmemCols) - small_acol_base(bn)) / 32;
 }
+// A slots: the four A buffers of one k-group.
+__host__ __device__ constexpr int small_aslots(int bn) { return small_abufs(bn) / kSmallGroupKb; }
 
 __host__ __device__ constexpr int small_stages(int bn) { return bn <= 16 ? 8 : 6; }
 
@@ -75,8 +78,8 @@ struct SmallSmem {
   uint8_t b[S][kSmallGroupKb][BN * kGemmBK];           // activations, 128-byte swizzle
   uint64_t full[S];
   uint64_t empty[S];                                   // MMA commit + 4 unpack warps
-  uint64_t afull[small_abufs(BN)];                     // 4 unpack warps
-  uint64_t aempty[small_abufs(BN)];                    // MMA commit
+  uint64_t afull[small_aslots(BN)];                    // 4 unpack warps
+  uint64_t aempty[small_aslots(BN)];                   // MMA commit
   uint64_t tfull[2];
   uint64_t tempty[2];                                  // 4 epilogue warps
   uint64_t drain;
@@ -90,7 +93,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Smem = SmallSmem<BN>;
   constexpr int S = Smem::S;
-  constexpr int kSmallABufs = small_abufs(BN);
+  constexpr int kSlots = small_aslots(BN);
   constexpr uint32_t kSmallAColBase = small_acol_base(BN);
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
@@ -106,7 +109,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1 + 4);
     }
-    for (int i = 0; i < kSmallABufs; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(&s.afull[i], 4);
       mbar_init(&s.aempty[i], 1);
     }
@@ -162,7 +165,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
-      uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
+      uint32_t stage = 0, phase = 0, slot = 0, sphase = 0;
       for (int ti = 0; ti < ntiles; ++ti) {
         int pi, m_blk, n_blk;
         gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
@@ -172,30 +175,26 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + db * kSmallAcc * BN;
         bool ok = true;
-        for (int kb0 = 0; kb0 < kblocks && ok; kb0 += kSmallGroupKb) {
+        for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallGroupKb) {
           const int nkb = min(kSmallGroupKb, kblocks - kb0);
-          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns)) {
+          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
+              !mbar_wait(&s.afull[slot], sphase, abort, p.wait_ns)) {
             ok = false;
             break;
           }
+          tc_fence_after();
+          const uint32_t a_slot = tmem_base + kSmallAColBase + 32 * kSmallGroupKb * slot;
           for (int j = 0; j < nkb; ++j) {
-            if (!mbar_wait(&s.afull[ab], aphase, abort, p.wait_ns)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a_tmem = tmem_base + kSmallAColBase + 32 * ab;
             const uint32_t b_addr = smem_u32(s.b[stage][j]);
 #pragma unroll
             for (int kk = 0; kk < kGemmBK / 32; ++kk)   // accumulator kk (kSmallAcc == 4)
-              mma_i8_ts(d_tmem + kk * BN, a_tmem + 8 * kk, smem_desc_k_sw128(b_addr + 32 * kk),
-                        idesc, (kb0 + j) != 0);
-            mma_commit(&s.aempty[ab]);
-            if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
+              mma_i8_ts(d_tmem + kk * BN, a_slot + 32 * j + 8 * kk,
+                        smem_desc_k_sw128(b_addr + 32 * kk), idesc, (kb0 + j) != 0);
           }
-          if (!ok) break;
+          mma_commit(&s.aempty[slot]);
           mma_commit(&s.empty[stage]);
           if (++stage == S) { stage = 0; phase ^= 1u; }
+          if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
         }
         if (!ok) break;
         mma_commit(&s.tfull[db]);
@@ -210,7 +209,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
     const int u = static_cast<int>(quarter) * 32 + lane;   // weight row within the tile
     const uint32_t sw = static_cast<uint32_t>(u & 7);       // the row's 128-byte swizzle
     const uint32_t lane_addr = (quarter * 32u) << 16;
-    uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
+    uint32_t stage = 0, phase = 0, slot = 0, sphase = 0;
     int seq = 0;
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
@@ -218,51 +217,46 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallGroupKb, ++seq) {
         const int nkb = min(kSmallGroupKb, kblocks - kb0);
-        if (seq % kSmallUnpackGroups != group) {   // the other group's k-group
-          if (++stage == S) { stage = 0; phase ^= 1u; }
-          ab += nkb;
-          if (ab >= kSmallABufs) { ab -= kSmallABufs; aphase ^= 1u; }
-          continue;
-        }
-        if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns)) goto unpack_done;
-        // the row's 128 bytes: 16-byte chunk c at chunk c ^ (row % 8)
-        const uint8_t* row = s.apk[stage] + u * kSmallGroupBytes;
-        uint4 c[8];
+        if (seq % kSmallUnpackGroups == group) {
+          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
+              !mbar_wait(&s.aempty[slot], sphase ^ 1u, abort, p.wait_ns))
+            goto unpack_done;
+          tc_fence_after();
+          // the row's 128 bytes: 16-byte chunk c at chunk c ^ (row % 8)
+          const uint8_t* row = s.apk[stage] + u * kSmallGroupBytes;
+          uint4 c[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          c[q] = *reinterpret_cast<const uint4*>(row + ((static_cast<uint32_t>(q) ^ sw) << 4));
-        uint32_t ab_first = ab, aphase_first = aphase;
+          for (int q = 0; q < 8; ++q)
+            c[q] = *reinterpret_cast<const uint4*>(row + ((static_cast<uint32_t>(q) ^ sw) << 4));
+          const uint32_t a_slot =
+              tmem_base + lane_addr + kSmallAColBase + 32 * kSmallGroupKb * slot;
 #pragma unroll
-        for (int j = 0; j < kSmallGroupKb; ++j) {
-          if (j < nkb) {
-            if (!mbar_wait(&s.aempty[ab], aphase ^ 1u, abort, p.wait_ns)) goto unpack_done;
-            tc_fence_after();
-            const uint32_t words[8] = {c[2 * j].x,     c[2 * j].y,     c[2 * j].z,
-                                       c[2 * j].w,     c[2 * j + 1].x, c[2 * j + 1].y,
-                                       c[2 * j + 1].z, c[2 * j + 1].w};
-            uint32_t r[32];
+          for (int j = 0; j < kSmallGroupKb; ++j) {
+            if (j < nkb) {
+              const uint32_t words[8] = {c[2 * j].x,     c[2 * j].y,     c[2 * j].z,
+                                         c[2 * j].w,     c[2 * j + 1].x, c[2 * j + 1].y,
+                                         c[2 * j + 1].z, c[2 * j + 1].w};
+              uint32_t r[32];
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {   // column 4w + i holds weights 16w + 4i .. +3
-              r[4 * w + 0] = words[w] & 0x03030303u;
-              r[4 * w + 1] = (words[w] >> 2) & 0x03030303u;
-              r[4 * w + 2] = (words[w] >> 4) & 0x03030303u;
-              r[4 * w + 3] = (words[w] >> 6) & 0x03030303u;
+              for (int w = 0; w < 8; ++w) {   // column 4w + i holds weights 16w + 4i .. +3
+                r[4 * w + 0] = words[w] & 0x03030303u;
+                r[4 * w + 1] = (words[w] >> 2) & 0x03030303u;
+                r[4 * w + 2] = (words[w] >> 4) & 0x03030303u;
+                r[4 * w + 3] = (words[w] >> 6) & 0x03030303u;
+              }
+              tmem_st_32x32b_x32(a_slot + 32 * j, r);
             }
-            tmem_st_32x32b_x32(tmem_base + lane_addr + kSmallAColBase + 32 * ab, r);
-            if (++ab == kSmallABufs) { ab = 0; aphase ^= 1u; }
           }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          for (int j = 0; j < nkb; ++j) {
-            mbar_arrive(&s.afull[ab_first]);
-            if (++ab_first == kSmallABufs) { ab_first = 0; aphase_first ^= 1u; }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&s.afull[slot]);
+            mbar_arrive(&s.empty[stage]);   // this warp has read its packed rows
           }
-          mbar_arrive(&s.empty[stage]);   // this warp has read its packed rows
         }
         if (++stage == S) { stage = 0; phase ^= 1u; }
+        if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
       }
     }
   unpack_done:;
