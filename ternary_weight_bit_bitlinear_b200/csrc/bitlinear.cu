@@ -369,9 +369,12 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
     total += seg_pairs[g];
   }
   p.total_pairs = total;
+  // A whole number of waves (a partial extra wave would leave a tail).
   const int64_t slots = static_cast<int64_t>(dev->sms) * best_per_sm;
-  const int64_t by_work = total / (static_cast<int64_t>(best_w) * bl::kGqMinPairsPerWarp);
-  const int64_t ctas = std::max<int64_t>(slots, std::min<int64_t>(by_work, slots * bl::kGqOversub));
+  const int64_t waves = std::max<int64_t>(
+      1, std::min<int64_t>(bl::kGqOversub,
+                           total / (slots * best_w * bl::kGqMinPairsPerWarp)));
+  const int64_t ctas = slots * waves;
   *grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(ctas, units), INT_MAX / 2));
   *warps = best_w;
   return BITLINEAR_OK;
