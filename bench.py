@@ -49,6 +49,7 @@ HEADLINE_CFG = 5       # 70B-shaped 80-layer stream: the largest single-GPU conf
 STREAM2B_CFG = 2
 PREFILL_CFG = 3
 SWEEP_CFG = 4
+CROSSOVER_COPIES = 4      # 4 x 54.5 MB of packed weights > 126 MB L2
 SINGLE_CFG = 1
 HEADLINE_LAUNCH_LAYERS = 20   # layers per grouped call of the headline step (4 calls)
 SUSTAINED_S = 2.0
@@ -192,8 +193,28 @@ def time_graph(fn, s, reps):
         return "failed: %s" % exc
 
 
+FLUSH_BYTES = 256 * 1024 * 1024
+
+
+def flush_buffer(dev):
+    """Two 256 MB halves for flush_l2: the first is written, the second read."""
+    return torch.empty(2 * FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+
+def device_busy(s, us=100):
+    """Queue a ~us microsecond spin on stream s, so that the event recorded
+    next and the launch after it reach a busy device: the timed region then
+    holds the kernel alone, not the host's work to enqueue it."""
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(int(us * 2000))
+
+
 def flush_l2(buf):
-    buf.zero_()
+    """Evict L2 (126 MB) before a timed launch: write 256 MB, then read another
+    256 MB so that the written lines go back to HBM here, outside the timed
+    region, and the timed kernel's misses evict clean lines only."""
+    buf[:FLUSH_BYTES].zero_()
+    buf[FLUSH_BYTES:].view(torch.int64).sum()
 
 
 def rounded(v, nd=4):
@@ -427,7 +448,7 @@ def measure_prefill(dev, s, peaks, cfg, N, reps, breakdown=True):
     grouped GEMM launch, timed with events around it, L2 flushed before every
     timed step (the quantiser launch timed separately)."""
     pre = PrefillLayer(dev, cfg, N)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = flush_buffer(dev)
     for _ in range(3):
         pre.quant_all(s)
         pre.gemm_all(s)
@@ -479,7 +500,8 @@ def measure_prefill(dev, s, peaks, cfg, N, reps, breakdown=True):
                      "peak_note": "int8 peak = bf16 burst peak (%s) x nominal int8:bf16 ratio 2"
                                   % peaks["source"],
                      "frac_of_nominal_4500": round(tops / 4500.0, 4)},
-        "l2": "256 MB buffer written between timed steps (flush)",
+        "l2": "flush before every timed step: 256 MB written, then another 256 MB read "
+              "(the written lines go back to HBM before the timed launch)",
     })
     if cfg == PREFILL_CFG:
         out["roofline"]["traffic"] = ncu_traffic("gemm")
@@ -491,8 +513,11 @@ def measure_prefill(dev, s, peaks, cfg, N, reps, breakdown=True):
 
 def measure_crossover(dev, s, reps=30):
     """The 8B-shaped batch sweep on one layer (7 projections, one grouped launch
-    per path): the CUDA-core GEMV (N <= 16) against the tensor-core GEMM, with
-    L2 flushed before every timed launch.  Locates the GEMV -> GEMM crossover."""
+    per path): the CUDA-core GEMV (N <= 16) against the tensor-core GEMM.
+    Timed launches rotate over CROSSOVER_COPIES copies of the layer's packed
+    weights (218 MB > the 126 MB L2), so every launch reads its weights from
+    HBM, as a decoder reading layer after layer does, and nothing is written
+    to evict L2.  Locates the GEMV -> GEMM crossover."""
     wl = inputs.WORKLOADS[SWEEP_CFG]
     layers = []
     for p, (name, M, K) in enumerate(wl.model.projections()):
@@ -500,7 +525,8 @@ def measure_crossover(dev, s, reps=30):
         layers.append(api.pack_weights(W) + (M, K))
         del W
     packed_bytes = sum(M * K // 4 for (_, _, M, K) in layers)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    copies = [layers] + [[(packed.clone(), alpha, M, K) for (packed, alpha, M, K) in layers]
+                         for _ in range(CROSSOVER_COPIES - 1)]
     out = {"workload": "8B-shaped layer (q 4096x4096, k/v 1024x4096, o 4096x4096, gate/up "
                        "14336x4096, down 4096x14336), 7 projections per grouped launch",
            "N": [], "gemv_us": [], "gemv_quant_us": [], "gemm_us": [], "gemv_gbs": [],
@@ -516,20 +542,21 @@ def measure_crossover(dev, s, reps=30):
                                    outlier_frac=wl.outlier_frac)
             xf[p] = x
             xs[p] = api.quant_act(x)
-        ents = []
-        for p, (packed, alpha, M, K) in enumerate(layers):
-            xq, am, xsum = xs[input_proj(p)]
-            ents.append((packed, alpha, M, K, xq, am, xsum,
-                         torch.empty((N, M), device=dev), None))
-        prob = _lib.make_problems(ents)
-        fents = [(packed, alpha, M, K, xf[input_proj(p)], torch.empty((N, M), device=dev), None)
-                 for p, (packed, alpha, M, K) in enumerate(layers)]
-        fprob = _lib.make_fused_problems(fents)
+        ys = [torch.empty((N, M), device=dev) for (_, _, M, _) in layers]
+        probs, fprobs = [], []
+        for cp in copies:
+            ents = [(packed, alpha, M, K) + tuple(xs[input_proj(p)]) + (ys[p], None)
+                    for p, (packed, alpha, M, K) in enumerate(cp)]
+            probs.append(_lib.make_problems(ents))
+            fents = [(packed, alpha, M, K, xf[input_proj(p)], ys[p], None)
+                     for p, (packed, alpha, M, K) in enumerate(cp)]
+            fprobs.append(_lib.make_fused_problems(fents))
+        nproj = len(layers)
         res = {}
-        for path, fn in (("gemv", lambda: _lib.bitlinear_gemv_grouped(prob, len(ents), N, s)),
+        for path, fn in (("gemv", lambda c: _lib.bitlinear_gemv_grouped(probs[c], nproj, N, s)),
                          ("gemv_quant",
-                          lambda: _lib.bitlinear_gemv_quant_grouped(fprob, len(fents), N, s)),
-                         ("gemm", lambda: _lib.bitlinear_gemm_grouped(prob, len(ents), N, s))):
+                          lambda c: _lib.bitlinear_gemv_quant_grouped(fprobs[c], nproj, N, s)),
+                         ("gemm", lambda c: _lib.bitlinear_gemm_grouped(probs[c], nproj, N, s))):
             if path != "gemm" and N > api.GEMV_MAX_TOKENS:
                 res[path] = None
                 continue
@@ -537,14 +564,15 @@ def measure_crossover(dev, s, reps=30):
                                                 for (_, _, _, K) in layers):
                 res[path] = None      # the fused kernel's int8 copy of x does not fit
                 continue
-            for _ in range(3):
-                _lib.check(fn(), path)
+            for c in range(CROSSOVER_COPIES):
+                _lib.check(fn(c), path)
+            torch.cuda.synchronize()
             tot = 0.0
-            for _ in range(reps):
-                flush_l2(flush)
+            for i in range(reps):
                 a, b = events(2)
+                device_busy(s)
                 a.record(s)
-                _lib.check(fn(), path)
+                _lib.check(fn(i % CROSSOVER_COPIES), path)
                 b.record(s)
                 torch.cuda.synchronize()
                 tot += a.elapsed_time(b)
@@ -564,7 +592,10 @@ def measure_crossover(dev, s, reps=30):
     out["gemm_faster_at_N"] = faster
     out["packed_bytes"] = packed_bytes
     out["dispatch"] = "api.matmul: GEMV below N = %d, GEMM from there" % api.GEMM_MIN_TOKENS
-    del flush
+    out["l2"] = ("no flush: %d copies of the layer (%.0f MB) visited in turn, so each timed "
+                 "launch reads weights that left L2 three launches earlier"
+                 % (CROSSOVER_COPIES, CROSSOVER_COPIES * packed_bytes / 1e6))
+    del copies
     torch.cuda.empty_cache()
     return out
 

@@ -12,31 +12,37 @@
 // and the MMAs read A from there, so no expanded tile is written to or read
 // from shared memory.
 //
-// The ring moves k-groups of four k-blocks (512 weights): per stage one TMA
-// box of 128 weight rows x 128 packed bytes (128-byte swizzle, so the row
-// reads below are conflict-free) and the group's activation tiles (BN x 128
-// int8 each, 128-byte swizzle).  Whole 128-byte rows keep the number of
-// memory requests per weight byte low: rows 32 bytes wide (one k-block) left
-// DRAM at a seventh of its bandwidth, most of each row's sectors missing L2
-// one 32-byte request at a time.
+// Measured on B200 and built in:
+//   * a tcgen05.mma of M = 128, N = 16, K = 32 keeps the tensor pipe busy
+//     for ~10 cycles when a whole warp runs the issue loop and an elected
+//     lane issues; a loop run by one lane alone took ~50 cycles per MMA, and
+//     ~85 with ALU-bound warps on its SM sub-partition (the unpack warps
+//     share it: a warp's tensor-memory lane quarter is fixed by its index);
+//     descriptors are built once per stage and the 16 MMAs of a k-group are
+//     unrolled with immediate offsets;
+//   * DRAM serves 256 contiguous bytes of a row better than 128: a ring stage
+//     holds two k-groups (2 x 128 bytes of each of the 128 rows).
 //
-//   warp 0        TMA producer;
-//   warps 4-11    unpackers, in kSmallUnpackGroups groups of four that take
-//                 alternate k-groups: warp w owns tensor-memory lanes
-//                 32 (w % 4) .. +31, one weight row per lane; per k-group it
-//                 reads its row's 128 packed bytes, expands each k-block's 32
-//                 bytes to 32 words of codes+1 (four int8 per word, in k order)
-//                 and stores them with one tcgen05.st into one of the four A
-//                 buffers (32 columns each) of the group's slot, then waits once
-//                 for the group's stores and hands the slot to the MMA;
-//   warp 1        MMA issuer: 4 x tcgen05.mma kind::i8 (K = 32) per k-block,
-//                 A from tensor memory, B from the ring; one commit per k-group
-//                 frees the A slot and one its ring stage (barrier waits and
-//                 commits, not the MMAs, took most of this thread's time when
-//                 they were per k-block); accumulators double-buffered;
-//   warps 2,3,12,13  epilogue, one per lane quarter: tcgen05.ld of BN columns,
-//                 subtract the token's sum of q (the +1 code offset), rescale
-//                 by alpha * amax / 127, store y (lane = row: coalesced).
+//   warp 0        TMA producer (an elected lane issues): per stage two boxes of 128 weight rows x 128
+//                 packed bytes (128-byte swizzle, one per k-group) and the
+//                 stage's activation tiles (BN x 128 int8 per k-block);
+//   warps 4-11    unpackers, two groups of four; group g expands k-group g of
+//                 every stage.  Warp w owns tensor-memory lanes 32 (w % 4) ..
+//                 +31, one weight row per lane: it reads its row's 128 packed
+//                 bytes, expands each k-block's 32 bytes to 32 words of codes+1
+//                 (four int8 per word, in k order), stores them with one
+//                 tcgen05.st per k-block into the k-group's A slot (128
+//                 columns), waits once, and hands the slot to the MMA;
+//   warp 1        MMA issue warp (an elected lane issues): per k-group 16 x
+//                 tcgen05.mma kind::i8 (K = 32),
+//                 A from tensor memory, B from the ring, one accumulator per
+//                 tile (double-buffered across tiles); a commit per k-group
+//                 frees its A slot, one per stage frees the ring stage (the
+//                 unpackers have read the packed bytes before they hand over
+//                 the slot, so the MMA's completion implies theirs);
+//   warps 2,3,12,13  epilogue, one per lane quarter: tcgen05.ld of BN
+//                 columns, subtract the token's sum of q (the +1 code offset),
+//                 rescale by alpha * amax / 127, store y (lane = row: coalesced).
 //
 // Tiles (one per 128-row block of every problem of the launch) are spread
 // over persistent CTAs by the host's longest-first schedule, as in gemm.cuh.
@@ -48,43 +54,48 @@
 
 namespace bl {
 
-constexpr int kSmallUnpackGroups = 2;
+constexpr int kSmallUnpackGroups = 2;                              // = k-groups per stage
 constexpr int kSmallThreads = (6 + 4 * kSmallUnpackGroups) * 32;   // 14 warps
-constexpr int kSmallGroupKb = 4;                                   // k-blocks per ring stage
+constexpr int kSmallGroupKb = 4;                                   // k-blocks per k-group
 constexpr int kSmallGroupBytes = kSmallGroupKb * kGemmPackedRowBytes;   // 128 per row
-// Each tile accumulates into kSmallAcc independent accumulators (MMA kk of every
-// k-block into accumulator kk), summed in the epilogue: consecutive MMAs then
-// do not wait for each other's result, which short MMAs (N = 16 or 32) would
-// otherwise do once per K = 32 step.
-constexpr int kSmallAcc = 4;
-static_assert(kSmallAcc == kGemmBK / 32, "one accumulator per K = 32 step of a k-block");
+constexpr int kSmallStageKb = kSmallUnpackGroups * kSmallGroupKb;  // k-blocks per stage
 constexpr uint32_t kSmallTmemCols = 512;
-// Tensor memory: two sets of kSmallAcc accumulators of BN columns, then the A
-// buffers (32 columns each) in what is left.
-__host__ __device__ constexpr int small_acol_base(int bn) { return 2 * kSmallAcc * bn; }
-__host__ __device__ constexpr int small_abufs(int bn) {
-  return (static_cast<int>(kSmallTmemCols) - small_acol_base(bn)) / 32;
+constexpr int kSmallSlotCols = 32 * kSmallGroupKb;                 // one k-group of A
+// Tensor memory: two accumulators of BN columns, then the A slots.
+__host__ __device__ constexpr int small_acol_base(int bn) { return 2 * bn; }
+__host__ __device__ constexpr int small_aslots(int bn) {
+  return (static_cast<int>(kSmallTmemCols) - small_acol_base(bn)) / kSmallSlotCols;
 }
-// A slots: the four A buffers of one k-group.
-__host__ __device__ constexpr int small_aslots(int bn) { return small_abufs(bn) / kSmallGroupKb; }
-
-__host__ __device__ constexpr int small_stages(int bn) { return bn <= 16 ? 8 : 6; }
+__host__ __device__ constexpr int small_stages(int bn) { return bn <= 16 ? 4 : 3; }
 
 template <int BN>
 struct SmallSmem {
   static constexpr int S = small_stages(BN);
   // each array up to the barriers is a multiple of 1024 bytes
-  uint8_t apk[S][kGemmBM * kSmallGroupBytes];          // packed weights, 16 KB, swizzled
-  uint8_t b[S][kSmallGroupKb][BN * kGemmBK];           // activations, 128-byte swizzle
+  uint8_t apk[S][kSmallUnpackGroups][kGemmBM * kSmallGroupBytes];   // packed, swizzled
+  uint8_t b[S][kSmallStageKb][BN * kGemmBK];                         // 128-byte swizzle
   uint64_t full[S];
-  uint64_t empty[S];                                   // MMA commit + 4 unpack warps
-  uint64_t afull[small_aslots(BN)];                    // 4 unpack warps
-  uint64_t aempty[small_aslots(BN)];                   // MMA commit
+  uint64_t empty[S];                      // MMA commit
+  uint64_t afull[small_aslots(BN)];       // 4 unpack warps
+  uint64_t aempty[small_aslots(BN)];      // MMA commit
   uint64_t tfull[2];
-  uint64_t tempty[2];                                  // 4 epilogue warps
+  uint64_t tempty[2];                     // 4 epilogue warps
   uint64_t drain;
   uint32_t tmem_slot;
   int abort;
+};
+static_assert(small_aslots(16) == 3 && small_aslots(32) == 3, "three A slots");
+static_assert(sizeof(SmallSmem<16>) + 1024 <= 232448, "shared memory");
+static_assert(sizeof(SmallSmem<32>) + 1024 <= 232448, "shared memory");
+
+// Ring position of a k-group: its stage's k-groups get consecutive sequence
+// numbers, and sequence number q uses A slot q % kSlots.
+struct SmallSlot {
+  uint32_t slot = 0, phase = 0;
+  template <int kSlots>
+  __device__ __forceinline__ void advance() {
+    if (++slot == kSlots) { slot = 0; phase ^= 1u; }
+  }
 };
 
 template <int BN>
@@ -94,7 +105,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
   using Smem = SmallSmem<BN>;
   constexpr int S = Smem::S;
   constexpr int kSlots = small_aslots(BN);
-  constexpr uint32_t kSmallAColBase = small_acol_base(BN);
+  constexpr uint32_t kAColBase = small_acol_base(BN);
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
   const uint32_t base = smem_u32(smem_raw);
@@ -107,7 +118,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], 1 + 4);
+      mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(&s.afull[i], 4);
@@ -137,102 +148,149 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
-      int issued = 0;
-      for (int ti = 0; ti < ntiles; ++ti) {
-        int pi, m_blk, n_blk;
-        gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
-        const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-        for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallGroupKb) {
-          const int nkb = min(kSmallGroupKb, kblocks - kb0);
-          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort, p.wait_ns)) goto producer_done;
-          mbar_arrive_expect_tx(&s.full[stage],
-                                kGemmBM * kSmallGroupBytes + nkb * BN * kGemmBK);
-          tma_load_2d(s.apk[stage], &p.tmA[pi], &s.full[stage], kb0 * kGemmPackedRowBytes,
-                      m_blk * kGemmBM);
-          for (int j = 0; j < nkb; ++j)
-            tma_load_2d(s.b[stage][j], &p.tmB[pi], &s.full[stage], (kb0 + j) * kGemmBK,
-                        n_blk * BN);
-          ++issued;
-          if (++stage == S) { stage = 0; phase ^= 1u; }
-        }
-      }
-    producer_done:
-      gemm_drain_loads<S>(s.full, issued);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
-      uint32_t stage = 0, phase = 0, slot = 0, sphase = 0;
-      for (int ti = 0; ti < ntiles; ++ti) {
-        int pi, m_blk, n_blk;
-        gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
-        const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-        const uint32_t db = ti & 1, dp = (ti >> 1) & 1;
-        if (!mbar_wait(&s.tempty[db], dp ^ 1u, abort, p.wait_ns)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + db * kSmallAcc * BN;
-        bool ok = true;
-        for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallGroupKb) {
-          const int nkb = min(kSmallGroupKb, kblocks - kb0);
-          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
-              !mbar_wait(&s.afull[slot], sphase, abort, p.wait_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_slot = tmem_base + kSmallAColBase + 32 * kSmallGroupKb * slot;
-          for (int j = 0; j < nkb; ++j) {
-            const uint32_t b_addr = smem_u32(s.b[stage][j]);
-#pragma unroll
-            for (int kk = 0; kk < kGemmBK / 32; ++kk)   // accumulator kk (kSmallAcc == 4)
-              mma_i8_ts(d_tmem + kk * BN, a_slot + 32 * j + 8 * kk,
-                        smem_desc_k_sw128(b_addr + 32 * kk), idesc, (kb0 + j) != 0);
-          }
-          mma_commit(&s.aempty[slot]);
-          mma_commit(&s.empty[stage]);
-          if (++stage == S) { stage = 0; phase ^= 1u; }
-          if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
-        }
-        if (!ok) break;
-        mma_commit(&s.tfull[db]);
-      }
-      mma_commit(&s.drain);
-      mbar_drain(&s.drain, 0);
-    }
-  } else if (warp >= 4 && warp < 4 + 4 * kSmallUnpackGroups) {
-    // ------------------------------------------------------------ unpackers
-    const uint32_t quarter = static_cast<uint32_t>(warp & 3);
-    const int group = (warp - 4) >> 2;   // takes the k-groups whose sequence number % groups == group
-    const int u = static_cast<int>(quarter) * 32 + lane;   // weight row within the tile
-    const uint32_t sw = static_cast<uint32_t>(u & 7);       // the row's 128-byte swizzle
-    const uint32_t lane_addr = (quarter * 32u) << 16;
-    uint32_t stage = 0, phase = 0, slot = 0, sphase = 0;
-    int seq = 0;
+    // The whole warp runs the loop; the elected lane issues the copies.
+    const bool leader = elect_one_sync();
+    uint32_t stage = 0, phase = 0;
+    int issued = 0;
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
       gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-      for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallGroupKb, ++seq) {
-        const int nkb = min(kSmallGroupKb, kblocks - kb0);
-        if (seq % kSmallUnpackGroups == group) {
-          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
-              !mbar_wait(&s.aempty[slot], sphase ^ 1u, abort, p.wait_ns))
+      for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallStageKb) {
+        const int nkb = min(kSmallStageKb, kblocks - kb0);
+        const int ngroups = (nkb + kSmallGroupKb - 1) / kSmallGroupKb;
+        if (!mbar_wait_warp(&s.empty[stage], phase ^ 1u, abort, p.wait_ns)) goto producer_done;
+        if (leader) {
+          mbar_arrive_expect_tx(&s.full[stage], ngroups * (kGemmBM * kSmallGroupBytes) +
+                                                    nkb * (BN * kGemmBK));
+          for (int g = 0; g < ngroups; ++g)
+            tma_load_2d(s.apk[stage][g], &p.tmA[pi], &s.full[stage],
+                        (kb0 + g * kSmallGroupKb) * kGemmPackedRowBytes, m_blk * kGemmBM);
+          for (int j = 0; j < nkb; ++j)
+            tma_load_2d(s.b[stage][j], &p.tmB[pi], &s.full[stage], (kb0 + j) * kGemmBK,
+                        n_blk * BN);
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
+    }
+  producer_done:
+    if (leader) gemm_drain_loads<S>(s.full, issued);
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs the loop; the elected lane issues the MMAs and the
+    // commits (a commit tracks the MMAs of the thread that issues it).
+    const bool leader = elect_one_sync();
+    constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
+    uint32_t stage = 0, phase = 0;
+    SmallSlot sl;
+    const uint64_t b_desc0 = smem_desc_k_sw128(smem_u32(s.b[0][0]));
+    for (int ti = 0; ti < ntiles; ++ti) {
+      int pi, m_blk, n_blk;
+      gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
+      const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
+      const uint32_t db = ti & 1, dp = (ti >> 1) & 1;
+      if (!mbar_wait_warp(&s.tempty[db], dp ^ 1u, abort, p.wait_ns)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + db * BN;
+      bool ok = true;
+      for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallStageKb) {
+        const int nkb = min(kSmallStageKb, kblocks - kb0);
+        if (!mbar_wait_warp(&s.full[stage], phase, abort, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        // descriptor of this stage's first activation tile; the others are
+        // immediate offsets from it (start address >> 4 in the low bits)
+        const uint64_t bd =
+            b_desc0 + static_cast<uint64_t>((stage * (kSmallStageKb * BN * kGemmBK)) >> 4);
+        for (int g = 0; g * kSmallGroupKb < nkb; ++g) {
+          if (!mbar_wait_warp(&s.afull[sl.slot], sl.phase, abort, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_slot = tmem_base + kAColBase + kSmallSlotCols * sl.slot;
+          const uint64_t bg =
+              bd + static_cast<uint64_t>((g * kSmallGroupKb * BN * kGemmBK) >> 4);
+          const int gkb = min(kSmallGroupKb, nkb - g * kSmallGroupKb);
+          const uint32_t first = (kb0 == 0 && g == 0) ? 0u : 1u;   // accumulate flag of MMA 0
+          if (gkb == kSmallGroupKb) {
+#pragma unroll
+            for (int j = 0; j < kSmallGroupKb; ++j)
+#pragma unroll
+              for (int kk = 0; kk < kGemmBK / 32; ++kk) {
+                const uint64_t bdesc =
+                    bg + static_cast<uint64_t>((j * BN * kGemmBK + 32 * kk) >> 4);
+                if (leader)
+                  mma_i8_ts(d_tmem, a_slot + 32 * j + 8 * kk, bdesc, idesc,
+                            (j | kk) == 0 ? first : 1u);
+              }
+          } else {
+            for (int j = 0; j < gkb; ++j)
+#pragma unroll
+              for (int kk = 0; kk < kGemmBK / 32; ++kk) {
+                const uint64_t bdesc =
+                    bg + static_cast<uint64_t>((j * BN * kGemmBK + 32 * kk) >> 4);
+                if (leader)
+                  mma_i8_ts(d_tmem, a_slot + 32 * j + 8 * kk, bdesc, idesc,
+                            (j | kk) == 0 ? first : 1u);
+              }
+          }
+          if (leader) mma_commit(&s.aempty[sl.slot]);
+          __syncwarp();
+          sl.advance<kSlots>();
+        }
+        if (!ok) break;
+        if (leader) mma_commit(&s.empty[stage]);
+        __syncwarp();
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (leader) mma_commit(&s.tfull[db]);
+      __syncwarp();
+    }
+    if (leader) {
+      mma_commit(&s.drain);
+      mbar_drain(&s.drain, 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 4 + 4 * kSmallUnpackGroups) {
+    // ------------------------------------------------------------ unpackers
+    const uint32_t quarter = static_cast<uint32_t>(warp & 3);
+    const int group = (warp - 4) >> 2;                     // the stage's k-group it expands
+    const int u = static_cast<int>(quarter) * 32 + lane;   // weight row within the tile
+    const uint32_t sw = static_cast<uint32_t>(u & 7);       // the row's 128-byte swizzle
+    const uint32_t lane_addr = (quarter * 32u) << 16;
+    uint32_t stage = 0, phase = 0;
+    SmallSlot first;   // A slot of the current stage's first k-group
+    for (int ti = 0; ti < ntiles; ++ti) {
+      int pi, m_blk, n_blk;
+      gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
+      const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
+      for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallStageKb) {
+        const int nkb = min(kSmallStageKb, kblocks - kb0);
+        const int ngroups = (nkb + kSmallGroupKb - 1) / kSmallGroupKb;
+        if (group < ngroups) {
+          SmallSlot my = first;
+          for (int g = 0; g < group; ++g) my.advance<kSlots>();
+          const int gkb = min(kSmallGroupKb, nkb - group * kSmallGroupKb);
+          if (!mbar_wait_warp(&s.full[stage], phase, abort, p.wait_ns) ||
+              !mbar_wait_warp(&s.aempty[my.slot], my.phase ^ 1u, abort, p.wait_ns))
             goto unpack_done;
           tc_fence_after();
           // the row's 128 bytes: 16-byte chunk c at chunk c ^ (row % 8)
-          const uint8_t* row = s.apk[stage] + u * kSmallGroupBytes;
+          const uint8_t* row = s.apk[stage][group] + u * kSmallGroupBytes;
           uint4 c[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             c[q] = *reinterpret_cast<const uint4*>(row + ((static_cast<uint32_t>(q) ^ sw) << 4));
-          const uint32_t a_slot =
-              tmem_base + lane_addr + kSmallAColBase + 32 * kSmallGroupKb * slot;
+          const uint32_t a_slot = tmem_base + lane_addr + kAColBase + kSmallSlotCols * my.slot;
 #pragma unroll
           for (int j = 0; j < kSmallGroupKb; ++j) {
-            if (j < nkb) {
+            if (j < gkb) {
               const uint32_t words[8] = {c[2 * j].x,     c[2 * j].y,     c[2 * j].z,
                                          c[2 * j].w,     c[2 * j + 1].x, c[2 * j + 1].y,
                                          c[2 * j + 1].z, c[2 * j + 1].w};
@@ -250,13 +308,10 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&s.afull[slot]);
-            mbar_arrive(&s.empty[stage]);   // this warp has read its packed rows
-          }
+          if (lane == 0) mbar_arrive(&s.afull[my.slot]);
         }
+        for (int g = 0; g < ngroups; ++g) first.advance<kSlots>();
         if (++stage == S) { stage = 0; phase ^= 1u; }
-        if (++slot == kSlots) { slot = 0; sphase ^= 1u; }
       }
     }
   unpack_done:;
@@ -276,23 +331,14 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
         sc = __fmul_rn(__ldg(pr.alpha), __fdiv_rn(__ldg(pr.amax + nl), 127.0f));
         xs = __ldg(pr.xsum + nl);
       }
-      if (!mbar_wait(&s.tfull[db], dp, abort, p.wait_ns)) break;
+      if (!mbar_wait_warp(&s.tfull[db], dp, abort, p.wait_ns)) break;
       tc_fence_after();
       uint32_t r[BN];
-      const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + db * kSmallAcc * BN;
-#pragma unroll
-      for (int j = 0; j < BN; ++j) r[j] = 0;
-#pragma unroll
-      for (int a = 0; a < kSmallAcc; ++a) {   // the accumulators' int32 sums
-        uint32_t t[BN];
-        if constexpr (BN == 16) {
-          tmem_ld_32x32b_x16(taddr + a * BN, t);
-        } else {
-          tmem_ld_32x32b_x32(taddr + a * BN, t);
-        }
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < BN; ++j) r[j] += t[j];
+      const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + db * BN;
+      if constexpr (BN == 16) {
+        tmem_ld_32x32b_x16(taddr, r);
+      } else {
+        tmem_ld_32x32b_x32(taddr, r);
       }
       tmem_ld_wait();
       tc_fence_before();

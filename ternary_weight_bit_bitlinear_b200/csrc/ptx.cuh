@@ -103,6 +103,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait by every lane of a warp, with one answer for all of them: when
+// any lane gives up (its limit, or another role's abort), every lane returns
+// false, so the warp leaves its loop as a whole and never splits in front of
+// a warp-collective instruction (tcgen05.ld/st .sync.aligned, elect.sync).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort,
+                                               unsigned long long limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// True in exactly one lane of the (converged, full) warp that executes it.
+// MMA issue loops run on the whole warp and let the elected lane issue: loop
+// control and descriptor arithmetic are then warp-uniform, and a
+// tcgen05.mma costs its issuing warp a few cycles instead of the ~50 a
+// single-lane (divergent) issue loop takes.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Wait, without an abort flag, for a phase that work this CTA has already
 // issued will complete (its own copies or MMAs in flight), before the memory
 // they touch is released.  Gives up after kDrainLimitNs.
