@@ -5,7 +5,7 @@
 // left unoptimised by the CPU kernels).  Each CTA owns a 128-row weight block
 // and a BN-token block, accumulating D[128 x BN] (int32) in tensor memory:
 //
-//   warp 0      TMA producer: packed weight tile (128 rows x 32 bytes = 128
+//   warp 0      TMA producer (elected lane): packed weight tile (128 rows x 32 bytes = 128
 //               weights per row) and int8 activation tile (BN x 128, 128-byte
 //               swizzle) into a STAGES-deep shared-memory ring;
 //   warps 2-5   unpackers: one weight row per thread, 2-bit fields -> int8
@@ -13,7 +13,9 @@
 //               MMA reads (a double buffer of its own, so the TMA ring only
 //               holds what is in flight from memory), then a proxy fence and an
 //               mbarrier arrive;
-//   warp 1      MMA issuer: 4 x tcgen05.mma kind::i8 (K = 32 each) per stage,
+//   warp 1      MMA issue warp, an elected lane issuing (a loop run by one
+//               lane alone costs ~50 cycles per MMA in instruction overhead):
+//               4 x tcgen05.mma kind::i8 (K = 32 each) per stage,
 //               tcgen05.commit frees the stage; accumulators double-buffered
 //               in tensor memory so the epilogue of tile i overlaps tile i+1;
 //   warps 6-13  epilogue, two warps per TMEM lane quarter, alternate 32-column
@@ -181,69 +183,85 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
-      int issued = 0;
-      for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti) {
-        const int tile = gemm_my_tile(p, ti);
-        int pi, m_blk, n_blk;
-        gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
-        const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort, p.wait_ns)) goto producer_done;
+    // The whole warp runs the loop; the elected lane issues the copies.
+    const bool leader = elect_one_sync();
+    uint32_t stage = 0, phase = 0;
+    int issued = 0;
+    for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti) {
+      const int tile = gemm_my_tile(p, ti);
+      int pi, m_blk, n_blk;
+      gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+      const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!mbar_wait_warp(&s.empty[stage], phase ^ 1u, abort, p.wait_ns)) goto producer_done;
+        if (leader) {
           mbar_arrive_expect_tx(&s.full[stage], kStageTx);
           tma_load_2d(s.apk[stage], &p.tmA[pi], &s.full[stage], kb * kGemmPackedRowBytes,
                       m_blk * kGemmBM);
           tma_load_2d(s.b[stage], &p.tmB[pi], &s.full[stage], kb * kGemmBK, n_blk * BN);
-          ++issued;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        __syncwarp();
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-    producer_done:
-      gemm_drain_loads<STAGES>(s.full, issued);
     }
+  producer_done:
+    if (leader) gemm_drain_loads<STAGES>(s.full, issued);
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
-      uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
-      int it = 0;
-      for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti, ++it) {
-        const int tile = gemm_my_tile(p, ti);
-        int pi, m_blk, n_blk;
-        gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
-        const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-        const uint32_t ab = it & 1, ap = (it >> 1) & 1;
-        if (!mbar_wait(&s.tempty[ab], ap ^ 1u, abort, p.wait_ns)) break;
+    // The whole warp runs the loop (warp-uniform control and descriptors);
+    // the elected lane issues the MMAs and the commits.
+    const bool leader = elect_one_sync();
+    constexpr uint32_t idesc = idesc_i8(kGemmBM, BN);
+    const uint64_t a_desc0 = smem_desc_k_sw128(smem_u32(s.a[0]));
+    const uint64_t b_desc0 = smem_desc_k_sw128(smem_u32(s.b[0]));
+    uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
+    int it = 0;
+    for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti, ++it) {
+      const int tile = gemm_my_tile(p, ti);
+      int pi, m_blk, n_blk;
+      gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+      const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
+      const uint32_t ab = it & 1, ap = (it >> 1) & 1;
+      if (!mbar_wait_warp(&s.tempty[ab], ap ^ 1u, abort, p.wait_ns)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + ab * BN;
+      bool ok = true;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!mbar_wait_warp(&s.full[stage], phase, abort, p.wait_ns) ||
+            !mbar_wait_warp(&s.ufull[ub], uphase, abort, p.wait_ns)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ab * BN;
-        bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
-              !mbar_wait(&s.ufull[ub], uphase, abort, p.wait_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(s.a[ub]);
-          const uint32_t b_addr = smem_u32(s.b[stage]);
+        // descriptors: start address >> 4 in the low bits, so offsets add
+        const uint64_t ad = a_desc0 + static_cast<uint64_t>((ub * (kGemmBM * kGemmBK)) >> 4);
+        const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * (BN * kGemmBK)) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kGemmBK / 32; ++kk) {
-            mma_i8_ss(d_tmem, smem_desc_k_sw128(a_addr + 32 * kk),
-                      smem_desc_k_sw128(b_addr + 32 * kk), idesc, (kb | kk) != 0);
-          }
+        for (int kk = 0; kk < kGemmBK / 32; ++kk) {
+          if (leader)
+            mma_i8_ss(d_tmem, ad + static_cast<uint64_t>(2 * kk),
+                      bd + static_cast<uint64_t>(2 * kk), idesc, (kb | kk) != 0);
+        }
+        if (leader) {
           mma_commit(&s.empty[stage]);
           mma_commit(&s.uempty[ub]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          if (++ub == kGemmUnpackBufs) { ub = 0; uphase ^= 1u; }
         }
-        if (!ok) break;
-        mma_commit(&s.tfull[ab]);
+        __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++ub == kGemmUnpackBufs) { ub = 0; uphase ^= 1u; }
       }
-      // Everything issued must finish before tensor memory is released.
+      if (!ok) break;
+      if (leader) mma_commit(&s.tfull[ab]);
+      __syncwarp();
+    }
+    // Everything issued must finish before tensor memory is released.
+    if (leader) {
       mma_commit(&s.drain);
       mbar_drain(&s.drain, 0);
     }
+    __syncwarp();
   } else if (warp < 6) {
     // ------------------------------------------------------------ unpackers
     const int u = threadIdx.x - 64;   // weight row within the tile
@@ -256,8 +274,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(&s.full[stage], phase, abort, p.wait_ns) ||
-            !mbar_wait(&s.uempty[ub], uphase ^ 1u, abort, p.wait_ns))
+        if (!mbar_wait_warp(&s.full[stage], phase, abort, p.wait_ns) ||
+            !mbar_wait_warp(&s.uempty[ub], uphase ^ 1u, abort, p.wait_ns))
           goto unpack_done;
         const uint4* src = reinterpret_cast<const uint4*>(s.apk[stage] + u * kGemmPackedRowBytes);
         const uint4 h0 = src[half], h1 = src[half ^ 1];
@@ -296,7 +314,7 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
       // by value: registers, not re-read from parameter space after each store
       const GemmProblem pr = p.prob[pi];
       const uint32_t ab = it & 1, ap = (it >> 1) & 1;
-      if (!mbar_wait(&s.tfull[ab], ap, abort, p.wait_ns)) break;
+      if (!mbar_wait_warp(&s.tfull[ab], ap, abort, p.wait_ns)) break;
       tc_fence_after();
       const int m = m_blk * kGemmBM + r_in_tile;
       // this warp's copy of the tile's per-token scale and sum

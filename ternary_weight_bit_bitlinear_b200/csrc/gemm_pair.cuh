@@ -3,7 +3,8 @@
 //
 // The two CTAs of a cluster sit on two SMs.  Each loads its own 128 weight
 // rows (packed, then unpacked to int8 as in gemm.cuh) and its own half of the
-// tile's activations (128 tokens); one thread of the rank-0 CTA issues
+// tile's activations (128 tokens); an elected lane of the rank-0 CTA's MMA
+// warp (the whole warp runs the issue loop, as in gemm.cuh) issues
 // tcgen05.mma.cta_group::2 with M = 256 and N = 256, which reads A and B from
 // both shared memories and writes each CTA's 128 rows of D into that CTA's
 // tensor memory.  Per SM this halves the activation bytes that TMA brings in
@@ -112,44 +113,54 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      // The two producers must issue the same number of loads: rank 1's
-      // activation loads complete on rank 0's barriers, and rank 0 drains them
-      // before the pair exits.  So they do not follow the CTA's abort flag
-      // (which is per CTA) and wait on `empty` (committed to both CTAs alike)
-      // with the drain limit: both stop at the same stage when the commits stop.
-      volatile int no_abort = 0;
-      uint32_t stage = 0, phase = 0;
-      int issued = 0;
-      for (int ti = 0; ti < ntiles; ++ti) {
-        const int tile = gemm_my_tile(p, pair, npairs, ti);
-        int pi, m_blk, n_blk;
-        gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
-        const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_cluster(&s.empty[stage], phase ^ 1u, &no_abort, kDrainLimitNs))
-            goto producer_done;
+    // The whole warp runs the loop; the elected lane issues the copies.
+    // The two producers must issue the same number of loads: rank 1's
+    // activation loads complete on rank 0's barriers, and rank 0 drains them
+    // before the pair exits.  So they do not follow the CTA's abort flag
+    // (which is per CTA) and wait on `empty` (committed to both CTAs alike)
+    // with the drain limit: both stop at the same stage when the commits stop.
+    const bool leader = elect_one_sync();
+    volatile int no_abort = 0;
+    uint32_t stage = 0, phase = 0;
+    int issued = 0;
+    for (int ti = 0; ti < ntiles; ++ti) {
+      const int tile = gemm_my_tile(p, pair, npairs, ti);
+      int pi, m_blk, n_blk;
+      gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
+      const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!mbar_wait_cluster_warp(&s.empty[stage], phase ^ 1u, &no_abort, kDrainLimitNs))
+          goto producer_done;
+        if (leader) {
           mbar_arrive_expect_tx(&s.afull[stage], kATx);
           tma_load_2d(s.apk[stage], &p.tmA[pi], &s.afull[stage], kb * kGemmPackedRowBytes,
                       m_blk * kPairBM + static_cast<int>(rank) * kGemmBM);
           if (rank == 0) mbar_arrive_expect_tx(&s.bfull[stage], kBTx);
           tma_load_2d_pair(s.b[stage], &p.tmB[pi], &s.bfull[stage], kb * kGemmBK,
                            n_blk * kPairBN + static_cast<int>(rank) * kPairHalfN);
-          ++issued;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        __syncwarp();
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-    producer_done:
-      // This CTA's weight loads land on its own afull barriers; both CTAs'
-      // activation loads count on rank 0's bfull barriers, so rank 0 waits for
-      // those of the pair (the two producers issue the same sequence).
+    }
+  producer_done:
+    // This CTA's weight loads land on its own afull barriers; both CTAs'
+    // activation loads count on rank 0's bfull barriers, so rank 0 waits for
+    // those of the pair (the two producers issue the same sequence).
+    if (leader) {
       gemm_drain_loads<STAGES>(s.afull, issued);
       if (rank == 0) gemm_drain_loads<STAGES>(s.bfull, issued);
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (rank 0)
-    if (lane == 0 && rank == 0) {
+    // The whole warp of rank 0 runs the loop; the elected lane issues.
+    if (rank == 0) {
+      const bool leader = elect_one_sync();
       constexpr uint32_t idesc = idesc_i8(kPairBM, kPairBN);
+      const uint64_t a_desc0 = smem_desc_k_sw128(smem_u32(s.a[0]));
+      const uint64_t b_desc0 = smem_desc_k_sw128(smem_u32(s.b[0]));
       uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
       int it = 0;
       for (int ti = 0; ti < ntiles; ++ti, ++it) {
@@ -158,34 +169,43 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
         gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
         const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
         const uint32_t ab = it & 1, ap = (it >> 1) & 1;
-        if (!mbar_wait_cluster(&s.tempty[ab], ap ^ 1u, abort, p.wait_ns)) break;
+        if (!mbar_wait_cluster_warp(&s.tempty[ab], ap ^ 1u, abort, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * kPairBN;
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_cluster(&s.bfull[stage], phase, abort, p.wait_ns) ||
-              !mbar_wait_cluster(&s.ufull[ub], uphase, abort, p.wait_ns)) {
+          if (!mbar_wait_cluster_warp(&s.bfull[stage], phase, abort, p.wait_ns) ||
+              !mbar_wait_cluster_warp(&s.ufull[ub], uphase, abort, p.wait_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(s.a[ub]);
-          const uint32_t b_addr = smem_u32(s.b[stage]);
+          // descriptors: start address >> 4 in the low bits, so offsets add
+          const uint64_t ad =
+              a_desc0 + static_cast<uint64_t>((ub * static_cast<int>(sizeof(s.a[0]))) >> 4);
+          const uint64_t bd =
+              b_desc0 + static_cast<uint64_t>((stage * static_cast<int>(sizeof(s.b[0]))) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kGemmBK / 32; ++kk) {
-            mma_i8_ss_pair(d_tmem, smem_desc_k_sw128(a_addr + 32 * kk),
-                           smem_desc_k_sw128(b_addr + 32 * kk), idesc, (kb | kk) != 0);
+            if (leader)
+              mma_i8_ss_pair(d_tmem, ad + static_cast<uint64_t>(2 * kk),
+                             bd + static_cast<uint64_t>(2 * kk), idesc, (kb | kk) != 0);
           }
-          mma_commit_pair(&s.empty[stage]);
-          mma_commit_pair(&s.uempty[ub]);
+          if (leader) {
+            mma_commit_pair(&s.empty[stage]);
+            mma_commit_pair(&s.uempty[ub]);
+          }
+          __syncwarp();
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           if (++ub == kPairUnpackBufs) { ub = 0; uphase ^= 1u; }
         }
         if (!ok) break;
-        mma_commit_pair(&s.tfull[ab]);
+        if (leader) mma_commit_pair(&s.tfull[ab]);
+        __syncwarp();
       }
       // Both CTAs learn through `drain` when the pair's last MMAs are done.
-      mma_commit_pair(&s.drain);
+      if (leader) mma_commit_pair(&s.drain);
+      __syncwarp();
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ unpackers
@@ -199,8 +219,8 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
       gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(&s.afull[stage], phase, abort, p.wait_ns) ||
-            !mbar_wait_cluster(&s.uempty[ub], uphase ^ 1u, abort, p.wait_ns))
+        if (!mbar_wait_warp(&s.afull[stage], phase, abort, p.wait_ns) ||
+            !mbar_wait_cluster_warp(&s.uempty[ub], uphase ^ 1u, abort, p.wait_ns))
           goto unpack_done;
         const uint4* src = reinterpret_cast<const uint4*>(s.apk[stage] + u * kGemmPackedRowBytes);
         const uint4 h0 = src[half], h1 = src[half ^ 1];
@@ -238,7 +258,7 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
       gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
       const GemmProblem pr = p.prob[pi];   // by value: registers, not parameter-space reloads
       const uint32_t ab = it & 1, ap = (it >> 1) & 1;
-      if (!mbar_wait_cluster(&s.tfull[ab], ap, abort, p.wait_ns)) break;
+      if (!mbar_wait_cluster_warp(&s.tfull[ab], ap, abort, p.wait_ns)) break;
       tc_fence_after();
       const int m_base = m_blk * kPairBM + static_cast<int>(rank) * kGemmBM;
       const int m = m_base + r_in_tile;

@@ -412,6 +412,15 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
+// mbar_wait_cluster by every lane of a warp, one answer for all lanes (see
+// mbar_wait_warp).
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t* bar, uint32_t parity,
+                                                       volatile int* abort,
+                                                       unsigned long long limit_ns) {
+  const bool ok = mbar_wait_cluster(bar, parity, abort, limit_ns);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
 // 2-D tiled load into this CTA's shared memory whose completed bytes count on
 // the barrier at the same offset in the rank-0 CTA.  No multicast.
 __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map,
