@@ -254,11 +254,11 @@ BITLINEAR_API bitlinear_status bitlinear_gemm_grouped(const bitlinear_problem* p
  * keeps in shared memory): N = 1 takes K up to 65536, N = 16 up to 4096.
  * Larger cases return BITLINEAR_ERR_UNSUPPORTED_SHAPE; quantise with
  * bitlinear_quant_act and call bitlinear_gemv for them.
- * Two kernels give the same results.  A launch with at least as many 32-row
- * units as the GPU has warp slots for the one-warp kernel streams them with
- * one warp per CTA.  A smaller launch of up to 4 tokens, such as one layer of
- * a decoder, takes one 4-warp CTA per unit instead.  Its warps split the
- * quantisation and the unit's k-chunks and add their int32 sums at the end.
+ * One kernel: each CTA owns a contiguous range of 32-row units with about
+ * the same number of (unit, 512-weight k-chunk) pairs as the others,
+ * quantises the input once into shared memory with all its threads, and its
+ * warps split the range's pairs, adding the int32 sums of units they share
+ * at the end (integer sums: the result does not depend on the split).
  */
 BITLINEAR_API bitlinear_status bitlinear_gemv_quant(const uint32_t* packed, const float* alpha,
                                                     int64_t M, int64_t K, const float* x,

@@ -204,7 +204,14 @@ void build_gemm_schedule(bl::GemmParams& p, int sms) {
   for (int c = 0; c < grid; ++c)
     p.sched_begin[c + 1] = static_cast<uint16_t>(p.sched_begin[c] + count[c]);
   std::vector<int> fill(p.sched_begin, p.sched_begin + grid);
-  for (int t = 0; t < p.total_tiles; ++t) p.sched[fill[owner[t]]++] = static_cast<uint16_t>(t);
+  for (int pi = 0; pi < p.num_problems; ++pi) {
+    const bl::GemmProblem& g = p.prob[pi];
+    const int end = pi + 1 < p.num_problems ? p.prob[pi + 1].tile_begin : p.total_tiles;
+    for (int t = g.tile_begin; t < end; ++t) {
+      const int lt = t - g.tile_begin;
+      p.sched[fill[owner[t]]++] = bl::gemm_sched_entry(pi, lt / g.n_tiles, lt % g.n_tiles);
+    }
+  }
   p.use_sched = 1;
 }
 

@@ -66,8 +66,19 @@ struct GemmParams {
   int use_sched;
   unsigned long long wait_ns;   // limit of every bounded wait of the launch
   uint16_t sched_begin[kGemmMaxGrid + 1];
-  uint16_t sched[kGemmMaxSched];
+  uint32_t sched[kGemmMaxSched];   // gemm_sched_entry(problem, m_blk, n_blk)
 };
+static_assert(sizeof(GemmParams) <= 32764, "kernel parameter space");
+
+// A schedule entry packs a tile's problem, row block and token block, so a
+// CTA finds its tile with two parameter loads (begin, entry) instead of a
+// search over the problem table.  Schedules exist only for launches of at
+// most kGemmMaxSched tiles, so both blocks fit in their fields.
+__host__ __device__ constexpr uint32_t gemm_sched_entry(int pi, int m_blk, int n_blk) {
+  return (static_cast<uint32_t>(pi) << 29) | (static_cast<uint32_t>(m_blk) << 12) |
+         static_cast<uint32_t>(n_blk);
+}
+static_assert(kGemmMaxProblems <= 8 && kGemmMaxSched <= 4096, "schedule entry fields");
 
 // Tiles of worker `who` out of `nwho` (a CTA, or a CTA pair).
 __device__ __forceinline__ int gemm_my_count(const GemmParams& p, int who, int nwho) {
@@ -75,18 +86,11 @@ __device__ __forceinline__ int gemm_my_count(const GemmParams& p, int who, int n
   return who < p.total_tiles ? (p.total_tiles - 1 - who) / nwho + 1 : 0;
 }
 
-__device__ __forceinline__ int gemm_my_tile(const GemmParams& p, int who, int nwho, int i) {
-  if (p.use_sched) return p.sched[p.sched_begin[who] + i];
-  return who + i * nwho;
-}
 
 __device__ __forceinline__ int gemm_my_count(const GemmParams& p) {
   return gemm_my_count(p, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
 }
 
-__device__ __forceinline__ int gemm_my_tile(const GemmParams& p, int i) {
-  return gemm_my_tile(p, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), i);
-}
 
 // Per epilogue warp: the 32-token chunks it handles (alternate ones: half 0
 // takes chunks 0, 2, ..., half 1 takes 1, 3, ...), 32 table entries each.
@@ -133,6 +137,28 @@ __device__ __forceinline__ void gemm_locate(const GemmParams& p, int tile, int& 
   const int lt = tile - p.prob[pi].tile_begin;
   m_blk = lt / p.prob[pi].n_tiles;
   n_blk = lt - m_blk * p.prob[pi].n_tiles;
+}
+
+// Tile i of worker `who` (a CTA, or a CTA pair) out of `nwho`: its problem,
+// row block and token block.
+template <int BN>
+__device__ __forceinline__ void gemm_tile_at(const GemmParams& p, int who, int nwho, int i,
+                                             int& pi, int& m_blk, int& n_blk) {
+  if (p.use_sched) {
+    const uint32_t e = p.sched[p.sched_begin[who] + i];
+    pi = static_cast<int>(e >> 29);
+    m_blk = static_cast<int>((e >> 12) & 0x1FFFFu);
+    n_blk = static_cast<int>(e & 0xFFFu);
+    return;
+  }
+  gemm_locate<BN>(p, who + i * nwho, pi, m_blk, n_blk);
+}
+
+template <int BN>
+__device__ __forceinline__ void gemm_tile_at(const GemmParams& p, int i, int& pi, int& m_blk,
+                                             int& n_blk) {
+  gemm_tile_at<BN>(p, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), i, pi, m_blk,
+                   n_blk);
 }
 
 template <int BN, int STAGES>
@@ -188,9 +214,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     uint32_t stage = 0, phase = 0;
     int issued = 0;
     for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti) {
-      const int tile = gemm_my_tile(p, ti);
       int pi, m_blk, n_blk;
-      gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+      gemm_tile_at<BN>(p, ti, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait_warp(&s.empty[stage], phase ^ 1u, abort, p.wait_ns)) goto producer_done;
@@ -219,9 +244,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
     int it = 0;
     for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti, ++it) {
-      const int tile = gemm_my_tile(p, ti);
       int pi, m_blk, n_blk;
-      gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+      gemm_tile_at<BN>(p, ti, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       const uint32_t ab = it & 1, ap = (it >> 1) & 1;
       if (!mbar_wait_warp(&s.tempty[ab], ap ^ 1u, abort, p.wait_ns)) break;
@@ -269,9 +293,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     const int half = (u >> 2) & 1;   // read order of the two 16-byte halves: no bank conflict
     uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
     for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti) {
-        const int tile = gemm_my_tile(p, ti);
-      int pi, m_blk, n_blk;
-      gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+        int pi, m_blk, n_blk;
+        gemm_tile_at<BN>(p, ti, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait_warp(&s.full[stage], phase, abort, p.wait_ns) ||
@@ -308,9 +331,8 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
     const int half = e >> 2;                // this warp stores column chunks cc = half, half+2, ...
     int it = 0;
     for (int ti = 0, tn = gemm_my_count(p); ti < tn; ++ti, ++it) {
-        const int tile = gemm_my_tile(p, ti);
-      int pi, m_blk, n_blk;
-      gemm_locate<BN>(p, tile, pi, m_blk, n_blk);
+        int pi, m_blk, n_blk;
+        gemm_tile_at<BN>(p, ti, pi, m_blk, n_blk);
       // by value: registers, not re-read from parameter space after each store
       const GemmProblem pr = p.prob[pi];
       const uint32_t ab = it & 1, ap = (it >> 1) & 1;

@@ -124,9 +124,8 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
     uint32_t stage = 0, phase = 0;
     int issued = 0;
     for (int ti = 0; ti < ntiles; ++ti) {
-      const int tile = gemm_my_tile(p, pair, npairs, ti);
       int pi, m_blk, n_blk;
-      gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
+      gemm_tile_at<kPairBN>(p, pair, npairs, ti, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait_cluster_warp(&s.empty[stage], phase ^ 1u, &no_abort, kDrainLimitNs))
@@ -164,9 +163,8 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
       uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
       int it = 0;
       for (int ti = 0; ti < ntiles; ++ti, ++it) {
-        const int tile = gemm_my_tile(p, pair, npairs, ti);
         int pi, m_blk, n_blk;
-        gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
+        gemm_tile_at<kPairBN>(p, pair, npairs, ti, pi, m_blk, n_blk);
         const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
         const uint32_t ab = it & 1, ap = (it >> 1) & 1;
         if (!mbar_wait_cluster_warp(&s.tempty[ab], ap ^ 1u, abort, p.wait_ns)) break;
@@ -214,9 +212,8 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
     const int half = (u >> 2) & 1;   // read order of the two 16-byte halves: no bank conflict
     uint32_t stage = 0, phase = 0, ub = 0, uphase = 0;
     for (int ti = 0; ti < ntiles; ++ti) {
-      const int tile = gemm_my_tile(p, pair, npairs, ti);
       int pi, m_blk, n_blk;
-      gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
+      gemm_tile_at<kPairBN>(p, pair, npairs, ti, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait_warp(&s.afull[stage], phase, abort, p.wait_ns) ||
@@ -253,9 +250,8 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
     const int r_in_tile = static_cast<int>(quarter) * 32 + lane;
     int it = 0;
     for (int ti = 0; ti < ntiles; ++ti, ++it) {
-      const int tile = gemm_my_tile(p, pair, npairs, ti);
       int pi, m_blk, n_blk;
-      gemm_locate<kPairBN>(p, tile, pi, m_blk, n_blk);
+      gemm_tile_at<kPairBN>(p, pair, npairs, ti, pi, m_blk, n_blk);
       const GemmProblem pr = p.prob[pi];   // by value: registers, not parameter-space reloads
       const uint32_t ab = it & 1, ap = (it >> 1) & 1;
       if (!mbar_wait_cluster_warp(&s.tfull[ab], ap, abort, p.wait_ns)) break;

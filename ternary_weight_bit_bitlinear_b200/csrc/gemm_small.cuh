@@ -154,7 +154,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
     int issued = 0;
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
-      gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
+      gemm_tile_at<BN>(p, ti, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallStageKb) {
         const int nkb = min(kSmallStageKb, kblocks - kb0);
@@ -189,7 +189,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
     const uint64_t b_desc0 = smem_desc_k_sw128(smem_u32(s.b[0][0]));
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
-      gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
+      gemm_tile_at<BN>(p, ti, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       const uint32_t db = ti & 1, dp = (ti >> 1) & 1;
       if (!mbar_wait_warp(&s.tempty[db], dp ^ 1u, abort, p.wait_ns)) break;
@@ -268,7 +268,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
     SmallSlot first;   // A slot of the current stage's first k-group
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
-      gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
+      gemm_tile_at<BN>(p, ti, pi, m_blk, n_blk);
       const int kblocks = (p.prob[pi].K + kGemmBK - 1) / kGemmBK;
       for (int kb0 = 0; kb0 < kblocks; kb0 += kSmallStageKb) {
         const int nkb = min(kSmallStageKb, kblocks - kb0);
@@ -320,7 +320,7 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
     const uint32_t quarter = static_cast<uint32_t>(warp & 3);   // warps 2, 3, 12, 13
     for (int ti = 0; ti < ntiles; ++ti) {
       int pi, m_blk, n_blk;
-      gemm_locate<BN>(p, gemm_my_tile(p, ti), pi, m_blk, n_blk);
+      gemm_tile_at<BN>(p, ti, pi, m_blk, n_blk);
       const GemmProblem pr = p.prob[pi];   // by value: registers
       const uint32_t db = ti & 1, dp = (ti >> 1) & 1;
       // lane n holds token n's scale and activation sum

@@ -146,15 +146,25 @@ __device__ __forceinline__ GqItem gq_item(const GqParams& p, int seg, int u0, in
   return it;
 }
 
+// Index i (< K4, or past it: left alone) moved by rot (0 <= rot < K4) modulo K4.
+__device__ __forceinline__ int gq_rot(int i, int rot, int K4) {
+  if (i >= K4) return i;
+  const int r = i + rot;
+  return r >= K4 ? r - K4 : r;
+}
+
 // Quantise segment sg's input x [NT][K] into xs [NT][xstride] (zero from K up
 // to chunks * 512); amax / 127 and the sum of q per token go to s_a127 and
 // s_xsum.  Run by every thread of the CTA; starts and ends with a barrier's
-// worth of ordering (callers sync before reusing xs).
+// worth of ordering (callers sync before reusing xs).  Thread tid takes the
+// float4s (tid + rot + j n) mod K/4: CTAs that quantise one input at the same
+// moment pass different `rot` and so read different lines of it at any time
+// (the max and the integer sum do not depend on the order).
 template <int NT>
 __device__ __forceinline__ void gq_quantise_cta(const GqSegment& sg, uint8_t* xs, int xstride,
                                                 float (*red_f)[NT], int (*red_i)[NT],
                                                 float* s_a127, int* s_xsum, int tid,
-                                                int nthreads) {
+                                                int nthreads, int rot) {
   const int warp = tid >> 5, lane = tid & 31, nwarps = nthreads >> 5;
   const int K4 = sg.K / 4, P4 = sg.chunks * (kGemvChunkK / 4);
   constexpr int R = kGqRegF4 / NT > 0 ? kGqRegF4 / NT : 1;   // float4s per thread and token
@@ -170,7 +180,7 @@ __device__ __forceinline__ void gq_quantise_cta(const GqSegment& sg, uint8_t* xs
       const float4* x4 = reinterpret_cast<const float4*>(sg.x + static_cast<int64_t>(t) * sg.K);
 #pragma unroll
       for (int j = 0; j < R; ++j) {
-        const int i = tid + j * nthreads;
+        const int i = gq_rot(tid + j * nthreads, rot, K4);
         v[t][j] = i < K4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
         m[t] = fmaxf(m[t], absmax4(v[t][j]));
       }
@@ -185,7 +195,7 @@ __device__ __forceinline__ void gq_quantise_cta(const GqSegment& sg, uint8_t* xs
         float4 w[RB];
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
-          const int i = b + j * nthreads;
+          const int i = gq_rot(b + j * nthreads, rot, K4);
           w[j] = i < K4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
@@ -212,7 +222,7 @@ __device__ __forceinline__ void gq_quantise_cta(const GqSegment& sg, uint8_t* xs
     if (in_regs) {
 #pragma unroll
       for (int j = 0; j < R; ++j) {
-        const int i = tid + j * nthreads;
+        const int i = gq_rot(tid + j * nthreads, rot, K4);
         if (i < K4) out[i] = mt == 0.0f ? 0u : quant_pack4(v[t][j], s, sum[t]);
       }
     } else {
@@ -222,12 +232,12 @@ __device__ __forceinline__ void gq_quantise_cta(const GqSegment& sg, uint8_t* xs
         float4 w[RB];
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
-          const int i = b + j * nthreads;
+          const int i = gq_rot(b + j * nthreads, rot, K4);
           w[j] = i < K4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
-          const int i = b + j * nthreads;
+          const int i = gq_rot(b + j * nthreads, rot, K4);
           if (i < K4) out[i] = mt == 0.0f ? 0u : quant_pack4(w[j], s, sum[t]);
         }
       }
@@ -365,8 +375,11 @@ gemv_quant_kernel(const __grid_constant__ GqParams p) {
   for (int cseg = seg0;; ++cseg) {
     const GqItem it = gq_item(p, cseg, u0, u1, warp, nwarps);
     __syncthreads();   // every warp is done with the previous item's int8 copy and partials
+    // CTAs that start together read their common input from different offsets
     gq_quantise_cta<NT>(p.seg[cseg], xs, p.xstride, red_f, red_i, s_a127, s_xsum, tid,
-                        32 * nwarps);
+                        32 * nwarps,
+                        static_cast<int>(static_cast<int64_t>(blockIdx.x) *
+                                         (p.seg[cseg].K / 4) / gridDim.x));
 
     int acc[NT][4];
 #pragma unroll
