@@ -68,8 +68,17 @@ NCU_TRAFFIC = {
              "source": "ncu dram__bytes_read+write, gemv_tile_kernel<1>, 2B stream launch"},
     "gemm": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
                       "ternary_weight_bit_bitlinear_b200/csrc/gemm_pair.cuh"],
-             "sha256": "0eb46b29ec660fd4", "bytes": 62_596_096 + 29_230_080,
+             "sha256": "b73069191af7c054", "bytes": 62_601_216 + 31_635_200,
              "source": "ncu dram__bytes_read+write, gemm_i8_pair_kernel<5>, 7B prefill N=512"},
+    # captured on a 4-layer launch of the 70B stream (DRAM reads 1.002 x the
+    # packed bytes, so traffic grows with the layers), x5 to the headline's
+    # 20-layer launch
+    "gemv_quant": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemv_quant.cuh",
+                            "ternary_weight_bit_bitlinear_b200/csrc/gemv.cuh",
+                            "ternary_weight_bit_bitlinear_b200/csrc/quant_math.cuh"],
+                   "sha256": "74fd6e3c6cb1062e", "bytes": (857_407_232 + 4_813_568) * 5,
+                   "source": "ncu dram__bytes_read+write, gemv_quant_kernel<1>, 4-layer launch of "
+                             "the 70B stream, scaled x5 to the 20-layer launch"},
 }
 
 
@@ -935,8 +944,8 @@ def emit(args, world, peaks, h, ms_per_step, gbs, K, K2, e2e_ms, h2d, d2h, prefi
             "bytes_per_launch": round(h["alg_bytes"] / h["ncalls"]),
             "avg_launch_ms": round(h["launch_ms"], 5),
             "timing": "events around each launch, %d steps x %d launches" % (K2, h["ncalls"]),
-            "traffic": None,
-            "traffic_note": "ncu DRAM bytes of this kernel on this workload: see profiles/",
+            "traffic": ncu_traffic("gemv_quant"),
+            "traffic_source": NCU_TRAFFIC["gemv_quant"]["source"],
         },
         "sustained": {
             "what": "the headline step back to back for >= %.0f s" % SUSTAINED_S,
