@@ -101,7 +101,8 @@ __device__ __forceinline__ GemvCopyPlan gemv_plan(const Problem& pr, int row0, i
 // Issue the weight copies of k-chunk `kc` (W words per row) into stage buffer
 // `st`.  Weight chunks outside the layer are skipped (rows past M are never
 // stored; past the last word, the activations are zero, so stale bytes
-// multiply zeros).
+// multiply zeros).  Each copy asks L2 for the aligned 256 bytes around it, so
+// the row's next k-chunk is already on its way when its stage is issued.
 __device__ __forceinline__ void gemv_issue_weights(int W, const GemvCopyPlan& cp, int kc,
                                                    uint8_t* st) {
   if (kc * (kGemvChunkBytes / 4) + cp.wword < W) {
@@ -109,7 +110,8 @@ __device__ __forceinline__ void gemv_issue_weights(int W, const GemvCopyPlan& cp
 #pragma unroll
     for (int i = 0; i < kGemvTileRows / 4; ++i) {
       if (i < cp.vrows)
-        cp_async16(st + ((i & 1) ? cp.dst_odd + (i - 1) * 512 : cp.dst_even + i * 512), src, 16u);
+        cp_async16_l2_256(st + ((i & 1) ? cp.dst_odd + (i - 1) * 512 : cp.dst_even + i * 512),
+                          src);
       src += cp.wstep;
     }
   }

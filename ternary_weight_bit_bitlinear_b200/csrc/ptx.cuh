@@ -180,6 +180,17 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src,
                : "memory");
 }
 
+// 16-byte asynchronous global -> shared copy whose L2 fill covers the whole
+// aligned 256 bytes around the source: a stream that reads 128 bytes of a
+// row per stage then finds the next stage's bytes of that row in L2 (or on
+// their way there), so the reads in flight to DRAM are not bounded by the
+// shared-memory ring alone.
+__device__ __forceinline__ void cp_async16_l2_256(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
