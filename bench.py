@@ -64,19 +64,19 @@ HBM_NOMINAL_GBS = 8000.0     # B200 HBM3e spec figure (context beside the measur
 # longer applies and the bench reports null.
 NCU_TRAFFIC = {
     "gemv": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemv.cuh"],
-             "sha256": "d0ffe60ca94b9a32", "bytes": 522_076_623 + 2_235_136,
+             "sha256": "35fa6f20632f142c", "bytes": 522_951_424 + 7_624_960,
              "source": "ncu dram__bytes_read+write, gemv_tile_kernel<1>, 2B stream launch"},
     "gemm": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
                       "ternary_weight_bit_bitlinear_b200/csrc/gemm_pair.cuh"],
              "sha256": "b73069191af7c054", "bytes": 62_601_216 + 31_635_200,
              "source": "ncu dram__bytes_read+write, gemm_i8_pair_kernel<5>, 7B prefill N=512"},
-    # captured on a 4-layer launch of the 70B stream (DRAM reads 1.002 x the
+    # captured on a 4-layer launch of the 70B stream (DRAM reads 1.003 x the
     # packed bytes, so traffic grows with the layers), x5 to the headline's
     # 20-layer launch
     "gemv_quant": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemv_quant.cuh",
                             "ternary_weight_bit_bitlinear_b200/csrc/gemv.cuh",
                             "ternary_weight_bit_bitlinear_b200/csrc/quant_math.cuh"],
-                   "sha256": "74fd6e3c6cb1062e", "bytes": (857_407_232 + 4_813_568) * 5,
+                   "sha256": "0c47ba719c21d7ae", "bytes": (858_458_112 + 6_199_552) * 5,
                    "source": "ncu dram__bytes_read+write, gemv_quant_kernel<1>, 4-layer launch of "
                              "the 70B stream, scaled x5 to the 20-layer launch"},
 }

@@ -364,11 +364,7 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
   }
   if (best_w == 0) return BITLINEAR_ERR_UNSUPPORTED_SHAPE;
   p.area = bl::gq_smem_bytes(nt, best_w, p.xstride);
-  // Up to kGqOversub CTAs per resident slot, so that SMs that drain their
-  // first range early take later ones -- but only while every warp keeps at
-  // least kGqMinPairsPerWarp pairs: each CTA quantises its inputs once, and on
-  // short launches (a decoder's per-group launches) more CTAs only repeat that
-  // work.  At most one CTA per unit.
+  // One CTA per resident slot, at most one per unit.
   p.total_units = static_cast<int>(units);
   int64_t total = 0;
   for (int g = 0; g < segs; ++g) {
@@ -376,13 +372,8 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
     total += seg_pairs[g];
   }
   p.total_pairs = total;
-  // A whole number of waves (a partial extra wave would leave a tail).
   const int64_t slots = static_cast<int64_t>(dev->sms) * best_per_sm;
-  const int64_t waves = std::max<int64_t>(
-      1, std::min<int64_t>(bl::kGqOversub,
-                           total / (slots * best_w * bl::kGqMinPairsPerWarp)));
-  const int64_t ctas = slots * waves;
-  *grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(ctas, units), INT_MAX / 2));
+  *grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(slots, units), INT_MAX / 2));
   *warps = best_w;
   return BITLINEAR_OK;
 }

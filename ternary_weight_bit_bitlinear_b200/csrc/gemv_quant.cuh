@@ -16,12 +16,11 @@
 // a segment holds units x ceil(K / 512) pairs.  The launch's units are cut
 // into one contiguous range per CTA with about the same number of pairs each:
 // CTA c starts at the unit nearest to pair (total pairs) x c / (CTAs), which
-// every CTA computes from the segment table.  On long launches the host
-// launches up to four times more CTAs than fit on the GPU at once
-// (kGqOversub), so the block scheduler hands the later ranges to whichever SMs
-// finish first: SMs do not all draw the same share of HBM bandwidth, and equal
-// static shares left the slowest SMs finishing a quarter of a launch after the
-// fastest.  A CTA's
+// every CTA computes from the segment table.  The host launches exactly the
+// CTAs that fit on the GPU at once (one per resident slot, at most one per
+// unit): with the two-stage rings and 256-byte L2 fills below, later waves of
+// CTAs only add start-up work (each CTA quantises its inputs), and the 70B-
+// shaped stream ran 2 to 3 % slower with two or four CTAs per slot.  A CTA's
 // range meets one or more segments; each such meeting is an item, and the
 // CTA takes its items in order:
 //   1. all its threads quantise the item's input, once, into the CTA's int8
@@ -61,8 +60,6 @@ constexpr int kGqStages = 2;                                          // power o
 constexpr int kGqStageBytes = kGemvTileRows * kGemvChunkBytes;        // 4 KB of weights
 constexpr int kGqRingBytes = kGqStages * kGqStageBytes;
 constexpr int kGqMaxProblems = 256;
-constexpr int kGqOversub = 4;         // at most this many CTAs launched per CTA slot
-constexpr int kGqMinPairsPerWarp = 64; // ... while each warp keeps this many pairs
 constexpr int kGqMaxWarps = 12;          // 12 x 16 KB of rings already fill shared memory
 constexpr int kGqMaxXBytes = 65536;   // tokens x K (rounded up to 512) held per CTA
 constexpr int kGqRegF4 = 16;          // float4s per thread kept in registers while quantising
