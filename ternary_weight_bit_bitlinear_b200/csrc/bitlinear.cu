@@ -512,6 +512,18 @@ bitlinear_status bitlinear_quant_act(const float* x, int64_t N, int64_t K, int8_
   return bitlinear_quant_act_grouped(&a, 1, stream);
 }
 
+// The row quantiser over `rows` rows, the widest kmax wide: when the rows do
+// not fill the SMs (each row's latency is then the launch's), CTAs wide
+// enough to hold the row in registers; 256-thread CTAs otherwise.
+static cudaError_t launch_quant_rows(int rows, int64_t kmax, const DeviceInfo* dev,
+                                     cudaStream_t s, const bl::QuantParams& p) {
+  const int threads = rows < dev->sms ? bl::quant_wide_threads(kmax) : bl::kQuantThreads;
+  if (threads == 1024)
+    return launch_pdl(bl::quant_rows_kernel<1024>, rows, 1024, 0, s, p);
+  if (threads == 512) return launch_pdl(bl::quant_rows_kernel<512>, rows, 512, 0, s, p);
+  return launch_pdl(bl::quant_rows_kernel<256>, rows, 256, 0, s, p);
+}
+
 bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* acts, int64_t count,
                                              bitlinear_stream_t stream) {
   if (count < 0 || (count > 0 && !acts)) return BITLINEAR_ERR_INVALID_ARG;
@@ -528,13 +540,18 @@ bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* acts, int64_t 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   bl::QuantParams p;
   memset(&p, 0, sizeof p);
-  int64_t rows = 0;
+  int64_t rows = 0, kmax = 0;
+  DeviceInfo* dev = nullptr;
   auto flush = [&]() -> bitlinear_status {
     if (p.count == 0) return BITLINEAR_OK;
-    const cudaError_t e =
-        launch_pdl(bl::quant_rows_kernel, static_cast<int>(rows), bl::kQuantThreads, 0, s, p);
+    if (!dev) {
+      const bitlinear_status dst = device_info(&dev);
+      if (dst != BITLINEAR_OK) return dst;
+    }
+    const cudaError_t e = launch_quant_rows(static_cast<int>(rows), kmax, dev, s, p);
     memset(&p, 0, sizeof p);
     rows = 0;
+    kmax = 0;
     return e == cudaSuccess ? launch_status() : BITLINEAR_ERR_CUDA;
   };
   for (int64_t i = 0; i < count; ++i) {
@@ -552,6 +569,7 @@ bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* acts, int64_t 
     m.K = static_cast<int>(a.K);
     m.row_begin = static_cast<int>(rows);
     rows += a.N;
+    kmax = std::max<int64_t>(kmax, a.K);
   }
   return flush();
 }
@@ -592,8 +610,7 @@ bitlinear_status bitlinear_quant_act_per_tensor(const float* x, int64_t N, int64
   p.m[0].tensor_amax = word;
   p.m[0].K = static_cast<int>(K);
   p.m[0].row_begin = 0;
-  if (launch_pdl(bl::quant_rows_kernel, static_cast<int>(N), bl::kQuantThreads, 0, s, p) !=
-      cudaSuccess)
+  if (launch_quant_rows(static_cast<int>(N), K, dev, s, p) != cudaSuccess)
     return BITLINEAR_ERR_CUDA;
   return launch_status();
 }

@@ -1,6 +1,6 @@
 // launch_gemv.cu -- launchers of the decode GEMV on int8 activations
 // (gemv.cuh: one warp per 32-row unit; gemv_split.cuh: one 4-warp CTA per
-// unit for launches smaller than the GPU).
+// unit for launches that would leave resident warps idle).
 #include "internal.h"
 #include "gemv_split.cuh"
 
@@ -24,9 +24,14 @@ bitlinear_status launch_gemv_tile(const bl::GemvParams& p, DeviceInfo* dev, cuda
   }
   // Every warp resident at once, with the same number of units (give or take
   // one) per warp: units per warp first, then just enough warps.  A launch
-  // with fewer units than that takes the split-unit kernel: one CTA per unit.
+  // with fewer units than resident warps, or one where that would leave more
+  // than a quarter of them idle (a little over a whole multiple: 1792 units on
+  // 1776 warps would run 896 warps of two units each), takes the split-unit
+  // kernel instead: one CTA per unit, its k-chunks split over the CTA's warps,
+  // CTAs handed to SMs as they free up.
   const int64_t cap = static_cast<int64_t>(dev->sms) * per_sm * bl::kGemvWarps;
-  if (p.total_units < cap) {
+  const int64_t upw = (p.total_units + cap - 1) / cap;
+  if (p.total_units < cap || p.total_units * 4 < upw * cap * 3) {
     auto split = bl::gemv_split_kernel<NT>;
     if (!dev->gemv_split_attr_set[NT]) {
       if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -38,7 +43,6 @@ bitlinear_status launch_gemv_tile(const bl::GemvParams& p, DeviceInfo* dev, cuda
       return BITLINEAR_ERR_CUDA;
     return launch_status();
   }
-  const int64_t upw = (p.total_units + cap - 1) / cap;
   const int64_t warps = (p.total_units + upw - 1) / upw;
   const int grid = static_cast<int>((warps + bl::kGemvWarps - 1) / bl::kGemvWarps);
   if (launch_pdl(kernel, grid, bl::kGemvThreads, smem, s, p) != cudaSuccess)

@@ -6,10 +6,15 @@
 //
 // One CTA per token row, rows of several matrices numbered across one launch.
 // Each thread loads its float4s of the row once and keeps up to kQuantRegF4 of
-// them in registers (rows up to 8192 wide are read exactly once); the maximum
-// is reduced with warp shuffles and one shared-memory exchange, the row is
-// quantised from registers, stored four int8 per 32-bit word, and the row sum
-// reduced the same way.
+// them in registers; the maximum is reduced with warp shuffles and one
+// shared-memory exchange, the row is quantised from registers, stored four
+// int8 per 32-bit word, and the row sum reduced the same way.  Launches of
+// many rows use 256-thread CTAs (rows up to 8192 wide read exactly once, and
+// several rows in flight per SM).  Launches of fewer rows than SMs (a
+// decoder's one token) take the fewest threads, from 256 up to 1024, that
+// hold the widest row in registers (quant_wide_threads), so a row's latency
+// is one read and two block reductions; more threads than that only lengthen
+// the reductions.
 //
 // Per-tensor mode (the reading notes' own I2_S setting, section 2.3 and
 // section 4.1: one int8 scale for the whole activation tensor): a first
@@ -22,7 +27,7 @@
 
 namespace bl {
 
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 256;        // row-kernel CTA size for launches of many rows
 constexpr int kQuantRegF4 = 8;             // float4 per thread kept in registers
 constexpr int kQuantMaxMatrices = 64;
 
@@ -41,10 +46,11 @@ struct QuantParams {
   int count;
 };
 
-static __global__ void __launch_bounds__(kQuantThreads)
+template <int kThreads>
+static __global__ void __launch_bounds__(kThreads)
 quant_rows_kernel(const __grid_constant__ QuantParams p) {
-  __shared__ float red_f[kQuantThreads / 32];
-  __shared__ int red_i[kQuantThreads / 32];
+  __shared__ float red_f[kThreads / 32];
+  __shared__ int red_i[kThreads / 32];
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
   const int g = blockIdx.x;
@@ -60,7 +66,7 @@ quant_rows_kernel(const __grid_constant__ QuantParams p) {
   float m = 0.0f;
 #pragma unroll
   for (int j = 0; j < kQuantRegF4; ++j) {
-    const int i = threadIdx.x + j * kQuantThreads;
+    const int i = threadIdx.x + j * kThreads;
     v[j] = i < K4 ? __ldg(row + i) : make_float4(0.f, 0.f, 0.f, 0.f);
     m = fmaxf(m, absmax4(v[j]));
   }
@@ -68,28 +74,28 @@ quant_rows_kernel(const __grid_constant__ QuantParams p) {
   if (A.tensor_amax) {
     amax = __uint_as_float(*A.tensor_amax);
   } else {
-    for (int i = threadIdx.x + kQuantRegF4 * kQuantThreads; i < K4; i += kQuantThreads)
+    for (int i = threadIdx.x + kQuantRegF4 * kThreads; i < K4; i += kThreads)
       m = fmaxf(m, absmax4(__ldg(row + i)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if (lane == 0) red_f[warp] = m;
     __syncthreads();
 #pragma unroll
-    for (int w = 0; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, red_f[w]);
+    for (int w = 0; w < kThreads / 32; ++w) amax = fmaxf(amax, red_f[w]);
   }
 
   uint32_t* out = reinterpret_cast<uint32_t*>(A.xq + static_cast<int64_t>(n) * A.K);
   int sum = 0;
   if (amax == 0.0f) {
-    for (int i = threadIdx.x; i < K4; i += kQuantThreads) out[i] = 0u;
+    for (int i = threadIdx.x; i < K4; i += kThreads) out[i] = 0u;
   } else {
     const float s = __fdiv_rn(127.0f, amax);
 #pragma unroll
     for (int j = 0; j < kQuantRegF4; ++j) {
-      const int i = threadIdx.x + j * kQuantThreads;
+      const int i = threadIdx.x + j * kThreads;
       if (i < K4) out[i] = quant_pack4(v[j], s, sum);
     }
-    for (int i = threadIdx.x + kQuantRegF4 * kQuantThreads; i < K4; i += kQuantThreads)
+    for (int i = threadIdx.x + kQuantRegF4 * kThreads; i < K4; i += kThreads)
       out[i] = quant_pack4(__ldg(row + i), s, sum);
   }
   if (threadIdx.x == 0) A.amax[n] = amax;
@@ -101,10 +107,15 @@ quant_rows_kernel(const __grid_constant__ QuantParams p) {
     if (threadIdx.x == 0) {
       int t = 0;
 #pragma unroll
-      for (int w = 0; w < kQuantThreads / 32; ++w) t += red_i[w];
+      for (int w = 0; w < kThreads / 32; ++w) t += red_i[w];
       A.xsum[n] = t;
     }
   }
+}
+
+// CTA size of a launch of fewer rows than SMs whose widest row is kmax wide.
+inline int quant_wide_threads(int64_t kmax) {
+  return kmax <= 4 * kQuantRegF4 * 256 ? 256 : kmax <= 4 * kQuantRegF4 * 512 ? 512 : 1024;
 }
 
 // Per-tensor maximum of |x| over n4 float4s, folded into *out (the bits of a
