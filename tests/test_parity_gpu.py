@@ -130,6 +130,31 @@ def test_quant_act_grouped_parity():
         assert np.array_equal(xsum.cpu().numpy(), s_ref)
 
 
+@pytest.mark.parametrize("N,K", [(1, 8320), (2, 12288), (1, 16384), (1, 16400), (3, 28672),
+                                 (1, 32768), (1, 32784)])
+def test_quant_act_few_rows_wide_ctas(N, K):
+    # fewer rows than SMs: CTAs of 512 threads for rows of 8193..16384, 1024
+    # above (rows past 32768 are read twice)
+    x = inputs.activations(N, K, seed=N * 31 + K, outlier_frac=0.01)
+    xq, amax, xsum = api.quant_act(x.cuda())
+    q_ref, a_ref, s_ref = oracle.quant_act(x.numpy())
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(amax.cpu().numpy(), a_ref)
+    assert np.array_equal(xsum.cpu().numpy(), s_ref)
+
+
+def test_quant_act_grouped_few_rows():
+    # one launch of 3 rows: every row on a CTA sized for the widest (28672)
+    shapes = [(1, 8192), (1, 28672), (0, 64), (1, 2560)]
+    xs = [inputs.activations(N, K, seed=3 * N + K, outlier_frac=0.01) for N, K in shapes]
+    outs = api.quant_act_grouped([x.cuda() for x in xs])
+    for x, (xq, amax, xsum) in zip(xs, outs):
+        q_ref, a_ref, s_ref = oracle.quant_act(x.numpy())
+        assert np.array_equal(xq.cpu().numpy(), q_ref)
+        assert np.array_equal(amax.cpu().numpy(), a_ref)
+        assert np.array_equal(xsum.cpu().numpy(), s_ref)
+
+
 @pytest.mark.parametrize("N,K", [(1, 2560), (7, 1024), (64, 4096), (300, 6912), (2, 131072)])
 def test_quant_act_per_tensor_parity(N, K):
     x = inputs.activations(N, K, seed=N * 5 + K, outlier_frac=0.01)
@@ -196,6 +221,17 @@ def test_gemv_parity_tile_kernel_many_units(M, K, N):
     # token count (148 SMs x at most 3 CTAs x 4 warps), so these launches take
     # it rather than the split-unit kernel that the smaller cases here take.
     ref, (packed, alpha, xq, amax, xsum) = _layer(M, K, N, seed=M + K + N)
+    y, acc = api.gemv(packed, alpha, xq, amax, xsum, with_acc=True)
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert np.array_equal(y.cpu().numpy(), ref["y"])
+
+
+@pytest.mark.parametrize("M,K", [(57600, 256), (113696, 128)])
+def test_gemv_parity_split_kernel_just_over_capacity(M, K):
+    # 1800 and 3553 units at N = 1, a little over one and two times the 1776
+    # warps gemv_tile_kernel can have resident: the tile kernel would idle
+    # about half and a third of them, so these take the split-unit kernel
+    ref, (packed, alpha, xq, amax, xsum) = _layer(M, K, 1, seed=M + K)
     y, acc = api.gemv(packed, alpha, xq, amax, xsum, with_acc=True)
     assert np.array_equal(acc.cpu().numpy(), ref["acc"])
     assert np.array_equal(y.cpu().numpy(), ref["y"])
