@@ -171,9 +171,11 @@ BITLINEAR_API bitlinear_status bitlinear_quant_act_grouped(const bitlinear_act* 
  *   acc  int32 [N,M] output of the raw accumulators, or NULL
  * N > 16 returns BITLINEAR_ERR_UNSUPPORTED_SHAPE.
  * Two kernels give the same results.  A launch with at least as many 32-row
- * units as the GPU has resident warps streams them with one warp per unit.
- * A smaller launch takes one 4-warp CTA per unit, whose warps split the unit's
- * k-chunks and add their int32 sums at the end.
+ * units as the GPU has resident warps streams them with one warp per run of
+ * units.  A smaller launch, or one where whole runs of units per warp would
+ * leave more than a quarter of the resident warps idle, takes one 4-warp CTA
+ * per unit, whose warps split the unit's k-chunks and add their int32 sums at
+ * the end.
  */
 BITLINEAR_API bitlinear_status bitlinear_gemv(const uint32_t* packed, const float* alpha,
                                 int64_t M, int64_t K,
@@ -250,7 +252,7 @@ BITLINEAR_API bitlinear_status bitlinear_gemm_grouped(const bitlinear_problem* p
  *   x    fp32 [N,K] activations, 16-byte aligned, row stride K
  *   y    fp32 [N,M] output, bit-identical to quant_act followed by gemv
  *   acc  int32 [N,M] raw accumulators, or NULL
- * 1 <= N <= 16, and N * 512 * ceil(K/512) <= 65536 (the int8 copy each warp
+ * 1 <= N <= 16, and N * 512 * ceil(K/512) <= 65536 (the int8 copy each CTA
  * keeps in shared memory): N = 1 takes K up to 65536, N = 16 up to 4096.
  * Larger cases return BITLINEAR_ERR_UNSUPPORTED_SHAPE; quantise with
  * bitlinear_quant_act and call bitlinear_gemv for them.
@@ -278,7 +280,7 @@ typedef struct {
 
 /*
  * bitlinear_gemv_quant over a list of layers, one launch per 256 layers.
- * Each warp quantises an input once for the run of rows it owns, so layers
+ * Each CTA quantises an input once for the run of rows it owns, so layers
  * that read the same activations (q, k and v; gate and up) should carry the
  * same x pointer and sit next to each other in the list.  `problems` is a HOST
  * array read during the call only.  The shared-memory limit above applies to
