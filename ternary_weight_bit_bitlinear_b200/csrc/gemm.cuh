@@ -166,8 +166,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Smem = GemmSmem<BN, STAGES>;
-  pdl_wait_prior_grid();
-  pdl_allow_next_grid();
   const uint32_t base = smem_u32(smem_raw);
   Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
 
@@ -205,6 +203,10 @@ gemm_i8_tcgen05_kernel(const __grid_constant__ GemmParams p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The set-up above (barriers, tensor-map prefetch, tensor memory) touches
+  // nothing the preceding kernel writes, so it overlaps that kernel's tail.
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
   const uint32_t tmem_base = s.tmem_slot;
 
   if (warp == 0) {

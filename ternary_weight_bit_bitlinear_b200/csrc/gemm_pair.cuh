@@ -64,8 +64,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   using Smem = GemmPairSmem<STAGES>;
-  pdl_wait_prior_grid();
-  pdl_allow_next_grid();
   const uint32_t base = smem_u32(smem_raw);
   Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
 
@@ -108,6 +106,10 @@ gemm_i8_pair_kernel(const __grid_constant__ GemmParams p) {
   tc_fence_before();
   cluster_sync();   // both CTAs' barriers exist before either CTA touches the other's
   tc_fence_after();
+  // The set-up above (barriers, tensor-map prefetch, tensor memory) touches
+  // nothing the preceding kernel writes, so it overlaps that kernel's tail.
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
   const uint32_t tmem_base = s.tmem_slot;
   const int ntiles = gemm_my_count(p, pair, npairs);
 

@@ -106,8 +106,6 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
   constexpr int S = Smem::S;
   constexpr int kSlots = small_aslots(BN);
   constexpr uint32_t kAColBase = small_acol_base(BN);
-  pdl_wait_prior_grid();
-  pdl_allow_next_grid();
   const uint32_t base = smem_u32(smem_raw);
   Smem& s = *reinterpret_cast<Smem*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
 
@@ -143,6 +141,10 @@ gemm_small_kernel(const __grid_constant__ GemmParams p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The set-up above (barriers, tensor-map prefetch, tensor memory) touches
+  // nothing the preceding kernel writes, so it overlaps that kernel's tail.
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
   const uint32_t tmem_base = s.tmem_slot;
   const int ntiles = gemm_my_count(p);
 
