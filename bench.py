@@ -68,7 +68,7 @@ NCU_TRAFFIC = {
              "source": "ncu dram__bytes_read+write, gemv_tile_kernel<1>, 2B stream launch"},
     "gemm": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemm.cuh",
                       "ternary_weight_bit_bitlinear_b200/csrc/gemm_pair.cuh"],
-             "sha256": "b73069191af7c054", "bytes": 62_601_216 + 31_635_200,
+             "sha256": "dc825d0a324fa159", "bytes": 62_600_960 + 31_451_648,
              "source": "ncu dram__bytes_read+write, gemm_i8_pair_kernel<5>, 7B prefill N=512"},
     # captured on a 4-layer launch of the 70B stream (DRAM reads 1.003 x the
     # packed bytes, so traffic grows with the layers), x5 to the headline's
