@@ -76,7 +76,7 @@ NCU_TRAFFIC = {
     "gemv_quant": {"file": ["ternary_weight_bit_bitlinear_b200/csrc/gemv_quant.cuh",
                             "ternary_weight_bit_bitlinear_b200/csrc/gemv.cuh",
                             "ternary_weight_bit_bitlinear_b200/csrc/quant_math.cuh"],
-                   "sha256": "0c47ba719c21d7ae", "bytes": (858_458_112 + 6_199_552) * 5,
+                   "sha256": "0c47ba719c21d7ae", "bytes": (859_360_000 + 4_622_336) * 5,
                    "source": "ncu dram__bytes_read+write, gemv_quant_kernel<1>, 4-layer launch of "
                              "the 70B stream, scaled x5 to the 20-layer launch"},
 }

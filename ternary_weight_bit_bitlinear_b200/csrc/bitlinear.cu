@@ -348,7 +348,11 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
   p.xstride = static_cast<int>((kmax + bl::kGemvChunkK - 1) / bl::kGemvChunkK * bl::kGemvChunkK);
   // CTA size: the most warps resident per SM, among sizes that fit at least
   // two CTAs per SM when there are any (a CTA that starts on an SM quantises
-  // its input while the other one streams weights); fewest warps on a tie.
+  // its input while the other one streams weights); on a tie, the most warps
+  // per CTA (fewer CTAs quantise each input, and each CTA's range is longer).
+  // The 70B-shaped stream then runs 2 CTAs of 6 warps per SM rather than 3 of
+  // 4 (6635-6644 against 6624 GB/s; the 2B-shaped stream 5617-5633 against
+  // 5570-5590, on one box).
   int best_w = 0, best_per_sm = 0, best_score = 0;
   for (int w = 4; w <= bl::gq_max_warps(nt); ++w) {
     int per_sm = 0;
@@ -356,7 +360,7 @@ bitlinear_status gemv_quant_plan(const bitlinear_fused_problem* probs, int n, in
         blh::gemv_quant_occupancy(nt, w, bl::gq_smem_bytes(nt, w, p.xstride), dev, &per_sm);
     if (st != BITLINEAR_OK) return st;
     const int score = per_sm * w + (per_sm >= 2 ? 1000 : 0);
-    if (per_sm > 0 && score > best_score) {
+    if (per_sm > 0 && score >= best_score) {
       best_score = score;
       best_w = w;
       best_per_sm = per_sm;
