@@ -14,9 +14,9 @@ GEMV_MAX_TOKENS = 16
 
 # Smallest token count for which `matmul` and `TernaryLinear` use the
 # tensor-core GEMM.  Measured on B200 on an 8B-shaped layer (7 projections,
-# one grouped launch, weights not in L2): GEMV 24.6 / 38.5 / 57.5 / 54.9 /
-# 186 us and GEMM 24.3 / 24.2 / 24.5 / 24.5 / 24.5 us at N = 1 / 2 / 4 / 8 /
-# 16; from fp32 activations, the fused quantise+GEMV 29.6 / 38.9 us at N = 1 /
+# one grouped launch, weights not in L2): GEMV 24.6 / 30.1 / 40.8 / 54.9 /
+# 104 us and GEMM 24.5 / 24.6 / 24.6 / 24.3 / 24.3 us at N = 1 / 2 / 4 / 8 /
+# 16; from fp32 activations, the fused quantise+GEMV 26.8 / 38.4 us at N = 1 /
 # 2.  The two tie at one token; from two on, the GEMV's per-token dp4a work
 # costs more than the GEMM's whole launch.
 GEMM_MIN_TOKENS = 2
